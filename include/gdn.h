@@ -1,0 +1,137 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the B200 (sm_100a) Gated DeltaNet (GDN) token mixer.
+ *
+ * The mixer (defined in the "Qwen3.8-Flash-Next" technical report, Fig. 2, and the
+ * "Qwen3-Next 80B-A3B" field guide, §02 "Gated DeltaNet state update"):
+ *   1. width-4 depthwise causal conv over the q, k and v streams, then SiLU;
+ *   2. L2 normalisation of q and k per head;
+ *   3. decay gate g = -exp(A_log) * softplus(a + dt_bias) (the decay-gate note of the
+ *      "Qwen3.8-Flash-Next" model notes) and write gate beta = sigmoid(b);
+ *   4. the gated delta rule on one d_v x d_k fp32 state per value head (field guide,
+ *      §02, steps 1-6):  S' = e^g S;  e = v - S'k;  S'' = S' + beta e k^T;  y = S'' q;
+ *   5. RMS normalisation of y per value head, times norm_w, gated by SiLU(z).
+ * Value head h reads QK head h / (h_v / h_qk) (16 QK heads shared by 32 value heads in
+ * the pages' model).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or synchronises on the hot path.  Work is enqueued on `stream`
+ *     and runs asynchronously.
+ *   - Tensors are contiguous, row-major, in the layouts given below, with 16-byte aligned
+ *     base pointers.
+ *   - Return value: GDN_OK (0) or a negative GDN_ERR_* code.  Arguments are validated on
+ *     the host before any launch; on an error nothing is launched and no output is
+ *     touched.
+ *   - State layout: S[n][h][i][j], i in [0, d_v) the value component, j in [0, d_k) the
+ *     key component (column-vector convention: S maps a key to a value).
+ *   - Conv weights conv_w[C_conv][4], C_conv = 2*h_qk*d_k + h_v*d_v, channel order
+ *     q (h_qk*d_k) | k (h_qk*d_k) | v (h_v*d_v); tap 3 multiplies the current token,
+ *     tap 0 the token three back.  No conv bias.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gdn_stream_t; /* identical to cudaStream_t */
+
+/* return codes */
+#define GDN_OK 0
+#define GDN_ERR_NULL (-1)           /* a required pointer is NULL */
+#define GDN_ERR_SHAPE (-2)          /* unsupported or inconsistent dimensions */
+#define GDN_ERR_DTYPE (-3)          /* unsupported dtype code */
+#define GDN_ERR_ALIGN (-4)          /* a base pointer is not 16-byte aligned */
+#define GDN_ERR_WORKSPACE (-5)      /* workspace missing or smaller than required */
+#define GDN_ERR_CUDA (-6)           /* a CUDA launch or runtime call failed */
+#define GDN_ERR_DEVICE_TIMEOUT (-7) /* a bounded device-side wait ran out (device status) */
+
+/* dtype codes */
+#define GDN_DTYPE_F32 0
+#define GDN_DTYPE_BF16 1
+
+typedef struct gdn_dims {
+  int32_t n_seqs;       /* N >= 1 sequences */
+  int32_t total_tokens; /* T_tot >= 0 packed tokens (decode: must equal n_seqs) */
+  int32_t h_qk, h_v;    /* QK heads, value heads; h_v % h_qk == 0 */
+  int32_t d_k, d_v;     /* head widths; only 128 x 128 is supported */
+  int32_t in_dtype;     /* GDN_DTYPE_BF16 | GDN_DTYPE_F32: q, k, v, z (and decode conv_state) */
+  int32_t out_dtype;    /* GDN_DTYPE_BF16 | GDN_DTYPE_F32: y */
+  float q_scale;        /* multiplies the normalised query; 1.0 gives the pages' y = S'' q */
+  float l2_eps;         /* q, k L2 norm: x / sqrt(sum x^2 + l2_eps); 1e-6 */
+  float rms_eps;        /* output norm: y / sqrt(mean y^2 + rms_eps); 1e-6 */
+} gdn_dims_t;
+
+/*
+ * Bytes of device workspace gdn_prefill needs for these dimensions (0 if the dims are
+ * invalid).  Depends only on the dims, never on cu_seqlens' contents.
+ */
+size_t gdn_prefill_workspace_size(const gdn_dims_t* d);
+
+/*
+ * Prefill over packed variable-length sequences (the whole mixer, steps 1-5 above).
+ *
+ *   q, k        [T_tot][h_qk][d_k]   in_dtype
+ *   v, z        [T_tot][h_v][d_v]    in_dtype
+ *   a, b        [T_tot][h_v]         fp32 (gate pre-activations)
+ *   A_log, dt_bias [h_v]             fp32
+ *   conv_w      [C_conv][4]          fp32
+ *   norm_w      [d_v]                fp32 (shared by all value heads)
+ *   init_state  [N][h_v][d_v][d_k]   fp32, or NULL for zero initial states
+ *   cu_seqlens  [N+1]                int32 DEVICE array of sequence offsets
+ *                                    (cu[0] = 0, non-decreasing, cu[N] = T_tot), or NULL
+ *                                    when N == 1 (one sequence of T_tot tokens)
+ *   y           [T_tot][h_v][d_v]    out_dtype (written)
+ *   final_state [N][h_v][d_v][d_k]   fp32 (written); may alias init_state
+ *   workspace   device scratch of at least gdn_prefill_workspace_size(d) bytes
+ *
+ * Each sequence starts with a zero conv history and with its init_state.  Empty
+ * sequences copy init_state (or zeros) to final_state.  T_tot == 0 writes final_state
+ * only.  cu_seqlens' contents are not validated on the host (they stay on the device).
+ */
+int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+                const float* a, const float* b, const float* A_log, const float* dt_bias,
+                const float* conv_w, const float* norm_w, const float* init_state,
+                const int32_t* cu_seqlens, void* y, float* final_state, void* workspace,
+                size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * One decode step: one new token for each of N sequences, on resident state
+ * (field guide, §02: the state size stays fixed as the sequence grows).
+ *
+ *   q, k        [N][h_qk][d_k]       in_dtype
+ *   v, z        [N][h_v][d_v]        in_dtype
+ *   a, b        [N][h_v]             fp32
+ *   A_log, dt_bias, conv_w, norm_w   as in gdn_prefill
+ *   conv_state  [N][3][C_conv]       in_dtype, in/out: raw (pre-conv) x_{t-3}, x_{t-2},
+ *                                    x_{t-1}; replaced by x_{t-2}, x_{t-1}, x_t (bit-exact)
+ *   state       [N][h_v][d_v][d_k]   fp32, in/out, updated in place to S''
+ *   y           [N][h_v][d_v]        out_dtype (written)
+ * d->total_tokens must equal d->n_seqs.
+ */
+int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+               const float* a, const float* b, const float* A_log, const float* dt_bias,
+               const float* conv_w, const float* norm_w, void* conv_state, float* state,
+               void* y, gdn_stream_t stream);
+
+/* Static, NUL-terminated name of a return code ("GDN_OK", "GDN_ERR_SHAPE", ...). */
+const char* gdn_status_string(int code);
+
+/*
+ * Synchronises `stream`, then returns and clears the library's device status word for
+ * the current device: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a bounded device-side wait
+ * gave up since the last read.  Returns GDN_ERR_CUDA if the synchronisation fails.
+ */
+int gdn_read_device_status(gdn_stream_t stream);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_H_ */

@@ -1,0 +1,238 @@
+"""fp64 CPU oracle for the Gated DeltaNet token mixer -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import this package.  The CUDA library never calls it, and it shares no code with
+the CUDA library: the arithmetic lives in ``gdn_oracle.c`` (plain C, fp64), this module
+only marshals numpy arrays through ctypes.
+
+Element encodings: numpy ``float32`` arrays are fp32 inputs, ``uint16`` arrays are raw
+bf16 bits.  Both are widened exactly to fp64 inside the C code.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+# A test may point this at a separately built copy of the oracle (the planted-mistake test).
+_LIB_OVERRIDE = os.environ.get("GDN_ORACLE_LIB")
+_lock = threading.Lock()
+_lib = None
+
+ENC_F32 = 0
+ENC_BF16 = 1
+
+
+class OracleDims(ctypes.Structure):
+    _fields_ = [
+        ("n_seqs", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int32),
+        ("h_qk", ctypes.c_int32),
+        ("h_v", ctypes.c_int32),
+        ("d_k", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+        ("in_enc", ctypes.c_int32),
+        ("q_scale", ctypes.c_double),
+        ("l2_eps", ctypes.c_double),
+        ("rms_eps", ctypes.c_double),
+        ("chunk", ctypes.c_int32),
+        ("n_threads", ctypes.c_int32),
+    ]
+
+
+def build(force: bool = False) -> str:
+    """Compile gdn_oracle.c into liboracle.so (plain -O2, no fast-math, OpenMP threads)."""
+    with _lock:
+        if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+            tmp = _LIB + f".{os.getpid()}.tmp"
+            subprocess.check_call(
+                ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o", tmp, _SRC, "-lm"]
+            )
+            os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if _LIB_OVERRIDE:
+            L = ctypes.CDLL(_LIB_OVERRIDE)
+        else:
+            build()
+            L = ctypes.CDLL(_LIB)
+        d = ctypes.c_double
+        dp = ctypes.POINTER(ctypes.c_double)
+        vp = ctypes.c_void_p
+        for name in ("oracle_softplus", "oracle_sigmoid", "oracle_silu"):
+            f = getattr(L, name)
+            f.restype, f.argtypes = d, [d]
+        L.oracle_decay_gate.restype, L.oracle_decay_gate.argtypes = d, [d, d, d]
+        L.oracle_conv_silu_channel.restype = None
+        L.oracle_conv_silu_channel.argtypes = [vp, ctypes.c_long, ctypes.c_long, vp, vp, vp]
+        L.oracle_l2norm.restype, L.oracle_l2norm.argtypes = None, [vp, ctypes.c_int, d]
+        L.oracle_gated_rmsnorm.restype = None
+        L.oracle_gated_rmsnorm.argtypes = [vp, vp, vp, ctypes.c_int, d, vp]
+        for name in ("oracle_recurrence_token",):
+            f = getattr(L, name)
+            f.restype = None
+            f.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, d, vp, vp]
+        L.oracle_recurrence_chunked.restype = None
+        L.oracle_recurrence_chunked.argtypes = [
+            ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, d, vp, vp]
+        L.oracle_prefill.restype = ctypes.c_int
+        L.oracle_prefill.argtypes = [ctypes.POINTER(OracleDims)] + [vp] * 12 + [
+            ctypes.c_int, ctypes.c_int, vp, vp, vp]
+        L.oracle_decode.restype = ctypes.c_int
+        L.oracle_decode.argtypes = [ctypes.POINTER(OracleDims)] + [vp] * 16
+        _ = dp
+        _lib = L
+    return _lib
+
+
+def _p(x):
+    return None if x is None else ctypes.c_void_p(x.ctypes.data)
+
+
+def _c64(x):
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _enc(x: np.ndarray) -> int:
+    if x.dtype == np.uint16:
+        return ENC_BF16
+    if x.dtype == np.float32:
+        return ENC_F32
+    raise TypeError(f"oracle inputs must be float32 or uint16 (bf16 bits), got {x.dtype}")
+
+
+# ---- scalar and stage functions -------------------------------------------------------
+
+def softplus(x: float) -> float:
+    return lib().oracle_softplus(float(x))
+
+
+def sigmoid(x: float) -> float:
+    return lib().oracle_sigmoid(float(x))
+
+
+def silu(x: float) -> float:
+    return lib().oracle_silu(float(x))
+
+
+def decay_gate(a: float, A_log: float, dt_bias: float) -> float:
+    return lib().oracle_decay_gate(float(a), float(A_log), float(dt_bias))
+
+
+def conv_silu(x: np.ndarray, w: np.ndarray, hist: np.ndarray | None = None) -> np.ndarray:
+    """Width-4 causal conv + SiLU over one channel: x [T], w [4], hist [3] or None."""
+    x = _c64(x)
+    out = np.empty_like(x)
+    w = _c64(w)
+    h = None if hist is None else _c64(hist)
+    lib().oracle_conv_silu_channel(_p(x), 1, x.shape[0], _p(w), _p(h), _p(out))
+    return out
+
+
+def l2norm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    x = _c64(x).copy()
+    lib().oracle_l2norm(_p(x), x.shape[0], eps)
+    return x
+
+
+def gated_rmsnorm(y_raw, z, norm_w, eps: float = 1e-6) -> np.ndarray:
+    y_raw, z, norm_w = _c64(y_raw), _c64(z), _c64(norm_w)
+    out = np.empty_like(y_raw)
+    lib().oracle_gated_rmsnorm(_p(y_raw), _p(z), _p(norm_w), y_raw.shape[0], eps, _p(out))
+    return out
+
+
+def recurrence(qh, kh, v, g, beta, S0, q_scale: float = 1.0, chunk: int = 0):
+    """Recurrence core of one (sequence, value head) on convolved, normalised streams.
+
+    qh, kh [T, d_k]; v [T, d_v]; g, beta [T]; S0 [d_v, d_k].  chunk = 0 runs the per-token
+    rule; chunk > 0 runs the chunked rewrite.  Returns (y_raw [T, d_v], S_final).
+    """
+    qh, kh, v, g, beta = map(_c64, (qh, kh, v, g, beta))
+    S = _c64(S0).copy()
+    T, dk = kh.shape
+    dv = v.shape[1]
+    y = np.zeros((T, dv), np.float64)
+    if chunk:
+        lib().oracle_recurrence_chunked(T, dk, dv, chunk, _p(qh), _p(kh), _p(v), _p(g), _p(beta),
+                                        q_scale, _p(S), _p(y))
+    else:
+        lib().oracle_recurrence_token(T, dk, dv, _p(qh), _p(kh), _p(v), _p(g), _p(beta), q_scale,
+                                      _p(S), _p(y))
+    return y, S
+
+
+# ---- whole mixer ----------------------------------------------------------------------
+
+def _dims(n_seqs, total, h_qk, h_v, d_k, d_v, enc, q_scale, l2_eps, rms_eps, chunk, threads):
+    return OracleDims(n_seqs, total, h_qk, h_v, d_k, d_v, enc, q_scale, l2_eps, rms_eps, chunk,
+                      threads)
+
+
+def prefill(inp: dict, heads: tuple[int, int] | None = None, chunk: int = 0, n_threads: int = 0,
+            q_scale: float = 1.0, l2_eps: float = 1e-6, rms_eps: float = 1e-6,
+            want_state: bool = True, want_y_raw: bool = False):
+    """Run the oracle prefill on an input dict (see gated_deltanet_token_b200.inputs).
+
+    Returns dict(y=[T,h_v,d_v] f64, final_state=[N,h_v,d_v,d_k] f64 or None, y_raw=...).
+    Only value heads in ``heads`` = (h0, h1) are computed; other entries stay zero.
+    """
+    q, k, v, z = (np.ascontiguousarray(inp[n]) for n in ("q", "k", "v", "z"))
+    enc = _enc(q)
+    T, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    cu = inp.get("cu_seqlens")
+    n_seqs = 1 if cu is None else len(cu) - 1
+    cu32 = None if cu is None else np.ascontiguousarray(cu, dtype=np.int32)
+    h0, h1 = heads if heads is not None else (0, h_v)
+    f32 = lambda n: np.ascontiguousarray(inp[n], dtype=np.float32)  # noqa: E731
+    init = inp.get("init_state")
+    init = None if init is None else np.ascontiguousarray(init, dtype=np.float32)
+    y = np.zeros((T, h_v, d_v), np.float64)
+    y_raw = np.zeros((T, h_v, d_v), np.float64) if want_y_raw else None
+    fs = np.zeros((n_seqs, h_v, d_v, d_k), np.float64) if want_state else None
+    dims = _dims(n_seqs, T, h_qk, h_v, d_k, d_v, enc, q_scale, l2_eps, rms_eps, chunk, n_threads)
+    a, b, A_log, dt_bias, conv_w, norm_w = (f32(n) for n in ("a", "b", "A_log", "dt_bias", "conv_w",
+                                                            "norm_w"))
+    rc = lib().oracle_prefill(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(z), _p(a), _p(b),
+                              _p(A_log), _p(dt_bias), _p(conv_w), _p(norm_w), _p(init), _p(cu32),
+                              h0, h1, _p(y), _p(y_raw), _p(fs))
+    if rc != 0:
+        raise ValueError("oracle_prefill rejected its arguments")
+    return {"y": y, "final_state": fs, "y_raw": y_raw}
+
+
+def decode(inp: dict, n_threads: int = 0, q_scale: float = 1.0, l2_eps: float = 1e-6,
+           rms_eps: float = 1e-6, want_state: bool = True):
+    """Oracle decode step.  Returns dict(y, y_raw, state, conv_state) in fp64."""
+    q, k, v, z = (np.ascontiguousarray(inp[n]) for n in ("q", "k", "v", "z"))
+    enc = _enc(q)
+    N, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    f32 = lambda n: np.ascontiguousarray(inp[n], dtype=np.float32)  # noqa: E731
+    a, b, A_log, dt_bias, conv_w, norm_w, state = (
+        f32(n) for n in ("a", "b", "A_log", "dt_bias", "conv_w", "norm_w", "state"))
+    cs = np.ascontiguousarray(inp["conv_state"])
+    if _enc(cs) != enc:
+        raise TypeError("conv_state must use the same encoding as q, k, v, z")
+    y = np.zeros((N, h_v, d_v), np.float64)
+    y_raw = np.zeros((N, h_v, d_v), np.float64)
+    st = np.zeros((N, h_v, d_v, d_k), np.float64) if want_state else None
+    cso = np.zeros(cs.shape, np.float64)
+    dims = _dims(N, N, h_qk, h_v, d_k, d_v, enc, q_scale, l2_eps, rms_eps, 0, n_threads)
+    rc = lib().oracle_decode(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(z), _p(a), _p(b),
+                             _p(A_log), _p(dt_bias), _p(conv_w), _p(norm_w), _p(cs), _p(state),
+                             _p(y), _p(y_raw), _p(st), _p(cso))
+    if rc != 0:
+        raise ValueError("oracle_decode rejected its arguments")
+    return {"y": y, "y_raw": y_raw, "state": st, "conv_state": cso}
