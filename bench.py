@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the GDN token-mixer hot path on B200 (one JSON line on rank 0).
+
+A step is one gdn_prefill over the model-shaped workload (one sequence of T = 4096 tokens,
+16 QK / 32 value heads, d = 128, bf16 q/k/v/z, fp32 gates and state): conv + SiLU + L2 norm
++ gates, the chunked gated delta rule, the gated RMSNorm, the final state.  `value` is the
+whole-job prefill throughput in Mtok/s (max device time over ranks).  The decode step
+(256 sequences x 1 token on 512 MiB of resident fp32 state) is timed in the same run and
+reported under "decode" as state GB/s against the measured HBM copy bandwidth.
+
+Timing: W untimed warm-up steps, then K steps between a barrier + cuda synchronize on both
+sides, timed with CUDA events on the launching stream.  Inputs rotate over three device
+copies (3 x 97 MiB > 126 MB L2) so no step starts with its inputs in L2.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Multi-GPU: launched with torch.distributed.run, one rank per GPU; every rank runs its own
+full workload (weak scaling, no data-path collective: the mixer shards by sequence/head).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill Mtok/s (T=4096, 32 V heads); decode state GB/s vs HBM peak"
+WORKLOAD = "prefill_T4096_bf16"
+DECODE_WORKLOAD = "decode_N256_bf16"
+HBM_FALLBACK_GBS = 6650.0
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+# Algorithmic work per (token, value head) of each kernel at d = 128, chunk 64 (16 QK heads
+# shared by 32 value heads; Q K^T and K K^T are counted once per QK head).
+D, C = 128, 64
+FLOP_PHASEA_PER_TOKEN = 16 * (2 * 2 * C * D) + 32 * (2 * 2 * C * D)      # K K^T, Q K^T; W, U'
+FLOP_PHASEB_PER_TOKEN = 32 * (3 * 2 * D * D + 2 * C * D)                  # W S^T, Q S^T, U^T K, (MoQK^T) U
+BYTES_PER_TOKEN_IO = 2 * (16 * D * 2) + 2 * (32 * D * 2) + 2 * 32 * 4 + 32 * D * 2  # q,k,v,z,a,b in; y out
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    p.add_argument("--decode-steps", type=int, default=None)
+    return p.parse_args(argv)
+
+
+# ---- host-side helpers (also exercised by the CPU multi-process tests) -------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def shard_units(n_units: int, rank: int, world: int) -> range:
+    """Contiguous, balanced share of n_units independent work units (sequences or QK-head
+    groups) for `rank`; shares differ by at most one unit and cover every unit once."""
+    base, extra = divmod(n_units, world)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_token_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    kernel sources changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("src_sha") != source_sha():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---- the timed oracle (CPU baseline and the reference arm) ---------------------------------
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(target_s: float):
+    """Time the fp64 oracle on a prefix of the bench workload (all 32 value heads), sized
+    to take about target_s seconds.  Returns (tokens/s, tokens, seconds, threads)."""
+    import oracle
+    from gated_deltanet_token_b200.inputs import make_inputs
+
+    cores = cpu_cores()
+    full = make_inputs(WORKLOAD)
+
+    def run(T):
+        inp = dict(full)
+        for n in ("q", "k", "v", "z", "a", "b"):
+            inp[n] = full[n][:T]
+        t0 = time.perf_counter()
+        oracle.prefill(inp, n_threads=cores, want_state=True)
+        return time.perf_counter() - t0
+
+    t_probe = run(64)
+    per_tok = t_probe / 64
+    T = int(min(4096, max(64, target_s / max(per_tok, 1e-9))))
+    dt = run(T)
+    return T / dt, T, dt, cores
+
+
+def reference_arm(args):
+    """`--impl reference`: the oracle, as it stands, on the host cores; each step a bounded
+    sample (a token prefix of the same workload)."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    import oracle
+    from gated_deltanet_token_b200.inputs import make_inputs
+
+    oracle.build()
+    cores = cpu_cores()
+    full = make_inputs(WORKLOAD)
+
+    def step(T):
+        inp = dict(full)
+        for n in ("q", "k", "v", "z", "a", "b"):
+            inp[n] = full[n][:T]
+        t0 = time.perf_counter()
+        oracle.prefill(inp, n_threads=cores)
+        return time.perf_counter() - t0
+
+    per_tok = step(32) / 32
+    T = int(min(4096, max(8, budget / max(per_tok, 1e-9))))
+    for _ in range(args.warmup):
+        step(T)
+    times = [step(T) for _ in range(args.steps)]
+    total = sum(times)
+    value = T * args.steps / total / 1e6
+    sample = f"first {T} of 4096 tokens, all 32 value heads, per step"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "B": 1, "T": 4096, "h_qk": 16, "h_v": 32,
+                                        "d": 128, "sample_tokens": T},
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---- the GPU arm ------------------------------------------------------------------------------
+
+def to_dev(x, device):
+    import numpy as np
+    import torch
+
+    if x is None:
+        return None
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if x.dtype == np.uint16:
+        t = t.view(torch.bfloat16)
+    return t.to(device)
+
+
+def gpu_arm(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from gated_deltanet_token_b200 import gdn
+    from gated_deltanet_token_b200.inputs import make_inputs
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+
+    # --- prefill workload: every rank runs its own copy (weak scaling) -----------------------
+    inp = make_inputs(WORKLOAD, seed=rank)
+    names = ("q", "k", "v", "z", "a", "b")
+    params = {n: to_dev(inp[n], dev) for n in ("A_log", "dt_bias", "conv_w", "norm_w")}
+    n_sets = 3
+    sets = [{n: to_dev(inp[n], dev) for n in names} for _ in range(n_sets)]
+    T = inp["spec"]["T"]
+    y = torch.empty((T, 32, 128), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, 32, 128, 128), dtype=torch.float32, device=dev)
+    dims = gdn.make_dims(1, T, 16, 32, gdn.GDN_DTYPE_BF16, gdn.GDN_DTYPE_BF16)
+    ws = torch.empty(gdn.gdn_prefill_workspace_size(dims), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        s = sets[i % n_sets]
+        gdn.gdn_prefill(s["q"], s["k"], s["v"], s["z"], s["a"], s["b"], params["A_log"],
+                        params["dt_bias"], params["conv_w"], params["norm_w"], None, None,
+                        out_dtype=torch.bfloat16, y=y, final_state=fs, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.2)
+    gdn.gdn_profile_enable(True)
+    gdn.gdn_profile_read()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    prof = gdn.gdn_profile_read()
+    gdn.gdn_profile_enable(False)
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local, dev)
+    ms_per_step = ms / args.steps
+    tokens_all = sum_over_ranks(float(T * args.steps), dev)
+    value = tokens_all / (ms / 1e3) / 1e6
+    launches = sum(v[0] for v in prof.values())
+
+    # --- roofline of the dominant kernel ------------------------------------------------------
+    dom = max(prof.items(), key=lambda kv: kv[1][1])
+    dom_name, (dom_n, dom_ms) = dom
+    dom_avg_s = dom_ms / dom_n / 1e3
+    if dom_name.startswith("chunk_phaseB"):
+        work, unit_kind = FLOP_PHASEB_PER_TOKEN * T, "flop"
+    elif dom_name.startswith("chunk_phaseA"):
+        work, unit_kind = FLOP_PHASEA_PER_TOKEN * T, "flop"
+    else:
+        work, unit_kind = None, None
+    if unit_kind == "flop" and "simt" in dom_name:
+        peak_tflops = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+        roof = {"kernel": dom_name, "bound": "alu", "achieved": work / dom_avg_s / 1e12,
+                "peak": peak_tflops, "unit": "TFLOP/s",
+                "peak_source": f"derived: {SM_COUNT} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x {sm_max:.0f} MHz"}
+    elif unit_kind == "flop":
+        pk = float(peaks["bf16_tflops"])
+        roof = {"kernel": dom_name, "bound": "tensor", "achieved": work / dom_avg_s / 1e12, "peak": pk,
+                "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops"}
+    else:
+        roof = {"kernel": dom_name, "bound": "hbm", "achieved": BYTES_PER_TOKEN_IO * T / dom_avg_s / 1e9,
+                "peak": hbm, "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(dom_name)
+    roof["avg_launch_us"] = dom_avg_s * 1e6
+    roof["kernels"] = {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3,
+                           "share": v[1] / sum(x[1] for x in prof.values())} for k, v in prof.items()}
+
+    # --- decode: 256 sequences x 1 token, resident fp32 state read and written in place --------
+    dinp = make_inputs(DECODE_WORKLOAD, seed=rank)
+    dd = {n: to_dev(dinp[n], dev) for n in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w",
+                                            "norm_w", "conv_state", "state")}
+    yd = torch.empty((256, 32, 128), dtype=torch.bfloat16, device=dev)
+    del dinp
+
+    def dstep():
+        gdn.gdn_decode(dd["q"], dd["k"], dd["v"], dd["z"], dd["a"], dd["b"], dd["A_log"], dd["dt_bias"],
+                       dd["conv_w"], dd["norm_w"], dd["conv_state"], dd["state"],
+                       out_dtype=torch.bfloat16, y=yd)
+
+    dsteps = args.decode_steps or max(args.steps, 20)
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(dsteps):
+        dstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    dms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
+    clk = clocks.stop()
+    state_bytes = 256 * 32 * 128 * 128 * 4 * 2
+    other = 256 * (2 * 16 * 128 * 2 + 2 * 32 * 128 * 2 + 2 * 32 * 4 + 32 * 128 * 2 + 2 * 3 * 8192 * 2)
+    decode = {"workload": DECODE_WORKLOAD, "ms_per_step": dms,
+              "state_GBps": state_bytes / (dms / 1e3) / 1e9,
+              "total_GBps": (state_bytes + other) / (dms / 1e3) / 1e9,
+              "peak_GBps": hbm, "frac_state": state_bytes / (dms / 1e3) / 1e9 / hbm,
+              "tokens_per_s": 256 / (dms / 1e3), "traffic": ncu_traffic("decode")}
+    del dd
+
+    # --- end to end through the public call with host buffers ----------------------------------
+    host = {n: to_dev(inp[n], "cpu").pin_memory() for n in names}
+    dbuf = {n: torch.empty_like(host[n], device=dev) for n in names}
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    fs_host = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = y.numel() * y.element_size() + fs.numel() * fs.element_size()
+
+    def e2e_step():
+        for n in names:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        gdn.gdn_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["z"], dbuf["a"], dbuf["b"], params["A_log"],
+                        params["dt_bias"], params["conv_w"], params["norm_w"], None, None,
+                        out_dtype=torch.bfloat16, y=y, final_state=fs, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+        fs_host.copy_(fs, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_val = sum_over_ranks(float(T * e2e_steps), dev) / (e2e_ms / 1e3) / 1e6
+
+    # --- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only ---------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, Ts, secs, cores = oracle_sample(12.0)
+        cpu = {"value": tps / 1e6, "unit": "Mtok/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {Ts} tokens of the T=4096 workload, all 32 value heads, {secs:.1f} s"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    out = {
+        "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": 1, "T": T, "h_qk": 16, "h_v": 32, "d": 128, "chunk": 64,
+                   "in_dtype": "bf16", "out_dtype": "bf16", "state_dtype": "f32",
+                   "l2": f"{n_sets} rotating input sets of 97 MiB (> 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches, "clocks": clk, "decode": decode,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference_arm(args)
+    return gpu_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,310 @@
+// gdn_api.cu -- host side of libgdn.so: argument validation, workspace layout and the
+// launch sequence of the prefill and decode paths.  Declarations and the contract of each
+// entry point are in include/gdn.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <type_traits>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+#include "k_chunk_simt.cuh"
+#include "k_decode.cuh"
+#include "k_stream.cuh"
+
+using namespace gdn;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of the prefill, carved from the caller's buffer in this order.
+struct WsLayout {
+  size_t tab, seqc0, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
+  int max_chunks;
+};
+
+WsLayout ws_layout(const gdn_dims_t* d) {
+  WsLayout L{};
+  const size_t T = (size_t)d->total_tokens, hq = (size_t)d->h_qk, hv = (size_t)d->h_v;
+  const size_t N = (size_t)d->n_seqs;
+  // every sequence contributes ceil(len / 64) <= len / 64 + 1 chunks
+  L.max_chunks = (int)((T + CH - 1) / CH + N);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.tab = take((size_t)L.max_chunks * sizeof(ChunkEntry));
+  L.seqc0 = take((N + 1) * sizeof(int));
+  L.qn = take(T * hq * D * 4);
+  L.kn = take(T * hq * D * 4);
+  L.vc = take(T * hv * D * 4);
+  L.g = take(T * hv * 4);
+  L.beta = take(T * hv * 4);
+  L.gam = take(T * hv * 4);
+  L.W = take(T * hv * D * 4);
+  L.Up = take(T * hv * D * 4);
+  L.mqk = take(T * hv * CH * 4);
+  L.yraw = take(T * hv * D * 4);
+  L.total = off;
+  return L;
+}
+
+// ---- optional per-kernel event timing (gdn_profile_enable / gdn_profile_read) ----------
+constexpr int kProfMax = 8192;
+struct Prof {
+  bool on = false;
+  bool created = false;
+  int n = 0;
+  cudaEvent_t ev[2 * kProfMax];
+  const char* name[kProfMax];
+};
+Prof g_prof;
+
+int prof_begin(const char* name, cudaStream_t s) {
+  if (!g_prof.on || g_prof.n >= kProfMax) return -1;
+  const int i = g_prof.n++;
+  g_prof.name[i] = name;
+  cudaEventRecord(g_prof.ev[2 * i], s);
+  return i;
+}
+void prof_end(int i, cudaStream_t s) {
+  if (i >= 0) cudaEventRecord(g_prof.ev[2 * i + 1], s);
+}
+struct ProfScope {
+  int i;
+  cudaStream_t s;
+  ProfScope(const char* name, cudaStream_t st) : i(prof_begin(name, st)), s(st) {}
+  ~ProfScope() { prof_end(i, s); }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const gdn_dims_t* d, bool decode) {
+  if (!d) return GDN_ERR_NULL;
+  if (d->n_seqs < 1 || d->total_tokens < 0 || d->h_qk < 1 || d->h_v < 1) return GDN_ERR_SHAPE;
+  if (d->h_v % d->h_qk != 0 || d->h_v / d->h_qk > 8) return GDN_ERR_SHAPE;
+  if (d->d_k != D || d->d_v != D) return GDN_ERR_SHAPE;
+  if (2 * d->h_qk + d->h_v > 65535 || d->h_v > 65535) return GDN_ERR_SHAPE;
+  if (decode && d->total_tokens != d->n_seqs) return GDN_ERR_SHAPE;
+  if ((int64_t)d->total_tokens / CH + d->n_seqs + 1 > INT32_MAX) return GDN_ERR_SHAPE;
+  if (!isfinite(d->q_scale) || !(d->l2_eps >= 0.0f) || !(d->rms_eps >= 0.0f)) return GDN_ERR_SHAPE;
+  if ((d->in_dtype != GDN_DTYPE_F32 && d->in_dtype != GDN_DTYPE_BF16) ||
+      (d->out_dtype != GDN_DTYPE_F32 && d->out_dtype != GDN_DTYPE_BF16))
+    return GDN_ERR_DTYPE;
+  return GDN_OK;
+}
+
+Dims kdims(const gdn_dims_t* d) {
+  Dims k;
+  k.n_seqs = d->n_seqs;
+  k.total_tokens = d->total_tokens;
+  k.h_qk = d->h_qk;
+  k.h_v = d->h_v;
+  k.in_bf16 = d->in_dtype == GDN_DTYPE_BF16;
+  k.out_bf16 = d->out_dtype == GDN_DTYPE_BF16;
+  k.q_scale = d->q_scale;
+  k.l2_eps = d->l2_eps;
+  k.rms_eps = d->rms_eps;
+  return k;
+}
+
+// Opt the large-shared-memory kernels in once per device.
+int configure_device() {
+  static std::atomic<uint64_t> done_mask{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_mask.load() & bit) return GDN_OK;
+  if (cudaFuncSetAttribute(k_phaseA_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(k_phaseB_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PB_SMEM) !=
+          cudaSuccess)
+    return GDN_ERR_CUDA;
+  done_mask.fetch_or(bit);
+  return GDN_OK;
+}
+
+template <bool IN_BF16>
+void launch_prologue(const Dims& kd, int max_chunks, const ChunkEntry* tab, const void* q,
+                     const void* k, const void* v, const float* a, const float* b,
+                     const float* A_log, const float* dt_bias, const float* conv_w, float* qn,
+                     float* kn, float* vc, float* g, float* beta, cudaStream_t s) {
+  dim3 grid(max_chunks, 2 * kd.h_qk + kd.h_v);
+  k_prologue<IN_BF16><<<grid, 256, 0, s>>>(kd, tab, q, k, v, a, b, A_log, dt_bias, conv_w, qn, kn,
+                                           vc, g, beta);
+}
+
+void launch_epilogue(const Dims& kd, const float* yraw, const void* z, const float* norm_w, void* y,
+                     cudaStream_t s) {
+  const long rows = (long)kd.total_tokens * kd.h_v;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  if (kd.in_bf16 && kd.out_bf16) k_epilogue<true, true><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);
+  else if (kd.in_bf16) k_epilogue<true, false><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);
+  else if (kd.out_bf16) k_epilogue<false, true><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);
+  else k_epilogue<false, false><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return kVersion; }
+
+const char* gdn_status_string(int code) {
+  switch (code) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_NULL: return "GDN_ERR_NULL";
+    case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE";
+    case GDN_ERR_DTYPE: return "GDN_ERR_DTYPE";
+    case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT";
+    default: return "GDN_ERR_UNKNOWN";
+  }
+}
+
+size_t gdn_prefill_workspace_size(const gdn_dims_t* d) {
+  if (check_dims(d, false) != GDN_OK) return 0;
+  return ws_layout(d).total;
+}
+
+int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+                const float* a, const float* b, const float* A_log, const float* dt_bias,
+                const float* conv_w, const float* norm_w, const float* init_state,
+                const int32_t* cu_seqlens, void* y, float* final_state, void* workspace,
+                size_t workspace_bytes, gdn_stream_t stream) {
+  int rc = check_dims(d, false);
+  if (rc != GDN_OK) return rc;
+  if (!final_state || !A_log || !dt_bias || !conv_w || !norm_w) return GDN_ERR_NULL;
+  if (d->total_tokens > 0 && (!q || !k || !v || !z || !a || !b || !y)) return GDN_ERR_NULL;
+  if (!cu_seqlens && d->n_seqs != 1) return GDN_ERR_NULL;
+  const void* ptrs[] = {q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, init_state, cu_seqlens,
+                        y, final_state, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+  const WsLayout L = ws_layout(d);
+  if (!workspace || workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+  rc = configure_device();
+  if (rc != GDN_OK) return rc;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  ChunkEntry* tab = reinterpret_cast<ChunkEntry*>(ws + L.tab);
+  int* seqc0 = reinterpret_cast<int*>(ws + L.seqc0);
+  const Dims kd = kdims(d);
+
+  {
+    ProfScope p("tilemap", s);
+    k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0);
+  }
+  if (d->total_tokens > 0) {
+    {
+      ProfScope p("prologue", s);
+      if (kd.in_bf16)
+        launch_prologue<true>(kd, L.max_chunks, tab, q, k, v, a, b, A_log, dt_bias, conv_w, F(L.qn),
+                              F(L.kn), F(L.vc), F(L.g), F(L.beta), s);
+      else
+        launch_prologue<false>(kd, L.max_chunks, tab, q, k, v, a, b, A_log, dt_bias, conv_w, F(L.qn),
+                               F(L.kn), F(L.vc), F(L.g), F(L.beta), s);
+    }
+    ProfScope p("chunk_phaseA_simt", s);
+    k_phaseA_simt<<<dim3(L.max_chunks, d->h_v), 256, PA_SMEM, s>>>(
+        kd, tab, F(L.qn), F(L.kn), F(L.vc), F(L.g), F(L.beta), F(L.gam), F(L.W), F(L.Up), F(L.mqk));
+  }
+  {
+    ProfScope p("chunk_phaseB_simt", s);
+    k_phaseB_simt<<<dim3(d->n_seqs, d->h_v, D / PB_VS), 256, PB_SMEM, s>>>(
+        kd, cu_seqlens, F(L.qn), F(L.kn), F(L.gam), F(L.W), F(L.Up), F(L.mqk), init_state, F(L.yraw),
+        final_state);
+  }
+  if (d->total_tokens > 0) {
+    ProfScope p("epilogue", s);
+    launch_epilogue(kd, F(L.yraw), z, norm_w, y, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+               const float* a, const float* b, const float* A_log, const float* dt_bias,
+               const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+               gdn_stream_t stream) {
+  int rc = check_dims(d, true);
+  if (rc != GDN_OK) return rc;
+  const void* ptrs[] = {q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y};
+  for (const void* p : ptrs)
+    if (!p) return GDN_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  if (d->h_qk > 65535) return GDN_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Dims kd = kdims(d);
+  dim3 grid(d->n_seqs, d->h_qk);
+  ProfScope p("decode", s);
+  if (kd.in_bf16 && kd.out_bf16)
+    k_decode<true, true><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
+                                              conv_state, state, y);
+  else if (kd.in_bf16)
+    k_decode<true, false><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
+                                               conv_state, state, y);
+  else if (kd.out_bf16)
+    k_decode<false, true><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
+                                               conv_state, state, y);
+  else
+    k_decode<false, false><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
+                                                conv_state, state, y);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_profile_enable(int on) {
+  if (on && !g_prof.created) {
+    for (int i = 0; i < 2 * kProfMax; ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return GDN_ERR_CUDA;
+    g_prof.created = true;
+  }
+  g_prof.on = on != 0;
+  return GDN_OK;
+}
+
+int gdn_profile_read(gdn_kernel_time_t* out, int max_entries) {
+  if (!out) return GDN_ERR_NULL;
+  int m = 0;
+  for (int i = 0; i < g_prof.n; ++i) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    int e = 0;
+    while (e < m && strcmp(out[e].name, g_prof.name[i]) != 0) ++e;
+    if (e == m) {
+      if (m == max_entries) continue;
+      out[m].name = g_prof.name[i];
+      out[m].launches = 0;
+      out[m].total_ms = 0.0;
+      ++m;
+    }
+    out[e].launches += 1;
+    out[e].total_ms += ms;
+  }
+  g_prof.n = 0;
+  return m;
+}
+
+int gdn_read_device_status(gdn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gdn_status, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_gdn_status, &zero, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

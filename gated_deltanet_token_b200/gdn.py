@@ -1,0 +1,186 @@
+"""Thin ctypes binding over libgdn.so: the C ABI of include/gdn.h with the same names.
+
+Only argument marshalling happens here: shapes, dtypes and devices of torch tensors are
+checked, outputs and the workspace are allocated with torch when the caller passes none,
+and raw device pointers plus the current CUDA stream go to the library.  Every step of
+the mixer runs in the library's CUDA kernels; there is no CPU or eager fallback.  If the
+library is missing this module raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+GDN_OK = 0
+GDN_DTYPE_F32 = 0
+GDN_DTYPE_BF16 = 1
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where} failed: {gdn_status_string(code)} ({code})")
+
+
+class gdn_dims_t(ctypes.Structure):
+    _fields_ = [
+        ("n_seqs", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int32),
+        ("h_qk", ctypes.c_int32),
+        ("h_v", ctypes.c_int32),
+        ("d_k", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+        ("in_dtype", ctypes.c_int32),
+        ("out_dtype", ctypes.c_int32),
+        ("q_scale", ctypes.c_float),
+        ("l2_eps", ctypes.c_float),
+        ("rms_eps", ctypes.c_float),
+    ]
+
+
+class gdn_kernel_time_t(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn.so (built by __graft_entry__.build() or gated_deltanet_token_b200._build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libgdn.so not found at {_LIB_PATH}: build it first "
+                               "(python -m gated_deltanet_token_b200._build)")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, dp = ctypes.c_void_p, ctypes.POINTER(gdn_dims_t)
+        L.gdn_prefill_workspace_size.restype = ctypes.c_size_t
+        L.gdn_prefill_workspace_size.argtypes = [dp]
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill.argtypes = [dp] + [vp] * 14 + [vp, ctypes.c_size_t, vp]
+        L.gdn_decode.restype = ctypes.c_int
+        L.gdn_decode.argtypes = [dp] + [vp] * 13 + [vp]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_read_device_status.restype = ctypes.c_int
+        L.gdn_read_device_status.argtypes = [vp]
+        L.gdn_profile_enable.restype = ctypes.c_int
+        L.gdn_profile_enable.argtypes = [ctypes.c_int]
+        L.gdn_profile_read.restype = ctypes.c_int
+        L.gdn_profile_read.argtypes = [ctypes.POINTER(gdn_kernel_time_t), ctypes.c_int]
+        L.gdn_version.restype = ctypes.c_int
+        L.gdn_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return GDN_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch tensor")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_dims(n_seqs, total_tokens, h_qk, h_v, in_dtype, out_dtype, d_k=128, d_v=128,
+              q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6) -> gdn_dims_t:
+    return gdn_dims_t(n_seqs, total_tokens, h_qk, h_v, d_k, d_v, in_dtype, out_dtype, q_scale,
+                      l2_eps, rms_eps)
+
+
+def gdn_status_string(code: int) -> str:
+    return lib().gdn_status_string(code).decode()
+
+
+def gdn_version() -> int:
+    return lib().gdn_version()
+
+
+def gdn_read_device_status(stream=None) -> int:
+    return lib().gdn_read_device_status(_stream(stream))
+
+
+def gdn_profile_enable(on: bool) -> None:
+    rc = lib().gdn_profile_enable(int(bool(on)))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_profile_enable")
+
+
+def gdn_profile_read() -> dict:
+    """{kernel name: (launches, total_ms)} since the last read."""
+    buf = (gdn_kernel_time_t * 64)()
+    m = lib().gdn_profile_read(buf, 64)
+    if m < 0:
+        raise GdnError(m, "gdn_profile_read")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(m)}
+
+
+def gdn_prefill_workspace_size(dims: gdn_dims_t) -> int:
+    return lib().gdn_prefill_workspace_size(ctypes.byref(dims))
+
+
+def gdn_prefill(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, init_state=None,
+                cu_seqlens=None, *, out_dtype=None, y=None, final_state=None, workspace=None,
+                q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6, stream=None):
+    """Prefill over packed sequences.  q, k [T, h_qk, 128]; v, z [T, h_v, 128]; a, b [T, h_v];
+    cu_seqlens int32 [N+1] on the device (None = one sequence).  Returns (y, final_state)."""
+    T, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    n = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if out_dtype is None:
+        out_dtype = q.dtype
+    dims = make_dims(n, T, h_qk, h_v, _dt(q), _dt(torch.empty(0, dtype=out_dtype)), d_k, d_v, q_scale,
+                     l2_eps, rms_eps)
+    dev = q.device
+    if y is None:
+        y = torch.empty((T, h_v, d_v), dtype=out_dtype, device=dev)
+    if final_state is None:
+        final_state = torch.empty((n, h_v, d_v, d_k), dtype=torch.float32, device=dev)
+    need = gdn_prefill_workspace_size(dims)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    rc = lib().gdn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(a), _ptr(b),
+                           _ptr(A_log), _ptr(dt_bias), _ptr(conv_w), _ptr(norm_w), _ptr(init_state),
+                           _ptr(cu_seqlens), _ptr(y), _ptr(final_state), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_prefill")
+    return y, final_state
+
+
+def gdn_decode(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, *,
+               out_dtype=None, y=None, q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6, stream=None):
+    """One decode step.  conv_state [N, 3, C_conv] and state [N, h_v, 128, 128] are updated in
+    place.  Returns y [N, h_v, 128]."""
+    N, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    if out_dtype is None:
+        out_dtype = q.dtype
+    dims = make_dims(N, N, h_qk, h_v, _dt(q), _dt(torch.empty(0, dtype=out_dtype)), d_k, d_v, q_scale,
+                     l2_eps, rms_eps)
+    if y is None:
+        y = torch.empty((N, h_v, d_v), dtype=out_dtype, device=q.device)
+    rc = lib().gdn_decode(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(a), _ptr(b),
+                          _ptr(A_log), _ptr(dt_bias), _ptr(conv_w), _ptr(norm_w), _ptr(conv_state),
+                          _ptr(state), _ptr(y), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode")
+    return y

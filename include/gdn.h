@@ -128,6 +128,27 @@ const char* gdn_status_string(int code);
  */
 int gdn_read_device_status(gdn_stream_t stream);
 
+/*
+ * Optional per-kernel timing, for benchmarks.  While enabled, every kernel launch of later
+ * gdn_prefill / gdn_decode calls is bracketed by CUDA events recorded on the call's stream
+ * (the first 8192 launches after the last read are kept; later ones are dropped).  Host state
+ * is process-wide and not thread-safe.  Returns GDN_OK or GDN_ERR_CUDA.
+ */
+int gdn_profile_enable(int on);
+
+typedef struct gdn_kernel_time {
+  const char* name;  /* static kernel name */
+  int launches;      /* launches recorded */
+  double total_ms;   /* summed event-to-event time of those launches */
+} gdn_kernel_time_t;
+
+/*
+ * Waits for the recorded events, sums the time per kernel name into `out` (at most
+ * max_entries entries) and clears the record.  Returns the number of entries written, or
+ * GDN_ERR_NULL / GDN_ERR_CUDA.
+ */
+int gdn_profile_read(gdn_kernel_time_t* out, int max_entries);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gdn_version(void);
 

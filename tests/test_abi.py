@@ -1,0 +1,111 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point that
+include/gdn.h declares, names its status codes, sizes its workspace, and rejects bad
+arguments with the documented codes before any launch (no GPU needed: the pointers
+passed here are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def glib():
+    from gated_deltanet_token_b200 import _build, gdn
+
+    _build.build()
+    return gdn
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(gdn_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(glib):
+    names = declared_functions()
+    assert {"gdn_prefill", "gdn_decode", "gdn_prefill_workspace_size", "gdn_status_string",
+            "gdn_read_device_status"} <= set(names)
+    L = glib.lib()
+    for n in names:
+        assert hasattr(L, n), f"{n} not exported"
+
+
+def test_status_strings(glib):
+    expect = {0: "GDN_OK", -1: "GDN_ERR_NULL", -2: "GDN_ERR_SHAPE", -3: "GDN_ERR_DTYPE",
+              -4: "GDN_ERR_ALIGN", -5: "GDN_ERR_WORKSPACE", -6: "GDN_ERR_CUDA",
+              -7: "GDN_ERR_DEVICE_TIMEOUT"}
+    for c, s in expect.items():
+        assert glib.gdn_status_string(c) == s
+    assert glib.gdn_status_string(-99) == "GDN_ERR_UNKNOWN"
+
+
+def test_workspace_size(glib):
+    d = glib.make_dims(1, 4096, 16, 32, 1, 1)
+    w = glib.gdn_prefill_workspace_size(d)
+    assert w > 0 and w % 256 == 0
+    d2 = glib.make_dims(1, 8192, 16, 32, 1, 1)
+    assert glib.gdn_prefill_workspace_size(d2) > w
+    assert glib.gdn_prefill_workspace_size(glib.make_dims(1, 16, 16, 32, 1, 1, d_k=64)) == 0
+    assert glib.gdn_prefill_workspace_size(glib.make_dims(1, 16, 3, 32, 1, 1)) == 0
+
+
+FAKE = 1 << 20  # 16-byte aligned fake device address, never dereferenced
+
+
+def _prefill(glib, dims, ptrs=None, ws_bytes=1 << 40):
+    p = [FAKE] * 14 if ptrs is None else ptrs
+    P = [ctypes.c_void_p(x) if x else None for x in p]
+    return glib.lib().gdn_prefill(ctypes.byref(dims), *P[:13], P[13], ctypes.c_void_p(FAKE),
+                                  ctypes.c_size_t(ws_bytes), None)
+
+
+def test_prefill_rejects_bad_arguments(glib):
+    ok = glib.make_dims(2, 100, 16, 32, 1, 1)
+    assert glib.lib().gdn_prefill(None, *([None] * 14), None, 0, None) == -1
+    assert _prefill(glib, glib.make_dims(0, 100, 16, 32, 1, 1)) == -2
+    assert _prefill(glib, glib.make_dims(1, -1, 16, 32, 1, 1)) == -2
+    assert _prefill(glib, glib.make_dims(1, 100, 16, 30, 1, 1)) == -2
+    assert _prefill(glib, glib.make_dims(1, 100, 16, 32, 1, 1, d_v=64)) == -2
+    assert _prefill(glib, glib.make_dims(1, 100, 1, 16, 1, 1)) == -2  # more than 8 V heads per QK head
+    assert _prefill(glib, glib.make_dims(1, 100, 16, 32, 2, 1)) == -3
+    assert _prefill(glib, glib.make_dims(1, 100, 16, 32, 1, 7)) == -3
+    ptrs = [FAKE] * 14
+    ptrs[0] = None  # q
+    assert _prefill(glib, ok, ptrs) == -1
+    ptrs = [FAKE] * 14
+    ptrs[11] = None  # cu_seqlens missing with two sequences
+    assert _prefill(glib, ok, ptrs) == -1
+    ptrs = [FAKE] * 14
+    ptrs[3] = FAKE + 4  # misaligned z
+    assert _prefill(glib, ok, ptrs) == -4
+    assert _prefill(glib, ok, ws_bytes=16) == -5
+
+
+def test_decode_rejects_bad_arguments(glib):
+    L = glib.lib()
+
+    def call(dims, ptrs):
+        return L.gdn_decode(ctypes.byref(dims), *[ctypes.c_void_p(x) if x else None for x in ptrs], None)
+
+    good = [FAKE] * 13
+    assert call(glib.make_dims(4, 5, 16, 32, 1, 1), good) == -2  # total_tokens != n_seqs
+    bad = list(good)
+    bad[11] = None
+    assert call(glib.make_dims(4, 4, 16, 32, 1, 1), bad) == -1
+    bad = list(good)
+    bad[10] = FAKE + 8
+    assert call(glib.make_dims(4, 4, 16, 32, 1, 1), bad) == -4
+    assert call(glib.make_dims(4, 4, 16, 32, 5, 1), good) == -3
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from gated_deltanet_token_b200 import gdn
+
+    monkeypatch.setattr(gdn, "_lib", None)
+    monkeypatch.setattr(gdn, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="libgdn.so not found"):
+        gdn.lib()

@@ -1,0 +1,119 @@
+"""GPU parity of gdn_prefill against the fp64 oracle on the same seeded inputs.
+
+Tolerances (fixed for the mixer): fp32 runs e_y = max|y - y_ref| <= 1e-4 and
+e_S = ||S - S_ref||_F / ||S_ref||_F <= 1e-4; bf16-input runs e_y <= 2e-2 RMS(y_ref) and
+e_S <= 1e-2, with half a bf16 ulp of y_ref per element added when y itself is bf16."""
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_token_b200.inputs import make_inputs
+from tests._helpers import check_bf16, check_fp32, run_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle(oracle_mod, inp, heads=None):
+    return oracle_mod.prefill(inp, heads=heads)
+
+
+def test_tiny_prefill_fp32(oracle_mod):
+    inp = make_inputs("tiny_prefill_fp32")
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_fp32(y, ref["y"], S, ref["final_state"])
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 63, 64, 65, 130, 200])
+def test_short_lengths_fp32(oracle_mod, T):
+    inp = make_inputs("tiny_prefill_fp32", T=T)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_fp32(y, ref["y"], S, ref["final_state"])
+
+
+@pytest.mark.parametrize("ratio", [1, 2, 4])
+def test_head_ratios_fp32(oracle_mod, ratio):
+    inp = make_inputs("tiny_prefill_fp32", T=77, h_qk=2, h_v=2 * ratio)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_fp32(y, ref["y"], S, ref["final_state"])
+
+
+def test_q_scale_and_init_state_fp32(oracle_mod):
+    inp = make_inputs("tiny_prefill_fp32", T=90)
+    inp["init_state"] = (np.random.default_rng(5).standard_normal((1, 4, 128, 128)) * 0.02).astype(np.float32)
+    ref = oracle_mod.prefill(inp, q_scale=128 ** -0.5)
+    y, S = run_prefill(inp, torch.float32, q_scale=128 ** -0.5)
+    check_fp32(y, ref["y"], S, ref["final_state"])
+
+
+def test_model_shape_short_bf16(oracle_mod):
+    inp = make_inputs("prefill_T4096_bf16", T=300)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_bf16(y, ref["y"], S, ref["final_state"])
+    yb, Sb = run_prefill(inp, torch.bfloat16)
+    check_bf16(yb, ref["y"], Sb, ref["final_state"], y_is_bf16=True)
+
+
+def test_prefill_T4096_bf16(oracle_mod):
+    inp = make_inputs("prefill_T4096_bf16")
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_bf16(y, ref["y"], S, ref["final_state"])
+    yb, Sb = run_prefill(inp, torch.bfloat16)
+    check_bf16(yb, ref["y"], Sb, ref["final_state"], y_is_bf16=True)
+
+
+def test_varlen_with_empty_sequences_and_alias(oracle_mod):
+    lens = [0, 5, 64, 0, 65, 1, 130, 0]
+    inp = make_inputs("varlen8_prefill_bf16", lengths=lens)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32, init_alias=True)
+    check_bf16(y, ref["y"], S, ref["final_state"])
+    for n, L in enumerate(lens):  # empty sequences copy their initial state exactly
+        if L == 0:
+            assert np.array_equal(S[n], inp["init_state"][n].astype(np.float64))
+
+
+def test_varlen_equals_separate_calls():
+    lens = [37, 100, 64]
+    inp = make_inputs("varlen8_prefill_bf16", lengths=lens, h_qk=4, h_v=8)
+    y, S = run_prefill(inp, torch.float32)
+    cu = inp["cu_seqlens"]
+    for n in range(len(lens)):
+        sub = dict(inp)
+        for nm in ("q", "k", "v", "z", "a", "b"):
+            sub[nm] = inp[nm][cu[n]:cu[n + 1]]
+        sub["init_state"] = inp["init_state"][n:n + 1]
+        sub["cu_seqlens"] = None
+        y1, S1 = run_prefill(sub, torch.float32)
+        assert np.array_equal(y1, y[cu[n]:cu[n + 1]])
+        assert np.array_equal(S1[0], S[n])
+
+
+def test_zero_tokens_copies_init():
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[0, 0], h_qk=2, h_v=4)
+    y, S = run_prefill(inp, torch.float32)
+    assert y.shape[0] == 0
+    assert np.array_equal(S, inp["init_state"].astype(np.float64))
+
+
+def test_varlen8_bf16_sampled_heads(oracle_mod):
+    inp = make_inputs("varlen8_prefill_bf16")
+    heads = (0, 4)
+    ref = _oracle(oracle_mod, inp, heads=heads)
+    y, S = run_prefill(inp, torch.float32)
+    sl = slice(*heads)
+    check_bf16(y[:, sl], ref["y"][:, sl], S[:, sl], ref["final_state"][:, sl])
+
+
+@pytest.mark.slow
+def test_long_prefill_T262144_sampled_heads(oracle_mod):
+    inp = make_inputs("long_prefill_T262144_bf16")
+    heads = (30, 32)
+    ref = _oracle(oracle_mod, inp, heads=heads)
+    y, S = run_prefill(inp, torch.float32)
+    sl = slice(*heads)
+    check_bf16(y[:, sl], ref["y"][:, sl], S[:, sl], ref["final_state"][:, sl])
