@@ -31,7 +31,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp,
-           os.path.join(CSRC, "gdn_api.cu")]
+           *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)

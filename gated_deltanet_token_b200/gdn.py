@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill_workspace_size.argtypes = [dp]
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_prefill.argtypes = [dp] + [vp] * 14 + [vp, ctypes.c_size_t, vp]
+        L.gdn_prefill_noalloc.restype = ctypes.c_int
+        L.gdn_prefill_noalloc.argtypes = [dp] + [vp] * 14 + [vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode.argtypes = [dp] + [vp] * 13 + [vp]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -163,6 +165,32 @@ def gdn_prefill(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, init_state=Non
                            workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_prefill")
+    return y, final_state
+
+
+def gdn_prefill_noalloc(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, init_state=None,
+                        cu_seqlens=None, *, out_dtype=None, y=None, final_state=None,
+                        q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6, stream=None):
+    """gdn_prefill on the library's built-in scratch (no workspace argument).  For callers
+    that cannot allocate device memory at call time; outputs must then be passed in.
+    Dims whose workspace exceeds the built-in scratch raise GdnError(GDN_ERR_WORKSPACE)."""
+    T, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    n = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out_dtype is None:
+        out_dtype = y.dtype if y is not None else q.dtype
+    dims = make_dims(n, T, h_qk, h_v, _dt(q), _dt(torch.empty(0, dtype=out_dtype)), d_k, d_v, q_scale,
+                     l2_eps, rms_eps)
+    if y is None:
+        y = torch.empty((T, h_v, d_v), dtype=out_dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((n, h_v, d_v, d_k), dtype=torch.float32, device=q.device)
+    rc = lib().gdn_prefill_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(a),
+                                   _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(conv_w), _ptr(norm_w),
+                                   _ptr(init_state), _ptr(cu_seqlens), _ptr(y), _ptr(final_state),
+                                   _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_prefill_noalloc")
     return y, final_state
 
 

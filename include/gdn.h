@@ -149,6 +149,38 @@ typedef struct gdn_kernel_time {
  */
 int gdn_profile_read(gdn_kernel_time_t* out, int max_entries);
 
+/*
+ * Size of the library's built-in prefill scratch used by gdn_prefill_noalloc: 64 MiB of
+ * device memory per GPU that loads the library, held until the process exits.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * gdn_prefill without a caller-provided workspace, for callers that cannot allocate
+ * device memory at call time: code whose device memory is entirely owned by another
+ * allocator (a serving framework's pre-reserved pool), or code that must not trigger the
+ * device-wide synchronisation that cudaMalloc / cudaFree can cause inside a
+ * latency-critical loop.  The pages define no such call; it exists only for such callers.
+ *
+ * Same arguments, layouts and results as gdn_prefill, minus workspace and its size.  The
+ * scratch is a fixed array inside the library (GDN_NOALLOC_SCRATCH_BYTES); this call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Returns GDN_ERR_WORKSPACE, launching nothing, when gdn_prefill_workspace_size(d)
+ *     exceeds GDN_NOALLOC_SCRATCH_BYTES (at the pages' model shape, 16 QK / 32 value
+ *     heads, that is about 740 packed tokens).
+ *   - The first call on a device looks up that device's address of the scratch array
+ *     (with that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous call's
+ *     contents; the prefill writes every scratch byte before reading it, so nothing needs
+ *     clearing.  Calls whose work overlaps on the GPU (two streams, or two host threads)
+ *     race on the array and corrupt each other's results: serialise them.
+ */
+int gdn_prefill_noalloc(const gdn_dims_t* d, const void* q, const void* k, const void* v,
+                        const void* z, const float* a, const float* b, const float* A_log,
+                        const float* dt_bias, const float* conv_w, const float* norm_w,
+                        const float* init_state, const int32_t* cu_seqlens, void* y,
+                        float* final_state, gdn_stream_t stream);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gdn_version(void);
 
