@@ -3,6 +3,7 @@
 // entry point are in include/gdn.h.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -11,6 +12,7 @@
 #include "gdn.h"
 #include "gdn_common.cuh"
 #include "k_chunk_simt.cuh"
+#include "k_chunk_tc.cuh"
 #include "k_decode.cuh"
 #include "k_stream.cuh"
 
@@ -18,17 +20,54 @@ using namespace gdn;
 
 namespace {
 
+__device__ float g_selftest_out[2];
+
 constexpr int kVersion = 100;  // 0.1.0
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The bf16-input prefill runs its chunk contractions on tcgen05 (bf16 hi/lo products); the
+// fp32-input prefill keeps true fp32 FFMA.  GDN_FORCE_SIMT=1 in the environment sends bf16
+// inputs down the fp32 path too (for comparisons).
+bool use_tc(const gdn_dims_t* d) {
+  if (d->in_dtype != GDN_DTYPE_BF16) return false;
+  const char* f = getenv("GDN_FORCE_SIMT");
+  return !(f && f[0] == '1');
+}
+
 // Workspace of the prefill, carved from the caller's buffer in this order.
 struct WsLayout {
   size_t tab, seqc0, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
+  size_t kq, tp, gb;  // tensor-core path
   int max_chunks;
+  bool tc;
 };
 
+WsLayout ws_layout_tc(const gdn_dims_t* d) {
+  WsLayout L{};
+  L.tc = true;
+  const size_t T = (size_t)d->total_tokens, hq = (size_t)d->h_qk, hv = (size_t)d->h_v;
+  const size_t N = (size_t)d->n_seqs;
+  L.max_chunks = (int)((T + CH - 1) / CH + N);
+  const size_t MC = (size_t)L.max_chunks;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.tab = take(MC * sizeof(ChunkEntry));
+  L.seqc0 = take((N + 1) * sizeof(int));
+  L.kq = take(MC * hq * KQ_BYTES);
+  L.tp = take(MC * hv * TP_BYTES);
+  L.gb = take(MC * hv * GB_FLOATS * 4);
+  L.yraw = take(T * hv * D * 4);
+  L.total = off;
+  return L;
+}
+
 WsLayout ws_layout(const gdn_dims_t* d) {
+  if (use_tc(d)) return ws_layout_tc(d);
   WsLayout L{};
   const size_t T = (size_t)d->total_tokens, hq = (size_t)d->h_qk, hv = (size_t)d->h_v;
   const size_t N = (size_t)d->n_seqs;
@@ -125,6 +164,10 @@ int configure_device() {
   if (cudaFuncSetAttribute(k_phaseA_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM) !=
           cudaSuccess ||
       cudaFuncSetAttribute(k_phaseB_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PB_SMEM) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkprep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_TC_SMEM) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkscan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PB_TC_SMEM) !=
           cudaSuccess)
     return GDN_ERR_CUDA;
   done_mask.fetch_or(bit);
@@ -205,6 +248,27 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
   {
     ProfScope p("tilemap", s);
     k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0);
+  }
+  if (L.tc) {
+    uint8_t* kq = reinterpret_cast<uint8_t*>(ws + L.kq);
+    uint8_t* tp = reinterpret_cast<uint8_t*>(ws + L.tp);
+    if (d->total_tokens > 0) {
+      ProfScope p("chunk_prep_tc", s);
+      k_chunkprep_tc<<<dim3(L.max_chunks, d->h_qk), 256, PA_TC_SMEM, s>>>(
+          kd, tab, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), a, b, A_log, dt_bias,
+          conv_w, kq, tp, F(L.gb));
+    }
+    {
+      ProfScope p("chunk_scan_tc", s);
+      k_chunkscan_tc<<<dim3(d->n_seqs, d->h_v, D / TC_NV), 128, PB_TC_SMEM, s>>>(
+          kd, cu_seqlens, seqc0, static_cast<const uint16_t*>(v), conv_w, kq, tp, F(L.gb), init_state,
+          F(L.yraw), final_state);
+    }
+    if (d->total_tokens > 0) {
+      ProfScope p("epilogue", s);
+      launch_epilogue(kd, F(L.yraw), z, norm_w, y, s);
+    }
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
   }
   if (d->total_tokens > 0) {
     {
@@ -296,6 +360,38 @@ int gdn_profile_read(gdn_kernel_time_t* out, int max_entries) {
   }
   g_prof.n = 0;
   return m;
+}
+
+int gdn_selftest_tc(int case_id, float* out2) {
+  if (!out2) return GDN_ERR_NULL;
+  if (case_id < 0 || case_id > 3) return GDN_ERR_SHAPE;
+  float zero[2] = {0.0f, 0.0f};
+  if (cudaMemcpyToSymbol(g_selftest_out, zero, sizeof zero) != cudaSuccess) return GDN_ERR_CUDA;
+  float* dptr = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&dptr), g_selftest_out) != cudaSuccess) return GDN_ERR_CUDA;
+  const int smem = 160 * 1024;
+  cudaError_t e = cudaSuccess;
+  switch (case_id) {
+    case 0:
+      e = cudaFuncSetAttribute(k_selftest_umma<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_selftest_umma<0><<<1, 128, smem>>>(dptr);
+      break;
+    case 1:
+      e = cudaFuncSetAttribute(k_selftest_umma<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_selftest_umma<1><<<1, 128, smem>>>(dptr);
+      break;
+    case 2:
+      e = cudaFuncSetAttribute(k_selftest_umma<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_selftest_umma<2><<<1, 128, smem>>>(dptr);
+      break;
+    default:
+      e = cudaFuncSetAttribute(k_selftest_umma<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_selftest_umma<3><<<1, 128, smem>>>(dptr);
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(out2, g_selftest_out, sizeof zero) != cudaSuccess) return GDN_ERR_CUDA;
+  return GDN_OK;
 }
 
 int gdn_read_device_status(gdn_stream_t stream) {

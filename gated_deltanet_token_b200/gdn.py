@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_profile_enable.argtypes = [ctypes.c_int]
         L.gdn_profile_read.restype = ctypes.c_int
         L.gdn_profile_read.argtypes = [ctypes.POINTER(gdn_kernel_time_t), ctypes.c_int]
+        L.gdn_selftest_tc.restype = ctypes.c_int
+        L.gdn_selftest_tc.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_float)]
         L.gdn_version.restype = ctypes.c_int
         L.gdn_version.argtypes = []
         _lib = L
@@ -116,6 +118,15 @@ def gdn_version() -> int:
 
 def gdn_read_device_status(stream=None) -> int:
     return lib().gdn_read_device_status(_stream(stream))
+
+
+def gdn_selftest_tc(case_id: int) -> tuple[float, float]:
+    """(max |tensor-core - CUDA-core|, max |reference|) for one operand-layout case."""
+    out = (ctypes.c_float * 2)()
+    rc = lib().gdn_selftest_tc(int(case_id), out)
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_selftest_tc")
+    return float(out[0]), float(out[1])
 
 
 def gdn_profile_enable(on: bool) -> None:
