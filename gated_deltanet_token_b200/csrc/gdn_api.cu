@@ -38,7 +38,7 @@ bool use_tc(const gdn_dims_t* d) {
 // Workspace of the prefill, carved from the caller's buffer in this order.
 struct WsLayout {
   size_t tab, seqc0, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
-  size_t kq, tp, gb;  // tensor-core path
+  size_t kq, tp, gb, bv;  // tensor-core path
   int max_chunks;
   bool tc;
 };
@@ -61,6 +61,7 @@ WsLayout ws_layout_tc(const gdn_dims_t* d) {
   L.kq = take(MC * hq * KQ_BYTES);
   L.tp = take(MC * hv * TP_BYTES);
   L.gb = take(MC * hv * GB_FLOATS * 4);
+  L.bv = take(MC * hv * BV_BYTES);
   L.yraw = take(T * hv * D * 4);
   L.total = off;
   return L;
@@ -253,16 +254,20 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     uint8_t* kq = reinterpret_cast<uint8_t*>(ws + L.kq);
     uint8_t* tp = reinterpret_cast<uint8_t*>(ws + L.tp);
     if (d->total_tokens > 0) {
+      {
+        ProfScope p("prologue_tc", s);
+        k_prologue_tc<<<dim3(L.max_chunks, 2 * d->h_qk + d->h_v), 256, 0, s>>>(
+            kd, tab, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+            static_cast<const uint16_t*>(v), b, conv_w, kq, F(L.bv));
+      }
       ProfScope p("chunk_prep_tc", s);
-      k_chunkprep_tc<<<dim3(L.max_chunks, d->h_qk), 256, PA_TC_SMEM, s>>>(
-          kd, tab, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), a, b, A_log, dt_bias,
-          conv_w, kq, tp, F(L.gb));
+      k_chunkprep_tc<<<dim3(L.max_chunks, d->h_qk), 256, PA_TC_SMEM, s>>>(kd, tab, a, b, A_log, dt_bias, kq, tp,
+                                                                          F(L.gb));
     }
     {
       ProfScope p("chunk_scan_tc", s);
-      k_chunkscan_tc<<<dim3(d->n_seqs, d->h_v, D / TC_NV), 128, PB_TC_SMEM, s>>>(
-          kd, cu_seqlens, seqc0, static_cast<const uint16_t*>(v), conv_w, kq, tp, F(L.gb), init_state,
-          F(L.yraw), final_state);
+      k_chunkscan_tc<<<dim3(d->n_seqs, d->h_v, D / TC_NV), 288, PB_TC_SMEM, s>>>(
+          kd, cu_seqlens, seqc0, kq, tp, F(L.gb), F(L.bv), init_state, F(L.yraw), final_state);
     }
     if (d->total_tokens > 0) {
       ProfScope p("epilogue", s);

@@ -35,6 +35,8 @@ constexpr uint32_t KQ_BYTES = 2 * KQ_TILE;           // per (chunk, QK head)
 constexpr uint32_t TP_TILE = 128 * 64 * 2;           // one bf16 tile of [T;P]: 16 KB
 constexpr uint32_t TP_BYTES = 2 * TP_TILE;           // per (chunk, value head)
 constexpr uint32_t GB_FLOATS = 128;                  // gamma[64], beta[64] per (chunk, value head)
+constexpr uint32_t BV_SLICE = 64 * TC_NV * 4;        // beta * v (fp32) of one 32-column slice: 8 KB
+constexpr uint32_t BV_BYTES = 4 * BV_SLICE;          // per (chunk, value head)
 constexpr uint32_t LBO128 = 2048;                    // K-direction core stride of 128-row tiles
 
 // Byte offset of element (r, k) in a K-major no-swizzle tile with 128 rows.
@@ -163,36 +165,159 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 }
 
 // ======================================================================================
+// Prologue of the tensor-core path (K1): one CTA per (chunk, stream unit), 256 threads.
+//   unit < h_qk:       K rows (0..63) of the [K;Q] tile of QK head `unit`
+//   unit < 2 h_qk:     Q rows (64..127) of the tile of QK head `unit - h_qk`
+//   otherwise:         beta * v of value head `unit - 2 h_qk`, as four contiguous 32-column
+//                      fp32 slices [4][64][32] (one per phase-B CTA)
+// Width-4 causal conv and SiLU ("Qwen3.8-Flash-Next" technical report, Fig. 2; field
+// guide §02), L2 norm of q and k (Fig. 2), beta = sigmoid(b).  q/k warps: 8 tokens per
+// warp, lane = (row r = lane % 8, 8-channel groups lane / 8 + 4 i); the four lanes of a
+// row reduce the L2 norm with two shuffles, and consecutive lanes store consecutive
+// 16-byte chunks of the tile (coalesced).
+// ======================================================================================
+__global__ void __launch_bounds__(256) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab,
+                                                     const uint16_t* __restrict__ q,
+                                                     const uint16_t* __restrict__ k,
+                                                     const uint16_t* __restrict__ v,
+                                                     const float* __restrict__ b,
+                                                     const float* __restrict__ conv_w,
+                                                     uint8_t* __restrict__ kq_ws, float* __restrict__ bv_ws) {
+  const ChunkEntry e = tab[blockIdx.x];
+  if (e.len == 0) return;
+  const int u = blockIdx.y, hq = d.h_qk, hv = d.h_v, L = e.len;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the unit's 128 channels x 4 taps, staged once
+  __shared__ float4 wsm[D];
+  const size_t chu = u < hq ? (size_t)(hq + u) * D : u < 2 * hq ? (size_t)(u - hq) * D
+                                                                 : (size_t)2 * hq * D + (size_t)(u - 2 * hq) * D;
+  if (tid < D) wsm[tid] = *reinterpret_cast<const float4*>(conv_w + (chu + tid) * 4);
+  __syncthreads();
+  if (u < 2 * hq) {
+    const bool isq = u >= hq;
+    const int j = isq ? u - hq : u;
+    const uint16_t* src = isq ? q : k;
+    const int r = lane & 7, g0 = lane >> 3;  // row within the warp's 8 tokens; first channel group
+    const int t = warp * 8 + r;              // chunk-relative token
+    // taps for the lane's 32 channels: groups g0, g0 + 4, g0 + 8, g0 + 12 (8 channels each)
+    float acc[4][8];
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[gi][c] = 0.0f;
+#pragma unroll
+    for (int tap = 0; tap < 4; ++tap) {
+      const long tg = (long)e.t0 + t - 3 + tap;
+      const bool ok = t < L && tg >= e.seq_start;
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        const int cg = (g0 + 4 * gi) * 8;
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (ok) x = *reinterpret_cast<const uint4*>(src + ((size_t)tg * hq + j) * D + cg);
+        const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float xv = bf2f(c & 1 ? wd[c >> 1] >> 16 : wd[c >> 1] & 0xffffu);
+          acc[gi][c] = fmaf(comp(wsm[cg + c], tap), xv, acc[gi][c]);
+        }
+      }
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float y = acc[gi][c] / (1.0f + __expf(-acc[gi][c]));
+        acc[gi][c] = y;
+        ss = fmaf(y, y, ss);
+      }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+    const float inv = t < L ? (isq ? d.q_scale : 1.0f) * rsqrtf(ss + d.l2_eps) : 0.0f;
+    uint8_t* tile = kq_ws + ((size_t)blockIdx.x * hq + j) * KQ_BYTES;
+    const int row = (isq ? 64 : 0) + t;
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) {
+      float x8[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x8[c] = acc[gi][c] * inv;
+      uint4 hi, lo;
+      tc::split8(x8, hi, lo);
+      const uint32_t off = kmaj128(row, (g0 + 4 * gi) * 8);
+      *reinterpret_cast<uint4*>(tile + off) = hi;
+      *reinterpret_cast<uint4*>(tile + KQ_TILE + off) = lo;
+    }
+  } else {
+    const int h = u - 2 * hq;
+    const int c0 = lane * 4, tb = warp * 8;
+    float w[4][4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float4 t4 = wsm[c0 + c];
+      w[c][0] = t4.x; w[c][1] = t4.y; w[c][2] = t4.z; w[c][3] = t4.w;
+    }
+    float4 x[11];
+#pragma unroll
+    for (int p = 0; p < 11; ++p) {
+      const int tcr = tb - 3 + p;
+      const long tg = (long)e.t0 + tcr;
+      const bool ok = tcr < L && tg >= e.seq_start;
+      x[p] = ok ? load4<true>(v, ((size_t)tg * hv + h) * D + c0) : make_float4(0, 0, 0, 0);
+    }
+    float* out = bv_ws + ((size_t)blockIdx.x * hv + h) * (BV_BYTES / 4) + (size_t)(c0 / TC_NV) * (BV_SLICE / 4);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int t = tb + i;
+      const float bt = t < L ? sigmoid_f(b[(size_t)(e.t0 + t) * hv + h]) : 0.0f;
+      float r4[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float acc = fmaf(w[c][3], comp(x[i + 3], c),
+                               fmaf(w[c][2], comp(x[i + 2], c), fmaf(w[c][1], comp(x[i + 1], c), w[c][0] * comp(x[i], c))));
+        r4[c] = bt * (acc / (1.0f + __expf(-acc)));
+      }
+      *reinterpret_cast<float4*>(out + t * TC_NV + (c0 % TC_NV)) = make_float4(r4[0], r4[1], r4[2], r4[3]);
+    }
+  }
+}
+
+// ======================================================================================
 // Phase A
 // ======================================================================================
-constexpr size_t PA_TC_SMEM = 65536 + 64 * 64 * 4 + TP_BYTES + 2 * 64 * 4;
+constexpr int PA_P = 68;  // pitch (floats) of the fp32 64 x 64 matrices of phase A
+constexpr uint32_t PA_MAT = 64 * PA_P * 4;
+// [0, 64K): [K;Q] tile (hi | lo), later the P operands: [Mq_a; Mq_b] (K-major, 128 x 64) hi | lo
+// and [T_a | T_b] (MN-major, K = 64, N = 128) hi | lo; then KK, QK, A, T_a, T_b (fp32), gates.
+constexpr uint32_t PA_OFF_KK = 65536;
+constexpr uint32_t PA_OFF_QK = PA_OFF_KK + PA_MAT;
+constexpr uint32_t PA_OFF_A = PA_OFF_QK + PA_MAT;  // two heads
+constexpr uint32_t PA_OFF_T = PA_OFF_A + 2 * PA_MAT;  // two heads
+constexpr uint32_t PA_OFF_G = PA_OFF_T + 2 * PA_MAT;
+constexpr size_t PA_TC_SMEM = PA_OFF_G + 4 * 64 * 4;
+static_assert(PA_TC_SMEM <= 232448, "phase-A shared memory");
 
-// Shared-memory fp32 64 x 64 matrices in phase A use pitch 64 with the column index
-// XOR-swizzled by the row's 4-bit group, so row-wise and column-wise sweeps hit
-// different banks.
-__device__ __forceinline__ int sw64(int t, int s) { return t * 64 + (s ^ ((t & 7) << 2)); }
-
-__global__ void __launch_bounds__(256, 2)
-    k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const uint16_t* __restrict__ q,
-                   const uint16_t* __restrict__ k, const float* __restrict__ a,
+__global__ void __launch_bounds__(256, 1)
+    k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
-                   const float* __restrict__ dt_bias, const float* __restrict__ conv_w,
-                   uint8_t* __restrict__ kq_ws, uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
+                   const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
+                   uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
   const ChunkEntry e = tab[blockIdx.x];
   if (e.len == 0) return;
   const int j = blockIdx.y, hq = d.h_qk, hv = d.h_v, G = hv / hq, L = e.len;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(128) uint8_t sm[];
-  uint8_t* kq_hi = sm;                        // [K;Q] tile, hi
-  uint8_t* kq_lo = sm + KQ_TILE;              // [K;Q] tile, lo
-  float* KK = reinterpret_cast<float*>(sm);   // aliases the tile once it is consumed
-  float* QK = KK + 64 * 64;
-  float* Am = QK + 64 * 64;
-  float* Mq = Am + 64 * 64;
-  float* Tm = reinterpret_cast<float*>(sm + 65536);
-  uint8_t* tp = sm + 65536 + 64 * 64 * 4;     // [T;P] staging: hi then lo
-  float* gs = reinterpret_cast<float*>(tp + TP_BYTES);
-  float* bs = gs + 64;
+  uint8_t* kq_hi = sm;
+  uint8_t* kq_lo = sm + KQ_TILE;
+  uint8_t* pa_hi = sm;             // [Mq_a; Mq_b] operand (aliases the [K;Q] tile)
+  uint8_t* pa_lo = sm + 16384;
+  uint8_t* pb_hi = sm + 32768;     // [T_a | T_b] operand
+  uint8_t* pb_lo = sm + 49152;
+  float* KK = reinterpret_cast<float*>(sm + PA_OFF_KK);
+  float* QK = reinterpret_cast<float*>(sm + PA_OFF_QK);
+  float* Amat = reinterpret_cast<float*>(sm + PA_OFF_A);  // [2][64][PA_P]
+  float* Tm = reinterpret_cast<float*>(sm + PA_OFF_T);    // [2][64][PA_P]
+  float* gs = reinterpret_cast<float*>(sm + PA_OFF_G);  // [2][64] gamma
+  float* bs = gs + 128;                                 // [2][64] beta
   __shared__ uint64_t mbar;
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
@@ -203,67 +328,25 @@ __global__ void __launch_bounds__(256, 2)
     tc::fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(&tslot), 64);
+    tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // cols 0..63: [K;Q]K^T, 128..255: P pair
     tc::tmem_relinquish();
   }
-
-  // ---- conv + SiLU + L2 norm of the chunk's q and k rows into the [K;Q] tile -------------
-  // warp w: tokens 8w .. 8w+7, lane: channels 4 lane .. 4 lane + 3; rows 0..63 are K, 64..127 Q.
-  {
-    const int tb = warp * 8, c0 = lane * 4;
-#pragma unroll
-    for (int st = 0; st < 2; ++st) {  // st 0: k (rows 0..63), st 1: q (rows 64..127)
-      const uint16_t* src = st ? q : k;
-      const size_t ch0 = st ? (size_t)j * D : (size_t)(hq + j) * D;
-      float w[4][4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float4 t4 = *reinterpret_cast<const float4*>(conv_w + (ch0 + c0 + c) * 4);
-        w[c][0] = t4.x; w[c][1] = t4.y; w[c][2] = t4.z; w[c][3] = t4.w;
-      }
-      float4 x[11];
-#pragma unroll
-      for (int p = 0; p < 11; ++p) {
-        const int tc_ = tb - 3 + p;
-        const long tg = (long)e.t0 + tc_;
-        const bool ok = tc_ < L && tg >= e.seq_start;
-        x[p] = ok ? load4<true>(src, ((size_t)tg * hq + j) * D + c0) : make_float4(0, 0, 0, 0);
-      }
-      const float scale = st ? d.q_scale : 1.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = tb + i;
-        float r[4] = {0, 0, 0, 0};
-        if (t < L) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float acc = fmaf(w[c][3], comp(x[i + 3], c),
-                                   fmaf(w[c][2], comp(x[i + 2], c),
-                                        fmaf(w[c][1], comp(x[i + 1], c), w[c][0] * comp(x[i], c))));
-            r[c] = silu_f(acc);
-          }
-        }
-        const float ss = warp_sum(r[0] * r[0] + r[1] * r[1] + r[2] * r[2] + r[3] * r[3]);
-        const float inv = t < L ? scale / sqrtf(ss + d.l2_eps) : 0.0f;
-        uint16_t h[4], l[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tc::split2(r[c] * inv, h[c], l[c]);
-        const int row = st * 64 + t;
-        const uint32_t off = kmaj128(row, c0);  // c0 % 8 in {0, 4}: 8-byte half of a core row
-        *reinterpret_cast<uint2*>(kq_hi + off) = make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
-        *reinterpret_cast<uint2*>(kq_lo + off) = make_uint2(l[0] | (uint32_t(l[1]) << 16), l[2] | (uint32_t(l[3]) << 16));
-      }
-    }
-  }
-  tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
-  uint8_t* kq_dst = kq_ws + ((size_t)blockIdx.x * hq + j) * KQ_BYTES;
-  if (tid == 0) {
-    tc::bulk_s2g(kq_dst, tc::smem_u32(sm), KQ_BYTES);
-    tc::bulk_commit();
+  if (tid == 0) {  // the [K;Q] tile written by the prologue
+    const uint32_t bar = tc::smem_u32(&mbar);
+    tc::mbar_arrive_expect_tx(bar, KQ_BYTES);
+    tc::bulk_g2s(tc::smem_u32(sm), kq_ws + ((size_t)blockIdx.x * hq + j) * KQ_BYTES, KQ_BYTES, bar);
+  }
+  if (!tc::mbar_wait(tc::smem_u32(&mbar), 0)) {
+    s_abort = 1;
+    atomicExch(&g_gdn_status, -7);
+  }
+  __syncthreads();
+  tc::tc_fence_after();
+  if (tid == 0 && !s_abort) {
     // D[128 x 64] = [K;Q] (K-major, 128 x 128) x K^T (B = rows 0..63 of the tile, K-major)
     constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
     const uint32_t base[2] = {tc::smem_u32(kq_hi), tc::smem_u32(kq_lo)};
@@ -275,40 +358,36 @@ __global__ void __launch_bounds__(256, 2)
       }
     tc::umma_commit(tc::smem_u32(&mbar));
   }
-  if (!tc::mbar_wait(tc::smem_u32(&mbar), 0)) {
+  if (!s_abort && !tc::mbar_wait(tc::smem_u32(&mbar), 1)) {
     s_abort = 1;
     atomicExch(&g_gdn_status, -7);
   }
   tc::tc_fence_after();
-  if (tid == 0) tc::bulk_wait_read_all();  // the tile may now be overwritten
-  __syncthreads();
-  const bool aborted = s_abort != 0;
-  // TMEM rows 0..63: K K^T, rows 64..127: Q K^T (warps 0..3, one row per thread)
-  uint32_t r0[32], r1[32];
-  if (warp < 4) {
+  if (warp < 4) {  // TMEM rows 0..63: K K^T, rows 64..127: Q K^T (one row per thread)
+    uint32_t r0[32], r1[32];
     const uint32_t ta = tbase + ((uint32_t)(warp * 32) << 16);
     tc::tmem_ld32(ta, r0);
     tc::tmem_ld32(ta + 32, r1);
     tc::tmem_wait_ld();
-  }
-  tc::tc_fence_before();
-  __syncthreads();  // every read of the tile (MMA, bulk store) is over: alias it
-  if (warp < 4 && !aborted) {
-    const int row = tid;
-    float* dst = row < 64 ? KK : QK;
-    const int t = row & 63;
+    float* dst = (tid < 64 ? KK : QK) + (tid & 63) * PA_P;
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      dst[sw64(t, c)] = __uint_as_float(r0[c]);
-      dst[sw64(t, 32 + c)] = __uint_as_float(r1[c]);
+    for (int c = 0; c < 32; c += 4) {
+      *reinterpret_cast<float4*>(dst + c) = make_float4(__uint_as_float(r0[c]), __uint_as_float(r0[c + 1]),
+                                                        __uint_as_float(r0[c + 2]), __uint_as_float(r0[c + 3]));
+      *reinterpret_cast<float4*>(dst + 32 + c) = make_float4(__uint_as_float(r1[c]), __uint_as_float(r1[c + 1]),
+                                                             __uint_as_float(r1[c + 2]), __uint_as_float(r1[c + 3]));
     }
   }
+  tc::tc_fence_before();
   __syncthreads();
+  const bool aborted = s_abort != 0;
 
-  // ---- per value head: gates, A, M o QK^T, T = (I + A)^-1, P = (M o QK^T) T ---------------
-  for (int g = 0; g < G && !aborted; ++g) {
-    const int h = j * G + g;
-    if (warp == 0) {
+  // ---- value heads in pairs (ga, gb = ga + 1, or ga again when G is odd) -------------------
+  uint32_t mma_phase = 0;
+  for (int ga = 0; ga < G && !aborted; ga += 2) {
+    const int gpair[2] = {ga, ga + 1 < G ? ga + 1 : ga};
+    if (warp < 2) {  // gates and gamma of the pair: warp 0 head a, warp 1 head b
+      const int h = j * G + gpair[warp];
       float g0 = 0.0f, g1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
       if (lane < L) {
         const size_t o = (size_t)(e.t0 + lane) * hv + h;
@@ -327,163 +406,239 @@ __global__ void __launch_bounds__(256, 2)
         if (lane >= o) { g0 += y0; g1 += y1; }
       }
       g1 += __shfl_sync(0xffffffffu, g0, 31);
-      gs[lane] = g0; gs[lane + 32] = g1;
-      bs[lane] = b0; bs[lane + 32] = b1;
-      float* gb = gb_ws + ((size_t)blockIdx.x * hv + h) * GB_FLOATS;
-      gb[lane] = g0; gb[lane + 32] = g1;
-      gb[64 + lane] = b0; gb[96 + lane] = b1;
+      gs[warp * 64 + lane] = g0; gs[warp * 64 + lane + 32] = g1;
+      bs[warp * 64 + lane] = b0; bs[warp * 64 + lane + 32] = b1;
+      if (warp == 0 || gpair[1] != gpair[0]) {
+        float* gbw = gb_ws + ((size_t)blockIdx.x * hv + h) * GB_FLOATS;
+        gbw[lane] = g0; gbw[lane + 32] = g1;
+        gbw[64 + lane] = b0; gbw[96 + lane] = b1;
+      }
     }
     __syncthreads();
-    for (int idx = tid; idx < 64 * 64; idx += 256) {
-      const int t = idx >> 6, s = idx & 63;
-      const float dec = s <= t ? expf(gs[t] - gs[s]) : 0.0f;  // mask before exp
-      Am[sw64(t, s)] = s < t ? bs[t] * dec * KK[sw64(t, s)] : 0.0f;
-      Mq[sw64(t, s)] = dec * QK[sw64(t, s)];
+    // A (fp32, for the solve) and the Mq rows of the P operand (bf16 hi/lo, K-major), both heads:
+    // item = (head hp, row t, 8 columns s0..s0+7)
+    for (int it = tid; it < 2 * 64 * 8; it += 256) {
+      const int t = it & 63, s0 = ((it >> 6) & 7) * 8, hp = it >> 9;
+      const float* g_ = gs + hp * 64;
+      float* Am = Amat + hp * 64 * PA_P;
+      float av[8], mv[8], kk[8], qk[8], gg[8];
+      const float gt = g_[t], bt = bs[hp * 64 + t];
+#pragma unroll
+      for (int q4 = 0; q4 < 2; ++q4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(KK + t * PA_P + s0 + q4 * 4);
+        const float4 m4 = *reinterpret_cast<const float4*>(QK + t * PA_P + s0 + q4 * 4);
+        const float4 g4 = *reinterpret_cast<const float4*>(g_ + s0 + q4 * 4);
+        kk[q4 * 4 + 0] = k4.x; kk[q4 * 4 + 1] = k4.y; kk[q4 * 4 + 2] = k4.z; kk[q4 * 4 + 3] = k4.w;
+        qk[q4 * 4 + 0] = m4.x; qk[q4 * 4 + 1] = m4.y; qk[q4 * 4 + 2] = m4.z; qk[q4 * 4 + 3] = m4.w;
+        gg[q4 * 4 + 0] = g4.x; gg[q4 * 4 + 1] = g4.y; gg[q4 * 4 + 2] = g4.z; gg[q4 * 4 + 3] = g4.w;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int s_ = s0 + c;
+        const float dec = s_ <= t ? __expf(gt - gg[c]) : 0.0f;  // mask before exp
+        av[c] = s_ < t ? bt * dec * kk[c] : 0.0f;
+        mv[c] = dec * qk[c];
+      }
+      *reinterpret_cast<float4*>(Am + t * PA_P + s0) = make_float4(av[0], av[1], av[2], av[3]);
+      *reinterpret_cast<float4*>(Am + t * PA_P + s0 + 4) = make_float4(av[4], av[5], av[6], av[7]);
+      uint4 hi, lo;
+      tc::split8(mv, hi, lo);
+      *reinterpret_cast<uint4*>(pa_hi + kmaj128(hp * 64 + t, s0)) = hi;
+      *reinterpret_cast<uint4*>(pa_lo + kmaj128(hp * 64 + t, s0)) = lo;
     }
     __syncthreads();
-    // T = (I + A)^-1, blocked by 16 x 16: diagonal blocks by forward substitution ...
-    if (tid < 64) {
-      const int blk = tid >> 4, c = tid & 15, o = blk * 16;
+    // T = (I + A)^-1 by 16 x 16 blocks.  Diagonal blocks by forward substitution, both heads at
+    // once (thread = head, block, column), each row of A read as four float4 loads ...
+    if (tid < 128) {
+      const int hp = tid >> 6, blk = (tid >> 4) & 3, c = tid & 15, o = blk * 16;
+      const float* Ab = Amat + hp * 64 * PA_P + o * PA_P + o;
+      float* Tb = Tm + hp * 64 * PA_P + o * PA_P + o;
       float x[16];
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
+        float ar[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(Ab + t * PA_P + q4 * 4);
+          ar[q4 * 4 + 0] = a4.x; ar[q4 * 4 + 1] = a4.y; ar[q4 * 4 + 2] = a4.z; ar[q4 * 4 + 3] = a4.w;
+        }
         float v = (t == c) ? 1.0f : 0.0f;
 #pragma unroll
-        for (int r = 0; r < t; ++r) v = fmaf(-Am[sw64(o + t, o + r)], x[r], v);
+        for (int r = 0; r < t; ++r) v = fmaf(-ar[r], x[r], v);
         x[t] = v;
       }
 #pragma unroll
-      for (int t = 0; t < 16; ++t) Tm[sw64(o + t, o + c)] = x[t];
-    }
-    for (int idx = tid; idx < 64 * 64; idx += 256) {  // zero the strict upper triangle of blocks
-      const int t = idx >> 6, s = idx & 63;
-      if ((s >> 4) > (t >> 4)) Tm[sw64(t, s)] = 0.0f;
+      for (int t = 0; t < 16; ++t) Tb[t * PA_P + c] = x[t];
+    } else {
+      for (int idx = tid - 128; idx < 2 * 64 * 16; idx += 128) {  // zero blocks above the diagonal
+        const int hp = idx >> 10, t = (idx >> 4) & 63, s4 = (idx & 15) * 4;
+        if ((s4 >> 4) > (t >> 4))
+          *reinterpret_cast<float4*>(Tm + hp * 64 * PA_P + t * PA_P + s4) = make_float4(0, 0, 0, 0);
+      }
     }
     __syncthreads();
-    // ... then block (bi, bj), bi > bj, by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
+    // ... then blocks by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj (both heads).  Item =
+    // (head, block column bj, column quad, row rr); the 16 rows of a quad sit in one half-warp,
+    // which shares the rows of W = sum_k A_ik T_kj by shuffles.
     for (int dist = 1; dist < 4; ++dist) {
-      const int nblk = 4 - dist;
-      int ti = -1, tj = -1;
-      if (tid < nblk * 64) {  // thread: (block bj, row-in-block rr, 4 columns)
-        const int bj = tid >> 6, bi = bj + dist, rr = (tid >> 2) & 15, cq = (tid & 3) * 4;
-        ti = bi * 16 + rr;
-        tj = bj * 16 + cq;
-        float w4[4] = {0, 0, 0, 0};
-        // W = sum_{k=bj}^{bi-1} A_{bi,k} T_{k,bj}, row rr of block bi, columns cq..cq+3
-        for (int kb = bj; kb < bi; ++kb)
-#pragma unroll 4
-          for (int kk = 0; kk < 16; ++kk) {
-            const float av = Am[sw64(ti, kb * 16 + kk)];
+      const int per_head = (4 - dist) * 64, nitems = 2 * per_head;
+      for (int it0 = 0; it0 < nitems; it0 += 256) {
+        const int it = it0 + tid;
+        if (it0 + (tid & ~31) >= nitems) break;  // whole warps only (nitems % 128 == 0)
+        const int hp = it / per_head, rem = it % per_head;
+        const int rr = rem & 15, cq = ((rem >> 4) & 3) * 4, bj = rem >> 6, bi = bj + dist;
+        const int ti = bi * 16 + rr, tj = bj * 16 + cq;
+        const float* Am = Amat + hp * 64 * PA_P;
+        float* T = Tm + hp * 64 * PA_P;
+        float4 wv = make_float4(0, 0, 0, 0);
+        for (int kk = bj * 16; kk < bi * 16; kk += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(Am + ti * PA_P + kk);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) w4[c] = fmaf(av, Tm[sw64(kb * 16 + kk, tj + c)], w4[c]);
+          for (int u = 0; u < 4; ++u) {
+            const float4 tv = *reinterpret_cast<const float4*>(T + (kk + u) * PA_P + tj);
+            wv.x = fmaf(av[u], tv.x, wv.x); wv.y = fmaf(av[u], tv.y, wv.y);
+            wv.z = fmaf(av[u], tv.z, wv.z); wv.w = fmaf(av[u], tv.w, wv.w);
           }
-        // stage W in the strict upper triangle of Am (read by nobody), transposed
-#pragma unroll
-        for (int c = 0; c < 4; ++c) Am[sw64(tj + c, ti)] = w4[c];
-      }
-      __syncthreads();
-      float res[4] = {0, 0, 0, 0};
-      if (tid < nblk * 64) {
-        const int bi = (tid >> 6) + dist, rr = (tid >> 2) & 15;
-        // T_ij[rr][c] = -sum_m T_ii[rr][m] W[m][c]
-        for (int m = 0; m <= rr; ++m) {
-          const float tv = Tm[sw64(bi * 16 + rr, bi * 16 + m)];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) res[c] = fmaf(-tv, Am[sw64(tj + c, bi * 16 + m)], res[c]);
         }
-      }
-      __syncthreads();
-      if (tid < nblk * 64) {
+        float4 trow[4];  // T_ii row rr
 #pragma unroll
-        for (int c = 0; c < 4; ++c) Tm[sw64(ti, tj + c)] = res[c];
+        for (int q4 = 0; q4 < 4; ++q4) trow[q4] = *reinterpret_cast<const float4*>(T + ti * PA_P + bi * 16 + q4 * 4);
+        float4 res = make_float4(0, 0, 0, 0);
+        const int base = lane & 16;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float tv = m <= rr ? comp(trow[m >> 2], m & 3) : 0.0f;
+          const float w0 = __shfl_sync(0xffffffffu, wv.x, base + m);
+          const float w1 = __shfl_sync(0xffffffffu, wv.y, base + m);
+          const float w2 = __shfl_sync(0xffffffffu, wv.z, base + m);
+          const float w3 = __shfl_sync(0xffffffffu, wv.w, base + m);
+          res.x = fmaf(-tv, w0, res.x); res.y = fmaf(-tv, w1, res.y);
+          res.z = fmaf(-tv, w2, res.z); res.w = fmaf(-tv, w3, res.w);
+        }
+        *reinterpret_cast<float4*>(T + ti * PA_P + tj) = res;
       }
       __syncthreads();
     }
-    // P = (M o QK^T) T, and the [T;P] hi/lo tile: thread (t = tid / 4, 16 columns)
-    {
-      const int t = tid >> 2, s0 = (tid & 3) * 16;
-      float p[16];
+    // [T_a | T_b] as the MN-major B operand of P (rows r, columns hp * 64 + s), and the T rows
+    // of each head's [T;P] output tile (K-major, straight to the workspace)
+    for (int it = tid; it < 2 * 64 * 8; it += 256) {
+      const int r = it & 63, s0 = ((it >> 6) & 7) * 8, hp = it >> 9;
+      const float* T = Tm + hp * 64 * PA_P + r * PA_P + s0;
+      float tv[8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) p[c] = 0.0f;
-      for (int r = s0; r <= t; ++r) {  // P[t][s] = sum_{s <= r <= t} Mq[t][r] T[r][s]
-        const float mv = Mq[sw64(t, r)];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) p[c] = fmaf(mv, Tm[sw64(r, s0 + c)], p[c]);
-      }
-      float tv[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) tv[c] = Tm[sw64(t, s0 + c)];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint4 th, tl, ph, pl;
-        tc::split8(tv + half * 8, th, tl);
-        tc::split8(p + half * 8, ph, pl);
-        const int kcol = s0 + half * 8;
-        *reinterpret_cast<uint4*>(tp + kmaj128(t, kcol)) = th;
-        *reinterpret_cast<uint4*>(tp + TP_TILE + kmaj128(t, kcol)) = tl;
-        *reinterpret_cast<uint4*>(tp + kmaj128(64 + t, kcol)) = ph;
-        *reinterpret_cast<uint4*>(tp + TP_TILE + kmaj128(64 + t, kcol)) = pl;
+      for (int c = 0; c < 8; ++c) tv[c] = T[c];
+      uint4 hi, lo;
+      tc::split8(tv, hi, lo);
+      const uint32_t boff = mnmaj(r, (hp * 64 + s0) >> 3, 64);
+      *reinterpret_cast<uint4*>(pb_hi + boff) = hi;
+      *reinterpret_cast<uint4*>(pb_lo + boff) = lo;
+      if (hp == 0 || gpair[1] != gpair[0]) {
+        uint8_t* out = tp_ws + ((size_t)blockIdx.x * hv + j * G + gpair[hp]) * TP_BYTES;
+        *reinterpret_cast<uint4*>(out + kmaj128(r, s0)) = hi;
+        *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(r, s0)) = lo;
       }
     }
     tc::fence_proxy_async();
+    tc::tc_fence_before();
     __syncthreads();
+    // P pair: D[128 x 128] = [Mq_a; Mq_b] (128 x 64) x [T_a | T_b] (64 x 128); the diagonal
+    // blocks are P_a = Mq_a T_a (rows 0..63, cols 0..63) and P_b (rows 64..127, cols 64..127)
     if (tid == 0) {
-      tc::bulk_s2g(tp_ws + ((size_t)blockIdx.x * hv + h) * TP_BYTES, tc::smem_u32(tp), TP_BYTES);
-      tc::bulk_commit();
-      tc::bulk_wait_read_all();  // staging reusable for the next head
+      tc::tc_fence_after();
+      constexpr uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
+      const uint32_t a0[2] = {tc::smem_u32(pa_hi), tc::smem_u32(pa_lo)};
+      const uint32_t b0[2] = {tc::smem_u32(pb_hi), tc::smem_u32(pb_lo)};
+      for (int ks = 0; ks < 4; ++ks)
+        for (int term = 0; term < 3; ++term) {
+          const int ai = term == 2, bi = term == 1;
+          tc::umma_bf16(tbase + 128, tc::sdesc(a0[ai] + ks * 2 * LBO128, LBO128, 128),
+                        tc::sdesc(b0[bi] + ks * 256, 128, 1024), idesc, (ks | term) != 0);
+        }
+      tc::umma_commit(tc::smem_u32(&mbar));
     }
+    bool ok = tc::mbar_wait(tc::smem_u32(&mbar), mma_phase);
+    mma_phase ^= 1;
+    if (!ok) atomicExch(&g_gdn_status, -7);
+    tc::tc_fence_after();
+    if (warp < 4 && ok) {  // lane = hp * 64 + t: P row t of head hp, columns hp * 64 ..
+      const int hp = tid >> 6, t = tid & 63;
+      const uint32_t ta = tbase + 128 + ((uint32_t)(warp * 32) << 16) + hp * 64;
+      uint32_t r0[32], r1[32];
+      tc::tmem_ld32(ta, r0);
+      tc::tmem_ld32(ta + 32, r1);
+      tc::tmem_wait_ld();
+      if (hp == 0 || gpair[1] != gpair[0]) {
+        uint8_t* out = tp_ws + ((size_t)blockIdx.x * hv + j * G + gpair[hp]) * TP_BYTES;
+#pragma unroll
+        for (int s0 = 0; s0 < 64; s0 += 8) {
+          float pv[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) pv[c] = __uint_as_float(s0 < 32 ? r0[s0 + c] : r1[s0 - 32 + c]);
+          uint4 hi, lo;
+          tc::split8(pv, hi, lo);
+          *reinterpret_cast<uint4*>(out + kmaj128(64 + t, s0)) = hi;
+          *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(64 + t, s0)) = lo;
+        }
+      }
+    }
+    tc::tc_fence_before();
     __syncthreads();
   }
-  if (tid == 0) tc::bulk_wait_all();
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tbase, 64);
+  if (warp == 0) tc::tmem_dealloc(tbase, 256);
 }
 
 // ======================================================================================
 // Phase B
 // ======================================================================================
-struct PBStage {  // byte offsets inside one stage
+struct PBStage {  // byte offsets inside one input stage
   static constexpr uint32_t KQ = 0;
   static constexpr uint32_t TP = KQ_BYTES;
   static constexpr uint32_t GB = KQ_BYTES + TP_BYTES;
-  static constexpr uint32_t BYTES = KQ_BYTES + TP_BYTES + GB_FLOATS * 4;
+  static constexpr uint32_t BV = GB + GB_FLOATS * 4;  // beta * v slice; later the R / U-tilde tile
+  static constexpr uint32_t BYTES = BV + BV_SLICE;
 };
 constexpr uint32_t PB_S_TILE = 128 * TC_NV * 2;  // S^T operand (K = 128, N = nv), one of hi/lo
-constexpr uint32_t PB_R_TILE = 64 * TC_NV * 2;   // R / U-tilde operand (K = 64, N = nv)
-constexpr size_t PB_TC_SMEM = 2 * (size_t)PBStage::BYTES + 2 * PB_S_TILE + 2 * PB_R_TILE;
+constexpr uint32_t PB_R_TILE = 64 * TC_NV * 2;   // R / U-tilde operand (K = 64, N = nv): 4 KB
+constexpr size_t PB_TC_SMEM = 2 * (size_t)PB_S_TILE + 2 * (size_t)PBStage::BYTES;
+static_assert(2 * PB_R_TILE == BV_SLICE, "the R / U-tilde tile reuses the beta * v slot");
 
-__global__ void __launch_bounds__(128, 1)
+// One CTA per (sequence, value head, 32-row state slice); 9 warps: warp w < 8 serves TMEM lane
+// quarter w % 4 and columns 16 (w / 4) .. 16 (w / 4) + 15 of the slice; warp 8 issues the
+// bulk copies of the next chunk.  Each product a b is taken as a_hi [b_hi | b_lo] (one MMA of
+// width 2 nv: the lo tile follows the hi tile at the operand's N stride) plus a_lo b_hi; the
+// epilogue adds the two column halves.
+__global__ void __launch_bounds__(288, 1)
     k_chunkscan_tc(Dims d, const int* __restrict__ cu, const int* __restrict__ seq_chunk0,
-                   const uint16_t* __restrict__ v, const float* __restrict__ conv_w,
                    const uint8_t* __restrict__ kq_ws, const uint8_t* __restrict__ tp_ws,
-                   const float* __restrict__ gb_ws, const float* init_state, float* __restrict__ y_raw,
-                   float* final_state) {
-  constexpr int NV = TC_NV;
-  const int n = blockIdx.x, h = blockIdx.y, i0 = blockIdx.z * NV;
+                   const float* __restrict__ gb_ws, const float* __restrict__ bv_ws,
+                   const float* init_state, float* __restrict__ y_raw, float* final_state) {
+  constexpr int NV = TC_NV, NH = NV / 2;
+  const int n = blockIdx.x, h = blockIdx.y, sl = blockIdx.z, i0 = sl * NV;
   const int hq = d.h_qk, hv = d.h_v, G = hv / hq, j = h / G;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, cb = ((warp >> 2) & 1) * NH;
+  const bool producer = warp == 8;
+  const int row = quarter * 32 + lane;  // TMEM lane: accumulator row
   const int ts = cu ? cu[n] : 0, te = cu ? cu[n + 1] : d.total_tokens;
   const int nchunks = te > ts ? (te - ts + CH - 1) / CH : 0;
   const int gc0 = seq_chunk0[n];
   extern __shared__ __align__(128) uint8_t sm[];
-  // small operand tiles first, then the two input stages
   uint8_t* s_hi = sm;
-  uint8_t* s_lo = s_hi + PB_S_TILE;
-  uint8_t* r_hi = s_lo + PB_S_TILE;  // R, then U-tilde
-  uint8_t* r_lo = r_hi + PB_R_TILE;
-  uint8_t* const stage0 = r_lo + PB_R_TILE;
-  uint8_t* stage[2] = {stage0, stage0 + PBStage::BYTES};
+  uint8_t* s_lo = sm + PB_S_TILE;
+  uint8_t* stage[2] = {sm + 2 * PB_S_TILE, sm + 2 * PB_S_TILE + PBStage::BYTES};
   __shared__ uint64_t mbar_ld[2];
   __shared__ uint64_t mbar_mma;
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
 
-  // state slice S[i0 + i][j'] as S^T rows: thread tid owns key component j' = tid
-  float S[NV];
+  // state: thread holds S[i0 + cb + i][row] (row = key component), i < 16
+  float S[NH];
   const size_t sbase = (((size_t)n * hv + h) * D + i0) * D;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) S[i] = init_state ? init_state[sbase + (size_t)i * D + tid] : 0.0f;
+  for (int i = 0; i < NH; ++i) S[i] = (init_state && !producer) ? init_state[sbase + (size_t)(cb + i) * D + row] : 0.0f;
 
   if (tid == 0) {
     s_abort = 0;
@@ -493,7 +648,7 @@ __global__ void __launch_bounds__(128, 1)
     tc::fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(&tslot), 128);
+    tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // D_a 0..63, D_cd 64..127, D_e 128..191
     tc::tmem_relinquish();
   }
   auto issue_load = [&](int c, int st) {
@@ -504,111 +659,103 @@ __global__ void __launch_bounds__(128, 1)
     tc::bulk_g2s(dst + PBStage::KQ, kq_ws + (gc * hq + j) * KQ_BYTES, KQ_BYTES, bar);
     tc::bulk_g2s(dst + PBStage::TP, tp_ws + (gc * hv + h) * TP_BYTES, TP_BYTES, bar);
     tc::bulk_g2s(dst + PBStage::GB, gb_ws + (gc * hv + h) * GB_FLOATS, GB_FLOATS * 4, bar);
+    tc::bulk_g2s(dst + PBStage::BV, bv_ws + (gc * hv + h) * (BV_BYTES / 4) + (size_t)sl * (BV_SLICE / 4), BV_SLICE,
+                 bar);
   };
-  // S^T operand: thread j' writes its row (K index j', N = nv values) into the MN-major tile
+  // S^T operand: thread writes its row (K index = row) for its 16 columns, MN-major
   auto write_s_tile = [&]() {
 #pragma unroll
-    for (int nb = 0; nb < NV / 8; ++nb) {
+    for (int q8 = 0; q8 < 2; ++q8) {
       uint4 hi, lo;
-      tc::split8(S + nb * 8, hi, lo);
-      const uint32_t off = mnmaj(tid, nb, 128);
+      tc::split8(S + q8 * 8, hi, lo);
+      const uint32_t off = mnmaj(row, (cb >> 3) + q8, 128);
       *reinterpret_cast<uint4*>(s_hi + off) = hi;
       *reinterpret_cast<uint4*>(s_lo + off) = lo;
     }
   };
-  write_s_tile();
+  if (!producer) write_s_tile();
   tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
-  const uint32_t t_a = tbase, t_cd = tbase + NV, t_e = tbase + 2 * NV;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  if (tid == 0 && nchunks > 0) issue_load(0, 0);
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  // accumulators (2 nv columns each: [a_hi b_hi + a_lo b_hi | a_hi b_lo])
+  const uint32_t T_A = tbase, T_CD = tbase + 2 * NV, T_E = tbase + 4 * NV;
+  const uint32_t t_a = T_A + lane_off + cb, t_cd = T_CD + lane_off + cb, t_e = T_E + lane_off + cb;
+  if (producer && lane == 0 && nchunks > 0) issue_load(0, 0);
+  constexpr uint32_t idesc_kn2 = tc::idesc_bf16(128, 2 * NV, 0, 1);  // A K-major, B MN-major, N = 2 nv
+  constexpr uint32_t idesc_kn = tc::idesc_bf16(128, NV, 0, 1);
+  constexpr uint32_t idesc_mn2 = tc::idesc_bf16(128, 2 * NV, 1, 1);  // A and B MN-major
+  constexpr uint32_t idesc_mn = tc::idesc_bf16(128, NV, 1, 1);
+  const uint64_t d_s[2] = {tc::sdesc(tc::smem_u32(s_hi), 128, 16 * 128), tc::sdesc(tc::smem_u32(s_lo), 128, 16 * 128)};
 
-  // conv taps of this slice's value channels (used by warps 0..1)
-  const size_t vch0 = (size_t)2 * hq * D + (size_t)h * D + i0;
   uint32_t ph_ld[2] = {0, 0}, ph_mma = 0;
   bool aborted = false;
   for (int c = 0; c < nchunks && !aborted; ++c) {
     const int st = c & 1;
     const int t0 = ts + c * CH, L = min(CH, te - t0);
-    const uint8_t* sg = stage[st];
-    // prefetch the next chunk into the other stage (its last reader finished last chunk)
-    if (tid == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);
-    // value rows of this chunk for R (warps 0..1: thread = token row t), conv + SiLU
-    float vc[NV];
-    const int t = tid & 63;
-    if (warp < 2) {
-#pragma unroll
-      for (int i = 0; i < NV; ++i) vc[i] = 0.0f;
-      if (t < L) {
-#pragma unroll
-        for (int tap = 0; tap < 4; ++tap) {
-          const long tg = (long)t0 + t - 3 + tap;
-          if (tg < ts) continue;
-          const uint16_t* row = v + ((size_t)tg * hv + h) * D + i0;
-#pragma unroll
-          for (int q4 = 0; q4 < NV / 8; ++q4) {
-            const uint4 u = *reinterpret_cast<const uint4*>(row + q4 * 8);
-            const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const int i = q4 * 8 + p * 2;
-              vc[i] = fmaf(conv_w[(vch0 + i) * 4 + tap], bf2f(wds[p] & 0xffffu), vc[i]);
-              vc[i + 1] = fmaf(conv_w[(vch0 + i + 1) * 4 + tap], bf2f(wds[p] >> 16), vc[i + 1]);
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < NV; ++i) vc[i] = silu_f(vc[i]);
-      }
-    }
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    uint8_t* sg = stage[st];
+    uint8_t* r_hi = sg + PBStage::BV;
+    uint8_t* r_lo = r_hi + PB_R_TILE;
+    const uint32_t kq0 = tc::smem_u32(sg + PBStage::KQ), tp0 = tc::smem_u32(sg + PBStage::TP);
+    if (!producer && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_ld[st] ^= 1;
     const float* gsm = reinterpret_cast<const float*>(sg + PBStage::GB);
     const float gL = gsm[L - 1];
-    // ---- round 1: [K S^T ; Q S^T] = [K;Q] (128 x 128) x S^T (K = 128, N = nv) -------------
+    const int t = row & 63;
+    float bvr[NH];  // beta * v of token row t (rows 0..63 only), read before the slot is reused
+    if (quarter < 2) {
+      const float4* bv = reinterpret_cast<const float4*>(sg + PBStage::BV) + (t * NV + cb) / 4;
+#pragma unroll
+      for (int q4 = 0; q4 < NH / 4; ++q4) {
+        const float4 x = bv[q4];
+        bvr[q4 * 4 + 0] = x.x; bvr[q4 * 4 + 1] = x.y; bvr[q4 * 4 + 2] = x.z; bvr[q4 * 4 + 3] = x.w;
+      }
+    }
+    const float eg = t < L ? __expf(gsm[t]) : 0.0f;
     __syncthreads();
     if (s_abort) { aborted = true; break; }
+    // ---- round 1: [K S^T ; Q S^T] = [K;Q] (128 x 128) x S^T (K = 128, N = nv) -------------
     if (tid == 0) {
       tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::idesc_bf16(128, NV, 0, 1);
-      const uint32_t a0[2] = {tc::smem_u32(sg + PBStage::KQ), tc::smem_u32(sg + PBStage::KQ + KQ_TILE)};
-      const uint32_t b0[2] = {tc::smem_u32(s_hi), tc::smem_u32(s_lo)};
-      for (int ks = 0; ks < 8; ++ks)
-        for (int term = 0; term < 3; ++term) {
-          const int ai = term == 2, bi = term == 1;
-          tc::umma_bf16(t_a, tc::sdesc(a0[ai] + ks * 2 * LBO128, LBO128, 128),
-                        tc::sdesc(b0[bi] + ks * 256, 128, 16 * 128), idesc, (ks | term) != 0);
-        }
+      const uint64_t da[2] = {tc::sdesc(kq0, LBO128, 128), tc::sdesc(kq0 + KQ_TILE, LBO128, 128)};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ao = (uint64_t)((ks * 2 * LBO128) >> 4), bo = (uint64_t)((ks * 256) >> 4);
+        tc::umma_bf16(T_A, da[0] + ao, d_s[0] + bo, idesc_kn2, ks != 0);  // a_hi [s_hi | s_lo]
+        tc::umma_bf16(T_A, da[1] + ao, d_s[0] + bo, idesc_kn, 1);         // a_lo s_hi
+      }
       tc::umma_commit(tc::smem_u32(&mbar_mma));
     }
+    if (producer && lane == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);  // stage last read by chunk c-1
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_mma ^= 1;
     tc::tc_fence_after();
-    float qs[NV];  // warps 2..3: e^{gamma_t} (Q S^T)[t][:]
-    {
-      uint32_t r[32];
-      tc::tmem_ld32(t_a + lane_off, r);
+    float qs[NH];  // rows 64..127: e^{gamma_t} (Q S^T)[t][:]
+    if (!producer) {
+      uint32_t r[16], r2[16];
+      tc::tmem_ld16(t_a, r);
+      tc::tmem_ld16(t_a + NV, r2);
       tc::tmem_wait_ld();
-      if (warp < 2) {  // R[t][i] = beta_t (v[t][i] - e^{gamma_t} (K S^T)[t][i])
-        const float eg = t < L ? expf(gsm[t]) : 0.0f, bt = t < L ? gsm[64 + t] : 0.0f;
-        float rr[NV];
 #pragma unroll
-        for (int i = 0; i < NV; ++i) rr[i] = bt * (vc[i] - eg * __uint_as_float(r[i]));
+      for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
+      if (quarter < 2) {  // R[t][i] = beta_t v[t][i] - beta_t e^{gamma_t} (K S^T)[t][i]
+        const float be = t < L ? gsm[64 + t] * eg : 0.0f;
+        float rr[NH];
 #pragma unroll
-        for (int nb = 0; nb < NV / 8; ++nb) {
+        for (int i = 0; i < NH; ++i) rr[i] = t < L ? fmaf(-be, __uint_as_float(r[i]), bvr[i]) : 0.0f;
+#pragma unroll
+        for (int q8 = 0; q8 < 2; ++q8) {
           uint4 hi, lo;
-          tc::split8(rr + nb * 8, hi, lo);
-          const uint32_t off = mnmaj(t, nb, 64);
+          tc::split8(rr + q8 * 8, hi, lo);
+          const uint32_t off = mnmaj(t, (cb >> 3) + q8, 64);
           *reinterpret_cast<uint4*>(r_hi + off) = hi;
           *reinterpret_cast<uint4*>(r_lo + off) = lo;
         }
       } else {
-        const float eg = t < L ? expf(gsm[t]) : 0.0f;
 #pragma unroll
-        for (int i = 0; i < NV; ++i) qs[i] = eg * __uint_as_float(r[i]);
+        for (int i = 0; i < NH; ++i) qs[i] = eg * __uint_as_float(r[i]);
       }
     }
     tc::fence_proxy_async();
@@ -618,48 +765,47 @@ __global__ void __launch_bounds__(128, 1)
     // ---- round 2: [U ; (M o QK^T) U] = [T;P] (128 x 64) x R (K = 64, N = nv) ----------------
     if (tid == 0) {
       tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::idesc_bf16(128, NV, 0, 1);
-      const uint32_t a0[2] = {tc::smem_u32(sg + PBStage::TP), tc::smem_u32(sg + PBStage::TP + TP_TILE)};
-      const uint32_t b0[2] = {tc::smem_u32(r_hi), tc::smem_u32(r_lo)};
-      for (int ks = 0; ks < 4; ++ks)
-        for (int term = 0; term < 3; ++term) {
-          const int ai = term == 2, bi = term == 1;
-          tc::umma_bf16(t_cd, tc::sdesc(a0[ai] + ks * 2 * LBO128, LBO128, 128),
-                        tc::sdesc(b0[bi] + ks * 256, 128, 8 * 128), idesc, (ks | term) != 0);
-        }
+      const uint64_t da[2] = {tc::sdesc(tp0, LBO128, 128), tc::sdesc(tp0 + TP_TILE, LBO128, 128)};
+      const uint64_t db = tc::sdesc(tc::smem_u32(r_hi), 128, 8 * 128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t ao = (uint64_t)((ks * 2 * LBO128) >> 4), bo = (uint64_t)((ks * 256) >> 4);
+        tc::umma_bf16(T_CD, da[0] + ao, db + bo, idesc_kn2, ks != 0);
+        tc::umma_bf16(T_CD, da[1] + ao, db + bo, idesc_kn, 1);
+      }
       tc::umma_commit(tc::smem_u32(&mbar_mma));
     }
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_mma ^= 1;
     tc::tc_fence_after();
-    {
-      uint32_t r[32];
-      tc::tmem_ld32(t_cd + lane_off, r);
+    if (!producer) {
+      uint32_t r[16], r2[16];
+      tc::tmem_ld16(t_cd, r);
+      tc::tmem_ld16(t_cd + NV, r2);
       tc::tmem_wait_ld();
-      if (warp < 2) {  // U-tilde[t][i] = e^{gamma_L - gamma_t} U[t][i]
-        const float f = t < L ? expf(gL - gsm[t]) : 0.0f;
-        float uu[NV];
 #pragma unroll
-        for (int i = 0; i < NV; ++i) uu[i] = f * __uint_as_float(r[i]);
+      for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
+      if (quarter < 2) {  // U-tilde[t][i] = e^{gamma_L - gamma_t} U[t][i]
+        const float f = t < L ? __expf(gL - gsm[t]) : 0.0f;
+        float uu[NH];
 #pragma unroll
-        for (int nb = 0; nb < NV / 8; ++nb) {
+        for (int i = 0; i < NH; ++i) uu[i] = f * __uint_as_float(r[i]);
+#pragma unroll
+        for (int q8 = 0; q8 < 2; ++q8) {
           uint4 hi, lo;
-          tc::split8(uu + nb * 8, hi, lo);
-          const uint32_t off = mnmaj(t, nb, 64);
+          tc::split8(uu + q8 * 8, hi, lo);
+          const uint32_t off = mnmaj(t, (cb >> 3) + q8, 64);
           *reinterpret_cast<uint4*>(r_hi + off) = hi;
           *reinterpret_cast<uint4*>(r_lo + off) = lo;
         }
       } else if (t < L) {  // Y = e^gamma Q S^T + (M o QK^T) U
-        float* yr = y_raw + ((size_t)(t0 + t) * hv + h) * D + i0;
+        float4* yr = reinterpret_cast<float4*>(y_raw + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
 #pragma unroll
-        for (int q4 = 0; q4 < NV / 4; ++q4) {
-          float4 o;
-          o.x = qs[q4 * 4 + 0] + __uint_as_float(r[q4 * 4 + 0]);
-          o.y = qs[q4 * 4 + 1] + __uint_as_float(r[q4 * 4 + 1]);
-          o.z = qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]);
-          o.w = qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]);
-          *reinterpret_cast<float4*>(yr + q4 * 4) = o;
-        }
+        for (int q4 = 0; q4 < NH / 4; ++q4)
+          yr[q4] = make_float4(qs[q4 * 4 + 0] + __uint_as_float(r[q4 * 4 + 0]),
+                               qs[q4 * 4 + 1] + __uint_as_float(r[q4 * 4 + 1]),
+                               qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]),
+                               qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]));
       }
     }
     tc::fence_proxy_async();
@@ -669,42 +815,41 @@ __global__ void __launch_bounds__(128, 1)
     // ---- round 3: K^T U-tilde: A = MN-major view of the K rows (M = 128 key comps, K = 64 tokens)
     if (tid == 0) {
       tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::idesc_bf16(128, NV, 1, 1);
-      const uint32_t a0[2] = {tc::smem_u32(sg + PBStage::KQ), tc::smem_u32(sg + PBStage::KQ + KQ_TILE)};
-      const uint32_t b0[2] = {tc::smem_u32(r_hi), tc::smem_u32(r_lo)};
-      for (int ks = 0; ks < 4; ++ks)
-        for (int term = 0; term < 3; ++term) {
-          const int ai = term == 2, bi = term == 1;
-          tc::umma_bf16(t_e, tc::sdesc(a0[ai] + ks * 256, 128, LBO128),
-                        tc::sdesc(b0[bi] + ks * 256, 128, 8 * 128), idesc, (ks | term) != 0);
-        }
+      const uint64_t da[2] = {tc::sdesc(kq0, 128, LBO128), tc::sdesc(kq0 + KQ_TILE, 128, LBO128)};
+      const uint64_t db = tc::sdesc(tc::smem_u32(r_hi), 128, 8 * 128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t o = (uint64_t)((ks * 256) >> 4);
+        tc::umma_bf16(T_E, da[0] + o, db + o, idesc_mn2, ks != 0);
+        tc::umma_bf16(T_E, da[1] + o, db + o, idesc_mn, 1);
+      }
       tc::umma_commit(tc::smem_u32(&mbar_mma));
     }
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_mma ^= 1;
     tc::tc_fence_after();
-    {
-      uint32_t r[32];
-      tc::tmem_ld32(t_e + lane_off, r);
+    if (!producer) {
+      uint32_t r[16], r2[16];
+      tc::tmem_ld16(t_e, r);
+      tc::tmem_ld16(t_e + NV, r2);
       tc::tmem_wait_ld();
-      const float eL = expf(gL);
+      const float eL = __expf(gL);
 #pragma unroll
-      for (int i = 0; i < NV; ++i) S[i] = fmaf(eL, S[i], __uint_as_float(r[i]));
+      for (int i = 0; i < NH; ++i) S[i] = fmaf(eL, S[i], __uint_as_float(r[i]) + __uint_as_float(r2[i]));
+      write_s_tile();
     }
-    write_s_tile();
     tc::fence_proxy_async();
     tc::tc_fence_before();
     __syncthreads();
     if (s_abort) { aborted = true; break; }
   }
-  // final state slice (thread j' writes column j' of rows i0 .. i0 + nv)
-  if (!aborted) {
+  if (!aborted && !producer) {
 #pragma unroll
-    for (int i = 0; i < NV; ++i) final_state[sbase + (size_t)i * D + tid] = S[i];
+    for (int i = 0; i < NH; ++i) final_state[sbase + (size_t)(cb + i) * D + row] = S[i];
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tbase, 128);
+  if (warp == 0) tc::tmem_dealloc(tbase, 256);
 }
 
 }  // namespace gdn
