@@ -350,9 +350,9 @@ def gpu_arm(args):
     dom = max(prof.items(), key=lambda kv: kv[1][1])
     dom_name, (dom_n, dom_ms) = dom
     dom_avg_s = dom_ms / dom_n / 1e3
-    if dom_name.startswith("chunk_phaseB"):
+    if dom_name.startswith("chunk_phaseB") or dom_name.startswith("chunk_scan"):
         work, unit_kind = FLOP_PHASEB_PER_TOKEN * T, "flop"
-    elif dom_name.startswith("chunk_phaseA"):
+    elif dom_name.startswith("chunk_phaseA") or dom_name.startswith("chunk_prep"):
         work, unit_kind = FLOP_PHASEA_PER_TOKEN * T, "flop"
     else:
         work, unit_kind = None, None
@@ -453,7 +453,7 @@ def gpu_arm(args):
     out = {
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16x3/f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": 1, "T": T, "h_qk": 16, "h_v": 32, "d": 128, "chunk": 64,
                    "in_dtype": "bf16", "out_dtype": "bf16", "state_dtype": "f32",
                    "l2": f"{n_sets} rotating input sets of 97 MiB (> 126 MB L2)",

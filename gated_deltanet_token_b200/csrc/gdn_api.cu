@@ -188,7 +188,7 @@ void launch_prologue(const Dims& kd, int max_chunks, const ChunkEntry* tab, cons
 void launch_epilogue(const Dims& kd, const float* yraw, const void* z, const float* norm_w, void* y,
                      cudaStream_t s) {
   const long rows = (long)kd.total_tokens * kd.h_v;
-  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  const unsigned blocks = (unsigned)((rows + 8 * EPI_ROWS - 1) / (8 * EPI_ROWS));
   if (kd.in_bf16 && kd.out_bf16) k_epilogue<true, true><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);
   else if (kd.in_bf16) k_epilogue<true, false><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);
   else if (kd.out_bf16) k_epilogue<false, true><<<blocks, 256, 0, s>>>(kd, yraw, z, norm_w, y, rows);

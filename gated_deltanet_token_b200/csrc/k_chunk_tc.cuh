@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 // row reduce the L2 norm with two shuffles, and consecutive lanes store consecutive
 // 16-byte chunks of the tile (coalesced).
 // ======================================================================================
-__global__ void __launch_bounds__(256) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab,
+__global__ void __launch_bounds__(256, 4) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab,
                                                      const uint16_t* __restrict__ q,
                                                      const uint16_t* __restrict__ k,
                                                      const uint16_t* __restrict__ v,

@@ -151,28 +151,49 @@ __global__ void __launch_bounds__(256) k_prologue(Dims d, const ChunkEntry* __re
 }
 
 // ---- K5: gated RMSNorm epilogue ----------------------------------------------------------
-// One warp per (token, value head): y = y_raw / sqrt(mean(y_raw^2) + eps) * norm_w * silu(z)
-// (field guide §02: RMS-normalise y, then gate with SiLU(z)).
+// y = y_raw / sqrt(mean(y_raw^2) + eps) * norm_w * silu(z) per (token, value head) (field
+// guide §02: RMS-normalise y, then gate with SiLU(z)).  One warp per EPI_ROWS consecutive
+// rows, all loads issued first so the rows' memory latencies overlap.
+constexpr int EPI_ROWS = 4;
+
 template <bool IN_BF16, bool OUT_BF16>
 __global__ void __launch_bounds__(256) k_epilogue(Dims d, const float* __restrict__ y_raw,
                                                   const void* __restrict__ z,
                                                   const float* __restrict__ norm_w, void* __restrict__ y,
                                                   long rows) {
-  const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
+  const long row0 = ((long)blockIdx.x * 8 + (threadIdx.x >> 5)) * EPI_ROWS;
+  if (row0 >= rows) return;
   const int c0 = (threadIdx.x & 31) * 4;
-  const size_t base = (size_t)row * D + c0;
-  const float4 yr = *reinterpret_cast<const float4*>(y_raw + base);
-  const float ss = warp_sum(yr.x * yr.x + yr.y * yr.y + yr.z * yr.z + yr.w * yr.w);
-  const float inv = 1.0f / sqrtf(ss * (1.0f / D) + d.rms_eps);
-  const float4 zz = load4<IN_BF16>(z, base);
+  float4 yr[EPI_ROWS], zz[EPI_ROWS];
+#pragma unroll
+  for (int r = 0; r < EPI_ROWS; ++r) {
+    if (row0 + r < rows) {
+      const size_t base = (size_t)(row0 + r) * D + c0;
+      yr[r] = *reinterpret_cast<const float4*>(y_raw + base);
+      zz[r] = load4<IN_BF16>(z, base);
+    } else {
+      yr[r] = zz[r] = make_float4(0, 0, 0, 0);
+    }
+  }
   const float4 nw = *reinterpret_cast<const float4*>(norm_w + c0);
-  float4 o;
-  o.x = yr.x * inv * nw.x * silu_f(zz.x);
-  o.y = yr.y * inv * nw.y * silu_f(zz.y);
-  o.z = yr.z * inv * nw.z * silu_f(zz.z);
-  o.w = yr.w * inv * nw.w * silu_f(zz.w);
-  store4<OUT_BF16>(y, base, o);
+  float ss[EPI_ROWS];
+#pragma unroll
+  for (int r = 0; r < EPI_ROWS; ++r) ss[r] = yr[r].x * yr[r].x + yr[r].y * yr[r].y + yr[r].z * yr[r].z + yr[r].w * yr[r].w;
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int r = 0; r < EPI_ROWS; ++r) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], o);
+#pragma unroll
+  for (int r = 0; r < EPI_ROWS; ++r) {
+    if (row0 + r >= rows) break;
+    const float inv = 1.0f / sqrtf(ss[r] * (1.0f / D) + d.rms_eps);
+    float4 o;
+    o.x = yr[r].x * inv * nw.x * silu_f(zz[r].x);
+    o.y = yr[r].y * inv * nw.y * silu_f(zz[r].y);
+    o.z = yr[r].z * inv * nw.z * silu_f(zz[r].z);
+    o.w = yr[r].w * inv * nw.w * silu_f(zz[r].w);
+    store4<OUT_BF16>(y, (size_t)(row0 + r) * D + c0, o);
+  }
 }
 
 }  // namespace gdn
