@@ -134,6 +134,9 @@ int check_dims(const gdn_dims_t* d, bool decode) {
   if (2 * d->h_qk + d->h_v > 65535 || d->h_v > 65535) return GDN_ERR_SHAPE;
   if (decode && d->total_tokens != d->n_seqs) return GDN_ERR_SHAPE;
   if ((int64_t)d->total_tokens / CH + d->n_seqs + 1 > INT32_MAX) return GDN_ERR_SHAPE;
+  // chunk slots index grid.y of the tensor-core kernels
+  if (!decode && d->in_dtype == GDN_DTYPE_BF16 && (int64_t)d->total_tokens / CH + d->n_seqs + 1 > 65535)
+    return GDN_ERR_SHAPE;
   if (!isfinite(d->q_scale) || !(d->l2_eps >= 0.0f) || !(d->rms_eps >= 0.0f)) return GDN_ERR_SHAPE;
   if ((d->in_dtype != GDN_DTYPE_F32 && d->in_dtype != GDN_DTYPE_BF16) ||
       (d->out_dtype != GDN_DTYPE_F32 && d->out_dtype != GDN_DTYPE_BF16))
@@ -155,16 +158,25 @@ Dims kdims(const gdn_dims_t* d) {
   return k;
 }
 
+int g_num_sms = 148;  // SM count of the current device (set by configure_device)
+
 // Opt the large-shared-memory kernels in once per device.
 int configure_device() {
   static std::atomic<uint64_t> done_mask{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
   const uint64_t bit = 1ull << (dev & 63);
+  {
+    int nsm = 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return GDN_ERR_CUDA;
+    g_num_sms = nsm > 0 ? nsm : 148;
+  }
   if (done_mask.load() & bit) return GDN_OK;
   if (cudaFuncSetAttribute(k_phaseA_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM) !=
           cudaSuccess ||
       cudaFuncSetAttribute(k_phaseB_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PB_SMEM) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(k_prologue_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PRO_SMEM) !=
           cudaSuccess ||
       cudaFuncSetAttribute(k_chunkprep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_TC_SMEM) !=
           cudaSuccess ||
@@ -256,12 +268,15 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     if (d->total_tokens > 0) {
       {
         ProfScope p("prologue_tc", s);
-        k_prologue_tc<<<dim3(L.max_chunks, 2 * d->h_qk + d->h_v), 256, 0, s>>>(
-            kd, tab, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-            static_cast<const uint16_t*>(v), b, conv_w, kq, F(L.bv));
+        const int ngroups = 2 * ((d->h_qk + PRO_HG - 1) / PRO_HG) + (d->h_v + PRO_HG - 1) / PRO_HG;
+        const int nitems = ngroups * 2 * L.max_chunks;
+        const int grid = nitems < g_num_sms ? nitems : g_num_sms;
+        k_prologue_tc<<<grid, 512, PRO_SMEM, s>>>(kd, tab, nitems, static_cast<const uint16_t*>(q),
+                                                  static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+                                                  b, conv_w, kq, F(L.bv));
       }
       ProfScope p("chunk_prep_tc", s);
-      k_chunkprep_tc<<<dim3(L.max_chunks, d->h_qk), 256, PA_TC_SMEM, s>>>(kd, tab, a, b, A_log, dt_bias, kq, tp,
+      k_chunkprep_tc<<<dim3(d->h_qk, L.max_chunks), 256, PA_TC_SMEM, s>>>(kd, tab, a, b, A_log, dt_bias, kq, tp,
                                                                           F(L.gb));
     }
     {

@@ -61,6 +61,12 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+// Hardware-approximate forms (ex2.approx, rcp.approx: a few ulp per factor) for the
+// streaming kernels of the bf16 path and the output gate, where operand rounding (bf16 hi/lo
+// products, ~2^-17) or the output tolerance dominates by orders of magnitude.  For x far
+// below zero e^-x overflows and the quotient goes to 0, the limit of silu and sigmoid.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
 __device__ __forceinline__ float softplus_f(float x) {
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));

@@ -165,118 +165,229 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 }
 
 // ======================================================================================
-// Prologue of the tensor-core path (K1): one CTA per (chunk, stream unit), 256 threads.
-//   unit < h_qk:       K rows (0..63) of the [K;Q] tile of QK head `unit`
-//   unit < 2 h_qk:     Q rows (64..127) of the tile of QK head `unit - h_qk`
-//   otherwise:         beta * v of value head `unit - 2 h_qk`, as four contiguous 32-column
-//                      fp32 slices [4][64][32] (one per phase-B CTA)
+// Prologue of the tensor-core path (K1).  Persistent: each CTA walks work items (head group,
+// half chunk) with a stride of the grid size.  A group is up to 8 heads of one stream -- q,
+// k or value heads -- whose slices of a token row are contiguous (2 KB).  The next item's
+// 32 + 3 token rows and conv taps are bulk-copied into the other of two shared-memory stages
+// while the current item is computed, so loads overlap compute.  16 warps: warp w works on
+// head w % 8 of the group and on token blocks 16 (w / 8) .. + 15 of the half chunk.
+//   q / k head j: rows 64..127 / 0..63 of the [K;Q] hi/lo tile of QK head j
+//   value head h: beta * v as four contiguous 32-column fp32 slices [4][64][32]
 // Width-4 causal conv and SiLU ("Qwen3.8-Flash-Next" technical report, Fig. 2; field
-// guide §02), L2 norm of q and k (Fig. 2), beta = sigmoid(b).  q/k warps: 8 tokens per
-// warp, lane = (row r = lane % 8, 8-channel groups lane / 8 + 4 i); the four lanes of a
-// row reduce the L2 norm with two shuffles, and consecutive lanes store consecutive
-// 16-byte chunks of the tile (coalesced).
+// guide §02), L2 norm of q and k (Fig. 2), beta = sigmoid(b).  q/k lanes: token r = lane % 4,
+// 8-channel groups lane / 4 and lane / 4 + 8; the eight lanes of a token reduce the L2 norm
+// with three shuffles and consecutive lanes store consecutive 16-byte chunks.  Every row of
+// a used chunk slot is written (rows past the chunk's length as zeros): phase B multiplies
+// those K rows by zero weights, so stale workspace bits must not survive.
 // ======================================================================================
-__global__ void __launch_bounds__(256, 4) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab,
-                                                     const uint16_t* __restrict__ q,
-                                                     const uint16_t* __restrict__ k,
-                                                     const uint16_t* __restrict__ v,
-                                                     const float* __restrict__ b,
-                                                     const float* __restrict__ conv_w,
-                                                     uint8_t* __restrict__ kq_ws, float* __restrict__ bv_ws) {
-  const ChunkEntry e = tab[blockIdx.x];
-  if (e.len == 0) return;
-  const int u = blockIdx.y, hq = d.h_qk, hv = d.h_v, L = e.len;
+constexpr int PRO_HG = 8;                  // heads per work item
+constexpr int PRO_TOK = 32;                // tokens per work item (half a chunk)
+constexpr int PRO_ROWS = PRO_TOK + 3;      // with the conv history
+constexpr uint32_t PRO_ROWS_BYTES = PRO_ROWS * PRO_HG * D * 2;
+constexpr uint32_t PRO_W_BYTES = PRO_HG * D * 16;
+constexpr uint32_t PRO_STAGE = PRO_ROWS_BYTES + PRO_W_BYTES;
+constexpr size_t PRO_SMEM = 2 * (size_t)PRO_STAGE;
+
+struct ProItem {
+  ChunkEntry e;
+  int chunk, tb0, stream, h0, nh, nheads;
+  size_t ch0;  // first conv channel of the group
+};
+
+__device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry* tab, int it, int ngroups) {
+  ProItem w;
+  const int grp = it % ngroups, hc = it / ngroups;
+  w.chunk = hc >> 1;
+  w.tb0 = (hc & 1) * PRO_TOK;
+  w.e = tab[w.chunk];
+  const int hq = d.h_qk, nqg = (hq + PRO_HG - 1) / PRO_HG;
+  w.stream = grp < nqg ? 0 : grp < 2 * nqg ? 1 : 2;
+  w.nheads = w.stream == 2 ? d.h_v : hq;
+  w.h0 = (w.stream == 2 ? grp - 2 * nqg : grp - w.stream * nqg) * PRO_HG;
+  w.nh = min(PRO_HG, w.nheads - w.h0);
+  w.ch0 = w.stream == 0 ? (size_t)w.h0 * D : w.stream == 1 ? (size_t)(hq + w.h0) * D
+                                                           : (size_t)2 * hq * D + (size_t)w.h0 * D;
+  return w;
+}
+
+__global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab, int nitems,
+                                                        const uint16_t* __restrict__ q,
+                                                        const uint16_t* __restrict__ k,
+                                                        const uint16_t* __restrict__ v,
+                                                        const float* __restrict__ b,
+                                                        const float* __restrict__ conv_w,
+                                                        uint8_t* __restrict__ kq_ws, float* __restrict__ bv_ws) {
+  const int hq = d.h_qk, hv = d.h_v;
+  const int ngroups = 2 * ((hq + PRO_HG - 1) / PRO_HG) + (hv + PRO_HG - 1) / PRO_HG;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // the unit's 128 channels x 4 taps, staged once
-  __shared__ float4 wsm[D];
-  const size_t chu = u < hq ? (size_t)(hq + u) * D : u < 2 * hq ? (size_t)(u - hq) * D
-                                                                 : (size_t)2 * hq * D + (size_t)(u - 2 * hq) * D;
-  if (tid < D) wsm[tid] = *reinterpret_cast<const float4*>(conv_w + (chu + tid) * 4);
+  const int hw = warp & (PRO_HG - 1), tsplit = warp >> 3;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t mbar[2];
+  __shared__ int s_abort;
+  if (tid == 0) {
+    s_abort = 0;
+    tc::mbar_init(tc::smem_u32(&mbar[0]), 1);
+    tc::mbar_init(tc::smem_u32(&mbar[1]), 1);
+    tc::fence_mbar_init();
+  }
   __syncthreads();
-  if (u < 2 * hq) {
-    const bool isq = u >= hq;
-    const int j = isq ? u - hq : u;
-    const uint16_t* src = isq ? q : k;
-    const int r = lane & 7, g0 = lane >> 3;  // row within the warp's 8 tokens; first channel group
-    const int t = warp * 8 + r;              // chunk-relative token
-    // taps for the lane's 32 channels: groups g0, g0 + 4, g0 + 8, g0 + 12 (8 channels each)
-    float acc[4][8];
+  // issue the copies of item `it` into stage `st` (thread 0); unused chunk slots copy nothing
+  auto issue = [&](int it, int st) -> bool {  // true if copies were issued
+    const ProItem w = pro_item(d, tab, it, ngroups);
+    if (w.e.len == 0) return false;
+    const uint16_t* src = w.stream == 0 ? q : w.stream == 1 ? k : v;
+    const uint32_t row_bytes = (uint32_t)w.nh * D * 2;
+    uint32_t bytes = (uint32_t)w.nh * D * 16;
+    for (int r = 0; r < PRO_ROWS; ++r) {
+      const int tcr = w.tb0 - 3 + r;
+      if (tcr < w.e.len && (long)w.e.t0 + tcr >= w.e.seq_start) bytes += row_bytes;
+    }
+    const uint32_t bar = tc::smem_u32(&mbar[st]);
+    uint8_t* base = sm + (size_t)st * PRO_STAGE;
+    tc::mbar_arrive_expect_tx(bar, bytes);
+    tc::bulk_g2s(tc::smem_u32(base + PRO_ROWS_BYTES), conv_w + w.ch0 * 4, (uint32_t)w.nh * D * 16, bar);
+    for (int r = 0; r < PRO_ROWS; ++r) {
+      const int tcr = w.tb0 - 3 + r;
+      const long tg = (long)w.e.t0 + tcr;
+      if (tcr < w.e.len && tg >= w.e.seq_start)
+        tc::bulk_g2s(tc::smem_u32(base) + r * row_bytes, src + ((size_t)tg * w.nheads + w.h0) * D, row_bytes, bar);
+    }
+    return true;
+  };
+  bool pending[2] = {false, false};  // (thread 0) copies in flight per stage
+  if (tid == 0 && (int)blockIdx.x < nitems) pending[0] = issue(blockIdx.x, 0);
+  uint32_t parity[2] = {0, 0};
+  int n = 0;
+  for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+    const int st = n & 1;
+    const ProItem w = pro_item(d, tab, it, ngroups);
+    if (tid == 0 && it + (int)gridDim.x < nitems) pending[st ^ 1] = issue(it + gridDim.x, st ^ 1);
+    if (w.e.len == 0) {
+      __syncthreads();
+      continue;
+    }
+    if (!tc::mbar_wait(tc::smem_u32(&mbar[st]), parity[st])) s_abort = 1;
+    parity[st] ^= 1;
+    if (tid == 0) pending[st] = false;
+    __syncthreads();  // the abort decision is uniform
+    if (s_abort) break;
+    const uint8_t* base = sm + (size_t)st * PRO_STAGE;
+    const float4* wsm = reinterpret_cast<const float4*>(base + PRO_ROWS_BYTES) + hw * D;
+    const uint16_t* hrow = reinterpret_cast<const uint16_t*>(base) + (size_t)hw * D;  // this head in a row
+    const int L = w.e.len, tb0 = w.tb0, nh = w.nh, head = w.h0 + hw;
+    auto row_ok = [&](int r) {  // smem row r holds a token inside the sequence and the chunk
+      const int tcr = tb0 - 3 + r;
+      return tcr < L && (long)w.e.t0 + tcr >= w.e.seq_start;
+    };
+    if (hw < nh) {
+      if (w.stream < 2) {
+        // lane: token r = lane % 4 of a 4-token block, channel groups g0 = lane / 4 and g0 + 8
+        const int r = lane & 3, g0 = lane >> 2;
+        uint8_t* tile = kq_ws + ((size_t)w.chunk * hq + head) * KQ_BYTES;
+        const float scale = w.stream == 0 ? d.q_scale : 1.0f;
+#pragma unroll 1
+        for (int blk = tsplit * (PRO_TOK / 2); blk < (tsplit + 1) * (PRO_TOK / 2); blk += 4) {
+          const int t = tb0 + blk + r;  // chunk-relative token
+          float acc[2][8];
+          bool okt[4];
 #pragma unroll
-    for (int gi = 0; gi < 4; ++gi)
+          for (int tap = 0; tap < 4; ++tap) okt[tap] = row_ok(blk + r + tap);  // row of token t - 3 + tap
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[gi][c] = 0.0f;
+          for (int gi = 0; gi < 2; ++gi) {
+            const int cg = (g0 + 8 * gi) * 8;
+            float4 w4[8];  // the group's 8 channels x 4 taps
 #pragma unroll
-    for (int tap = 0; tap < 4; ++tap) {
-      const long tg = (long)e.t0 + t - 3 + tap;
-      const bool ok = t < L && tg >= e.seq_start;
+            for (int c = 0; c < 8; ++c) w4[c] = wsm[cg + c];
 #pragma unroll
-      for (int gi = 0; gi < 4; ++gi) {
-        const int cg = (g0 + 4 * gi) * 8;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (ok) x = *reinterpret_cast<const uint4*>(src + ((size_t)tg * hq + j) * D + cg);
-        const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+            for (int c = 0; c < 8; ++c) acc[gi][c] = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float xv = bf2f(c & 1 ? wd[c >> 1] >> 16 : wd[c >> 1] & 0xffffu);
-          acc[gi][c] = fmaf(comp(wsm[cg + c], tap), xv, acc[gi][c]);
+            for (int tap = 0; tap < 4; ++tap) {
+              if (!okt[tap]) continue;
+              const uint4 x = *reinterpret_cast<const uint4*>(hrow + (size_t)(blk + r + tap) * nh * D + cg);
+              const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                acc[gi][c] = fmaf(comp(w4[c], tap), bf2f(c & 1 ? wd[c >> 1] >> 16 : wd[c >> 1] & 0xffffu), acc[gi][c]);
+            }
+          }
+          float ss0 = 0.0f, ss1 = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            acc[0][c] = silu_fast(acc[0][c]);
+            acc[1][c] = silu_fast(acc[1][c]);
+            ss0 = fmaf(acc[0][c], acc[0][c], ss0);
+            ss1 = fmaf(acc[1][c], acc[1][c], ss1);
+          }
+          float sst = ss0 + ss1;
+          sst += __shfl_xor_sync(0xffffffffu, sst, 4);
+          sst += __shfl_xor_sync(0xffffffffu, sst, 8);
+          sst += __shfl_xor_sync(0xffffffffu, sst, 16);
+          const float inv = t < L ? scale * rsqrtf(sst + d.l2_eps) : 0.0f;
+          const int row = (w.stream == 0 ? 64 : 0) + t;
+#pragma unroll
+          for (int gi = 0; gi < 2; ++gi) {
+            float x8[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) x8[c] = acc[gi][c] * inv;
+            uint4 hi, lo;
+            tc::split8(x8, hi, lo);
+            const uint32_t off = kmaj128(row, (g0 + 8 * gi) * 8);
+            *reinterpret_cast<uint4*>(tile + off) = hi;
+            *reinterpret_cast<uint4*>(tile + KQ_TILE + off) = lo;
+          }
+        }
+      } else {
+        const int c0 = lane * 4;
+        float wv[4][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 t4 = wsm[c0 + c];
+          wv[c][0] = t4.x; wv[c][1] = t4.y; wv[c][2] = t4.z; wv[c][3] = t4.w;
+        }
+        float* out = bv_ws + ((size_t)w.chunk * hv + head) * (BV_BYTES / 4) + (size_t)(c0 / TC_NV) * (BV_SLICE / 4) +
+                     (c0 % TC_NV);
+#pragma unroll 1
+        for (int blk = tsplit * (PRO_TOK / 2); blk < (tsplit + 1) * (PRO_TOK / 2); blk += 8) {
+          float bt[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int t = tb0 + blk + i;
+            bt[i] = t < L ? __ldg(b + (size_t)(w.e.t0 + t) * hv + head) : 0.0f;
+          }
+          uint2 x[11];  // raw bf16 of 4 channels, rows t - 3 .. t + 7
+#pragma unroll
+          for (int p = 0; p < 11; ++p) {
+            const int rr = blk + p;
+            x[p] = row_ok(rr) ? *reinterpret_cast<const uint2*>(hrow + (size_t)rr * nh * D + c0) : make_uint2(0, 0);
+          }
+          auto xv = [&](int p, int c) {
+            const uint32_t wd = c < 2 ? x[p].x : x[p].y;
+            return bf2f(c & 1 ? wd >> 16 : wd & 0xffffu);
+          };
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int t = tb0 + blk + i;
+            const float beta = t < L ? sigmoid_fast(bt[i]) : 0.0f;
+            float r4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float acc = fmaf(wv[c][3], xv(i + 3, c),
+                                     fmaf(wv[c][2], xv(i + 2, c), fmaf(wv[c][1], xv(i + 1, c), wv[c][0] * xv(i, c))));
+              r4[c] = beta * silu_fast(acc);
+            }
+            *reinterpret_cast<float4*>(out + t * TC_NV) = make_float4(r4[0], r4[1], r4[2], r4[3]);
+          }
         }
       }
     }
-    float ss = 0.0f;
-#pragma unroll
-    for (int gi = 0; gi < 4; ++gi)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float y = acc[gi][c] / (1.0f + __expf(-acc[gi][c]));
-        acc[gi][c] = y;
-        ss = fmaf(y, y, ss);
-      }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-    const float inv = t < L ? (isq ? d.q_scale : 1.0f) * rsqrtf(ss + d.l2_eps) : 0.0f;
-    uint8_t* tile = kq_ws + ((size_t)blockIdx.x * hq + j) * KQ_BYTES;
-    const int row = (isq ? 64 : 0) + t;
-#pragma unroll
-    for (int gi = 0; gi < 4; ++gi) {
-      float x8[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) x8[c] = acc[gi][c] * inv;
-      uint4 hi, lo;
-      tc::split8(x8, hi, lo);
-      const uint32_t off = kmaj128(row, (g0 + 4 * gi) * 8);
-      *reinterpret_cast<uint4*>(tile + off) = hi;
-      *reinterpret_cast<uint4*>(tile + KQ_TILE + off) = lo;
-    }
-  } else {
-    const int h = u - 2 * hq;
-    const int c0 = lane * 4, tb = warp * 8;
-    float w[4][4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float4 t4 = wsm[c0 + c];
-      w[c][0] = t4.x; w[c][1] = t4.y; w[c][2] = t4.z; w[c][3] = t4.w;
-    }
-    float4 x[11];
-#pragma unroll
-    for (int p = 0; p < 11; ++p) {
-      const int tcr = tb - 3 + p;
-      const long tg = (long)e.t0 + tcr;
-      const bool ok = tcr < L && tg >= e.seq_start;
-      x[p] = ok ? load4<true>(v, ((size_t)tg * hv + h) * D + c0) : make_float4(0, 0, 0, 0);
-    }
-    float* out = bv_ws + ((size_t)blockIdx.x * hv + h) * (BV_BYTES / 4) + (size_t)(c0 / TC_NV) * (BV_SLICE / 4);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int t = tb + i;
-      const float bt = t < L ? sigmoid_f(b[(size_t)(e.t0 + t) * hv + h]) : 0.0f;
-      float r4[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float acc = fmaf(w[c][3], comp(x[i + 3], c),
-                               fmaf(w[c][2], comp(x[i + 2], c), fmaf(w[c][1], comp(x[i + 1], c), w[c][0] * comp(x[i], c))));
-        r4[c] = bt * (acc / (1.0f + __expf(-acc)));
-      }
-      *reinterpret_cast<float4*>(out + t * TC_NV + (c0 % TC_NV)) = make_float4(r4[0], r4[1], r4[2], r4[3]);
+    tc::fence_proxy_async();
+    __syncthreads();  // this stage is free for the item after next
+  }
+  if (s_abort) {  // record, and let copies still in flight land (bounded) before leaving
+    if (tid == 0) {
+      atomicExch(&g_gdn_status, -7);
+      for (int q2 = 0; q2 < 2; ++q2)
+        if (pending[q2]) (void)tc::mbar_wait(tc::smem_u32(&mbar[q2]), parity[q2]);
     }
   }
 }
@@ -286,36 +397,34 @@ __global__ void __launch_bounds__(256, 4) k_prologue_tc(Dims d, const ChunkEntry
 // ======================================================================================
 constexpr int PA_P = 68;  // pitch (floats) of the fp32 64 x 64 matrices of phase A
 constexpr uint32_t PA_MAT = 64 * PA_P * 4;
-// [0, 64K): [K;Q] tile (hi | lo), later the P operands: [Mq_a; Mq_b] (K-major, 128 x 64) hi | lo
-// and [T_a | T_b] (MN-major, K = 64, N = 128) hi | lo; then KK, QK, A, T_a, T_b (fp32), gates.
-constexpr uint32_t PA_OFF_KK = 65536;
-constexpr uint32_t PA_OFF_QK = PA_OFF_KK + PA_MAT;
-constexpr uint32_t PA_OFF_A = PA_OFF_QK + PA_MAT;  // two heads
-constexpr uint32_t PA_OFF_T = PA_OFF_A + 2 * PA_MAT;  // two heads
-constexpr uint32_t PA_OFF_G = PA_OFF_T + 2 * PA_MAT;
+// [0, 64K): [K;Q] tile (hi | lo); after [K;Q]K^T it holds the P operands: [Mq_a; Mq_b]
+// (K-major, 128 x 64) hi | lo and [T_a | T_b] (MN-major, K = 64, N = 128) hi | lo.  Then A and T
+// (fp32, one value head at a time) and the gates of the pair.
+constexpr uint32_t PA_OFF_A = 65536;
+constexpr uint32_t PA_OFF_T = PA_OFF_A + PA_MAT;
+constexpr uint32_t PA_OFF_G = PA_OFF_T + PA_MAT;
 constexpr size_t PA_TC_SMEM = PA_OFF_G + 4 * 64 * 4;
-static_assert(PA_TC_SMEM <= 232448, "phase-A shared memory");
+static_assert(PA_TC_SMEM <= 113 * 1024, "two phase-A CTAs per SM");
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
     k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
                    uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
-  const ChunkEntry e = tab[blockIdx.x];
+  const int chunk = blockIdx.y;  // head-fastest grid: concurrent CTAs read adjacent tiles
+  const ChunkEntry e = tab[chunk];
   if (e.len == 0) return;
-  const int j = blockIdx.y, hq = d.h_qk, hv = d.h_v, G = hv / hq, L = e.len;
+  const int j = blockIdx.x, hq = d.h_qk, hv = d.h_v, G = hv / hq, L = e.len;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* kq_hi = sm;
   uint8_t* kq_lo = sm + KQ_TILE;
-  uint8_t* pa_hi = sm;             // [Mq_a; Mq_b] operand (aliases the [K;Q] tile)
+  uint8_t* pa_hi = sm;          // [Mq_a; Mq_b] operand (aliases the [K;Q] tile)
   uint8_t* pa_lo = sm + 16384;
-  uint8_t* pb_hi = sm + 32768;     // [T_a | T_b] operand
+  uint8_t* pb_hi = sm + 32768;  // [T_a | T_b] operand
   uint8_t* pb_lo = sm + 49152;
-  float* KK = reinterpret_cast<float*>(sm + PA_OFF_KK);
-  float* QK = reinterpret_cast<float*>(sm + PA_OFF_QK);
-  float* Amat = reinterpret_cast<float*>(sm + PA_OFF_A);  // [2][64][PA_P]
-  float* Tm = reinterpret_cast<float*>(sm + PA_OFF_T);    // [2][64][PA_P]
+  float* Am = reinterpret_cast<float*>(sm + PA_OFF_A);
+  float* T = reinterpret_cast<float*>(sm + PA_OFF_T);
   float* gs = reinterpret_cast<float*>(sm + PA_OFF_G);  // [2][64] gamma
   float* bs = gs + 128;                                 // [2][64] beta
   __shared__ uint64_t mbar;
@@ -338,53 +447,11 @@ __global__ void __launch_bounds__(256, 1)
   if (tid == 0) {  // the [K;Q] tile written by the prologue
     const uint32_t bar = tc::smem_u32(&mbar);
     tc::mbar_arrive_expect_tx(bar, KQ_BYTES);
-    tc::bulk_g2s(tc::smem_u32(sm), kq_ws + ((size_t)blockIdx.x * hq + j) * KQ_BYTES, KQ_BYTES, bar);
+    tc::bulk_g2s(tc::smem_u32(sm), kq_ws + ((size_t)chunk * hq + j) * KQ_BYTES, KQ_BYTES, bar);
   }
-  if (!tc::mbar_wait(tc::smem_u32(&mbar), 0)) {
-    s_abort = 1;
-    atomicExch(&g_gdn_status, -7);
-  }
-  __syncthreads();
-  tc::tc_fence_after();
-  if (tid == 0 && !s_abort) {
-    // D[128 x 64] = [K;Q] (K-major, 128 x 128) x K^T (B = rows 0..63 of the tile, K-major)
-    constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
-    const uint32_t base[2] = {tc::smem_u32(kq_hi), tc::smem_u32(kq_lo)};
-    for (int ks = 0; ks < 8; ++ks)
-      for (int term = 0; term < 3; ++term) {
-        const int ai = term == 2, bi = term == 1;
-        tc::umma_bf16(tbase, tc::sdesc(base[ai] + ks * 2 * LBO128, LBO128, 128),
-                      tc::sdesc(base[bi] + ks * 2 * LBO128, LBO128, 128), idesc, (ks | term) != 0);
-      }
-    tc::umma_commit(tc::smem_u32(&mbar));
-  }
-  if (!s_abort && !tc::mbar_wait(tc::smem_u32(&mbar), 1)) {
-    s_abort = 1;
-    atomicExch(&g_gdn_status, -7);
-  }
-  tc::tc_fence_after();
-  if (warp < 4) {  // TMEM rows 0..63: K K^T, rows 64..127: Q K^T (one row per thread)
-    uint32_t r0[32], r1[32];
-    const uint32_t ta = tbase + ((uint32_t)(warp * 32) << 16);
-    tc::tmem_ld32(ta, r0);
-    tc::tmem_ld32(ta + 32, r1);
-    tc::tmem_wait_ld();
-    float* dst = (tid < 64 ? KK : QK) + (tid & 63) * PA_P;
-#pragma unroll
-    for (int c = 0; c < 32; c += 4) {
-      *reinterpret_cast<float4*>(dst + c) = make_float4(__uint_as_float(r0[c]), __uint_as_float(r0[c + 1]),
-                                                        __uint_as_float(r0[c + 2]), __uint_as_float(r0[c + 3]));
-      *reinterpret_cast<float4*>(dst + 32 + c) = make_float4(__uint_as_float(r1[c]), __uint_as_float(r1[c + 1]),
-                                                             __uint_as_float(r1[c + 2]), __uint_as_float(r1[c + 3]));
-    }
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  const bool aborted = s_abort != 0;
-
-  // ---- value heads in pairs (ga, gb = ga + 1, or ga again when G is odd) -------------------
   uint32_t mma_phase = 0;
-  for (int ga = 0; ga < G && !aborted; ga += 2) {
+  bool aborted = false;
+  for (int ga = 0; ga < G; ga += 2) {
     const int gpair[2] = {ga, ga + 1 < G ? ga + 1 : ga};
     if (warp < 2) {  // gates and gamma of the pair: warp 0 head a, warp 1 head b
       const int h = j * G + gpair[warp];
@@ -409,135 +476,161 @@ __global__ void __launch_bounds__(256, 1)
       gs[warp * 64 + lane] = g0; gs[warp * 64 + lane + 32] = g1;
       bs[warp * 64 + lane] = b0; bs[warp * 64 + lane + 32] = b1;
       if (warp == 0 || gpair[1] != gpair[0]) {
-        float* gbw = gb_ws + ((size_t)blockIdx.x * hv + h) * GB_FLOATS;
+        float* gbw = gb_ws + ((size_t)chunk * hv + h) * GB_FLOATS;
         gbw[lane] = g0; gbw[lane + 32] = g1;
         gbw[64 + lane] = b0; gbw[96 + lane] = b1;
       }
     }
-    __syncthreads();
-    // A (fp32, for the solve) and the Mq rows of the P operand (bf16 hi/lo, K-major), both heads:
-    // item = (head hp, row t, 8 columns s0..s0+7)
-    for (int it = tid; it < 2 * 64 * 8; it += 256) {
-      const int t = it & 63, s0 = ((it >> 6) & 7) * 8, hp = it >> 9;
-      const float* g_ = gs + hp * 64;
-      float* Am = Amat + hp * 64 * PA_P;
-      float av[8], mv[8], kk[8], qk[8], gg[8];
-      const float gt = g_[t], bt = bs[hp * 64 + t];
+    if (ga == 0) {  // [K;Q] K^T once the tile is in (the gates above overlapped the copy)
+      if (!tc::mbar_wait(tc::smem_u32(&mbar), 0)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+      __syncthreads();
+      tc::tc_fence_after();
+      if (tid == 0 && !s_abort) {
+        constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
+        const uint64_t dd[2] = {tc::sdesc(tc::smem_u32(kq_hi), LBO128, 128), tc::sdesc(tc::smem_u32(kq_lo), LBO128, 128)};
 #pragma unroll
-      for (int q4 = 0; q4 < 2; ++q4) {
-        const float4 k4 = *reinterpret_cast<const float4*>(KK + t * PA_P + s0 + q4 * 4);
-        const float4 m4 = *reinterpret_cast<const float4*>(QK + t * PA_P + s0 + q4 * 4);
-        const float4 g4 = *reinterpret_cast<const float4*>(g_ + s0 + q4 * 4);
-        kk[q4 * 4 + 0] = k4.x; kk[q4 * 4 + 1] = k4.y; kk[q4 * 4 + 2] = k4.z; kk[q4 * 4 + 3] = k4.w;
-        qk[q4 * 4 + 0] = m4.x; qk[q4 * 4 + 1] = m4.y; qk[q4 * 4 + 2] = m4.z; qk[q4 * 4 + 3] = m4.w;
-        gg[q4 * 4 + 0] = g4.x; gg[q4 * 4 + 1] = g4.y; gg[q4 * 4 + 2] = g4.z; gg[q4 * 4 + 3] = g4.w;
-      }
+        for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int s_ = s0 + c;
-        const float dec = s_ <= t ? __expf(gt - gg[c]) : 0.0f;  // mask before exp
-        av[c] = s_ < t ? bt * dec * kk[c] : 0.0f;
-        mv[c] = dec * qk[c];
+          for (int term = 0; term < 3; ++term) {
+            const uint64_t o = (uint64_t)((ks * 2 * LBO128) >> 4);
+            tc::umma_bf16(tbase, dd[term == 2] + o, dd[term == 1] + o, idesc, (ks | term) != 0);
+          }
+        tc::umma_commit(tc::smem_u32(&mbar));
       }
-      *reinterpret_cast<float4*>(Am + t * PA_P + s0) = make_float4(av[0], av[1], av[2], av[3]);
-      *reinterpret_cast<float4*>(Am + t * PA_P + s0 + 4) = make_float4(av[4], av[5], av[6], av[7]);
-      uint4 hi, lo;
-      tc::split8(mv, hi, lo);
-      *reinterpret_cast<uint4*>(pa_hi + kmaj128(hp * 64 + t, s0)) = hi;
-      *reinterpret_cast<uint4*>(pa_lo + kmaj128(hp * 64 + t, s0)) = lo;
+      if (!s_abort && !tc::mbar_wait(tc::smem_u32(&mbar), 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+      tc::tc_fence_after();
     }
     __syncthreads();
-    // T = (I + A)^-1 by 16 x 16 blocks.  Diagonal blocks by forward substitution, both heads at
-    // once (thread = head, block, column), each row of A read as four float4 loads ...
-    if (tid < 128) {
-      const int hp = tid >> 6, blk = (tid >> 4) & 3, c = tid & 15, o = blk * 16;
-      const float* Ab = Amat + hp * 64 * PA_P + o * PA_P + o;
-      float* Tb = Tm + hp * 64 * PA_P + o * PA_P + o;
-      float x[16];
+    aborted = s_abort != 0;
+    if (aborted) break;
+    for (int hp = 0; hp < 2; ++hp) {
+      // A (fp32) and the Mq rows of the P operand, straight from the [K;Q]K^T accumulator:
+      // warp w reads TMEM lanes 32 (w % 4).. (rows 0..63 K K^T, 64..127 Q K^T), columns
+      // 32 (w / 4) .. + 31.
+      {
+        const int q4 = warp & 3, cbk = (warp >> 2) * 32;
+        const int t = (q4 * 32 + lane) & 63;
+        uint32_t r[32];
+        tc::tmem_ld32(tbase + ((uint32_t)(q4 * 32) << 16) + cbk, r);
+        tc::tmem_wait_ld();
+        const float* g_ = gs + hp * 64;
+        const float gt = g_[t];
+        if (q4 < 2) {  // A[t][s] = beta_t e^{gamma_t - gamma_s} (k_t . k_s), s < t
+          const float bt = bs[hp * 64 + t];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        float ar[16];
+          for (int c4 = 0; c4 < 8; ++c4) {
+            float4 o;
+            float* op = &o.x;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const float4 a4 = *reinterpret_cast<const float4*>(Ab + t * PA_P + q4 * 4);
-          ar[q4 * 4 + 0] = a4.x; ar[q4 * 4 + 1] = a4.y; ar[q4 * 4 + 2] = a4.z; ar[q4 * 4 + 3] = a4.w;
-        }
-        float v = (t == c) ? 1.0f : 0.0f;
+            for (int u = 0; u < 4; ++u) {
+              const int s_ = cbk + c4 * 4 + u;
+              op[u] = s_ < t ? bt * __expf(gt - g_[s_]) * __uint_as_float(r[c4 * 4 + u]) : 0.0f;
+            }
+            *reinterpret_cast<float4*>(Am + t * PA_P + cbk + c4 * 4) = o;
+          }
+        } else {  // Mq[t][s] = e^{gamma_t - gamma_s} (q_t . k_s), s <= t  (mask before exp)
 #pragma unroll
-        for (int r = 0; r < t; ++r) v = fmaf(-ar[r], x[r], v);
-        x[t] = v;
-      }
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float mv[8];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) Tb[t * PA_P + c] = x[t];
-    } else {
-      for (int idx = tid - 128; idx < 2 * 64 * 16; idx += 128) {  // zero blocks above the diagonal
-        const int hp = idx >> 10, t = (idx >> 4) & 63, s4 = (idx & 15) * 4;
-        if ((s4 >> 4) > (t >> 4))
-          *reinterpret_cast<float4*>(Tm + hp * 64 * PA_P + t * PA_P + s4) = make_float4(0, 0, 0, 0);
-      }
-    }
-    __syncthreads();
-    // ... then blocks by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj (both heads).  Item =
-    // (head, block column bj, column quad, row rr); the 16 rows of a quad sit in one half-warp,
-    // which shares the rows of W = sum_k A_ik T_kj by shuffles.
-    for (int dist = 1; dist < 4; ++dist) {
-      const int per_head = (4 - dist) * 64, nitems = 2 * per_head;
-      for (int it0 = 0; it0 < nitems; it0 += 256) {
-        const int it = it0 + tid;
-        if (it0 + (tid & ~31) >= nitems) break;  // whole warps only (nitems % 128 == 0)
-        const int hp = it / per_head, rem = it % per_head;
-        const int rr = rem & 15, cq = ((rem >> 4) & 3) * 4, bj = rem >> 6, bi = bj + dist;
-        const int ti = bi * 16 + rr, tj = bj * 16 + cq;
-        const float* Am = Amat + hp * 64 * PA_P;
-        float* T = Tm + hp * 64 * PA_P;
-        float4 wv = make_float4(0, 0, 0, 0);
-        for (int kk = bj * 16; kk < bi * 16; kk += 4) {
-          const float4 a4 = *reinterpret_cast<const float4*>(Am + ti * PA_P + kk);
-          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float4 tv = *reinterpret_cast<const float4*>(T + (kk + u) * PA_P + tj);
-            wv.x = fmaf(av[u], tv.x, wv.x); wv.y = fmaf(av[u], tv.y, wv.y);
-            wv.z = fmaf(av[u], tv.z, wv.z); wv.w = fmaf(av[u], tv.w, wv.w);
+            for (int u = 0; u < 8; ++u) {
+              const int s_ = cbk + c8 * 8 + u;
+              mv[u] = s_ <= t ? __expf(gt - g_[s_]) * __uint_as_float(r[c8 * 8 + u]) : 0.0f;
+            }
+            uint4 hi, lo;
+            tc::split8(mv, hi, lo);
+            *reinterpret_cast<uint4*>(pa_hi + kmaj128(hp * 64 + t, cbk + c8 * 8)) = hi;
+            *reinterpret_cast<uint4*>(pa_lo + kmaj128(hp * 64 + t, cbk + c8 * 8)) = lo;
           }
         }
-        float4 trow[4];  // T_ii row rr
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) trow[q4] = *reinterpret_cast<const float4*>(T + ti * PA_P + bi * 16 + q4 * 4);
-        float4 res = make_float4(0, 0, 0, 0);
-        const int base = lane & 16;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float tv = m <= rr ? comp(trow[m >> 2], m & 3) : 0.0f;
-          const float w0 = __shfl_sync(0xffffffffu, wv.x, base + m);
-          const float w1 = __shfl_sync(0xffffffffu, wv.y, base + m);
-          const float w2 = __shfl_sync(0xffffffffu, wv.z, base + m);
-          const float w3 = __shfl_sync(0xffffffffu, wv.w, base + m);
-          res.x = fmaf(-tv, w0, res.x); res.y = fmaf(-tv, w1, res.y);
-          res.z = fmaf(-tv, w2, res.z); res.w = fmaf(-tv, w3, res.w);
-        }
-        *reinterpret_cast<float4*>(T + ti * PA_P + tj) = res;
       }
       __syncthreads();
-    }
-    // [T_a | T_b] as the MN-major B operand of P (rows r, columns hp * 64 + s), and the T rows
-    // of each head's [T;P] output tile (K-major, straight to the workspace)
-    for (int it = tid; it < 2 * 64 * 8; it += 256) {
-      const int r = it & 63, s0 = ((it >> 6) & 7) * 8, hp = it >> 9;
-      const float* T = Tm + hp * 64 * PA_P + r * PA_P + s0;
-      float tv[8];
+      // T = (I + A)^-1 by 16 x 16 blocks: diagonal blocks by forward substitution (thread =
+      // block, column; rows of A read as float4) ...
+      if (tid < 64) {
+        const int blk = tid >> 4, c = tid & 15, o = blk * 16;
+        const float* Ab = Am + o * PA_P + o;
+        float* Tb = T + o * PA_P + o;
+        float x[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) tv[c] = T[c];
-      uint4 hi, lo;
-      tc::split8(tv, hi, lo);
-      const uint32_t boff = mnmaj(r, (hp * 64 + s0) >> 3, 64);
-      *reinterpret_cast<uint4*>(pb_hi + boff) = hi;
-      *reinterpret_cast<uint4*>(pb_lo + boff) = lo;
-      if (hp == 0 || gpair[1] != gpair[0]) {
-        uint8_t* out = tp_ws + ((size_t)blockIdx.x * hv + j * G + gpair[hp]) * TP_BYTES;
-        *reinterpret_cast<uint4*>(out + kmaj128(r, s0)) = hi;
-        *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(r, s0)) = lo;
+        for (int t = 0; t < 16; ++t) {
+          float ar[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(Ab + t * PA_P + q4 * 4);
+            ar[q4 * 4 + 0] = a4.x; ar[q4 * 4 + 1] = a4.y; ar[q4 * 4 + 2] = a4.z; ar[q4 * 4 + 3] = a4.w;
+          }
+          float v = (t == c) ? 1.0f : 0.0f;
+#pragma unroll
+          for (int r = 0; r < t; ++r) v = fmaf(-ar[r], x[r], v);
+          x[t] = v;
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) Tb[t * PA_P + c] = x[t];
+      } else {
+        for (int idx = tid - 64; idx < 64 * 16; idx += 192) {  // zero blocks above the diagonal
+          const int t = idx >> 4, s4 = (idx & 15) * 4;
+          if ((s4 >> 4) > (t >> 4)) *reinterpret_cast<float4*>(T + t * PA_P + s4) = make_float4(0, 0, 0, 0);
+        }
       }
+      __syncthreads();
+      // ... then by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  Item = (block column bj,
+      // column quad, row rr); the 16 rows of a quad sit in one half-warp and share the rows of
+      // W = sum_k A_ik T_kj by shuffles.
+      for (int dist = 1; dist < 4; ++dist) {
+        const int nitems = (4 - dist) * 64;
+        if ((tid & ~31) < nitems) {
+          const int rr = tid & 15, cq = ((tid >> 4) & 3) * 4, bj = tid >> 6, bi = bj + dist;
+          const int ti = bi * 16 + rr, tj = bj * 16 + cq;
+          float4 wv = make_float4(0, 0, 0, 0);
+          for (int kk = bj * 16; kk < bi * 16; kk += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(Am + ti * PA_P + kk);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 tv = *reinterpret_cast<const float4*>(T + (kk + u) * PA_P + tj);
+              wv.x = fmaf(av[u], tv.x, wv.x); wv.y = fmaf(av[u], tv.y, wv.y);
+              wv.z = fmaf(av[u], tv.z, wv.z); wv.w = fmaf(av[u], tv.w, wv.w);
+            }
+          }
+          float4 trow[4];  // T_ii row rr
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) trow[q4] = *reinterpret_cast<const float4*>(T + ti * PA_P + bi * 16 + q4 * 4);
+          float4 res = make_float4(0, 0, 0, 0);
+          const int base = lane & 16;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const float tv = m <= rr ? comp(trow[m >> 2], m & 3) : 0.0f;
+            const float w0 = __shfl_sync(0xffffffffu, wv.x, base + m);
+            const float w1 = __shfl_sync(0xffffffffu, wv.y, base + m);
+            const float w2 = __shfl_sync(0xffffffffu, wv.z, base + m);
+            const float w3 = __shfl_sync(0xffffffffu, wv.w, base + m);
+            res.x = fmaf(-tv, w0, res.x); res.y = fmaf(-tv, w1, res.y);
+            res.z = fmaf(-tv, w2, res.z); res.w = fmaf(-tv, w3, res.w);
+          }
+          *reinterpret_cast<float4*>(T + ti * PA_P + tj) = res;
+        }
+        __syncthreads();
+      }
+      // T as columns hp * 64 .. of the MN-major B operand of P, and the T rows of the head's
+      // [T;P] output tile (K-major, straight to the workspace)
+      for (int it = tid; it < 64 * 8; it += 256) {
+        const int r = it & 63, s0 = (it >> 6) * 8;
+        float tv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) tv[c] = T[r * PA_P + s0 + c];
+        uint4 hi, lo;
+        tc::split8(tv, hi, lo);
+        const uint32_t boff = mnmaj(r, (hp * 64 + s0) >> 3, 64);
+        *reinterpret_cast<uint4*>(pb_hi + boff) = hi;
+        *reinterpret_cast<uint4*>(pb_lo + boff) = lo;
+        if (hp == 0 || gpair[1] != gpair[0]) {
+          uint8_t* out = tp_ws + ((size_t)chunk * hv + j * G + gpair[hp]) * TP_BYTES;
+          *reinterpret_cast<uint4*>(out + kmaj128(r, s0)) = hi;
+          *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(r, s0)) = lo;
+        }
+      }
+      __syncthreads();  // A and T are reused by the next head
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
@@ -547,17 +640,17 @@ __global__ void __launch_bounds__(256, 1)
     if (tid == 0) {
       tc::tc_fence_after();
       constexpr uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
-      const uint32_t a0[2] = {tc::smem_u32(pa_hi), tc::smem_u32(pa_lo)};
-      const uint32_t b0[2] = {tc::smem_u32(pb_hi), tc::smem_u32(pb_lo)};
+      const uint64_t da[2] = {tc::sdesc(tc::smem_u32(pa_hi), LBO128, 128), tc::sdesc(tc::smem_u32(pa_lo), LBO128, 128)};
+      const uint64_t db[2] = {tc::sdesc(tc::smem_u32(pb_hi), 128, 1024), tc::sdesc(tc::smem_u32(pb_lo), 128, 1024)};
+#pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        for (int term = 0; term < 3; ++term) {
-          const int ai = term == 2, bi = term == 1;
-          tc::umma_bf16(tbase + 128, tc::sdesc(a0[ai] + ks * 2 * LBO128, LBO128, 128),
-                        tc::sdesc(b0[bi] + ks * 256, 128, 1024), idesc, (ks | term) != 0);
-        }
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::umma_bf16(tbase + 128, da[term == 2] + (uint64_t)((ks * 2 * LBO128) >> 4),
+                        db[term == 1] + (uint64_t)((ks * 256) >> 4), idesc, (ks | term) != 0);
       tc::umma_commit(tc::smem_u32(&mbar));
     }
-    bool ok = tc::mbar_wait(tc::smem_u32(&mbar), mma_phase);
+    const bool ok = tc::mbar_wait(tc::smem_u32(&mbar), mma_phase);
     mma_phase ^= 1;
     if (!ok) atomicExch(&g_gdn_status, -7);
     tc::tc_fence_after();
@@ -569,7 +662,7 @@ __global__ void __launch_bounds__(256, 1)
       tc::tmem_ld32(ta + 32, r1);
       tc::tmem_wait_ld();
       if (hp == 0 || gpair[1] != gpair[0]) {
-        uint8_t* out = tp_ws + ((size_t)blockIdx.x * hv + j * G + gpair[hp]) * TP_BYTES;
+        uint8_t* out = tp_ws + ((size_t)chunk * hv + j * G + gpair[hp]) * TP_BYTES;
 #pragma unroll
         for (int s0 = 0; s0 < 64; s0 += 8) {
           float pv[8];

@@ -186,12 +186,12 @@ __global__ void __launch_bounds__(256) k_epilogue(Dims d, const float* __restric
 #pragma unroll
   for (int r = 0; r < EPI_ROWS; ++r) {
     if (row0 + r >= rows) break;
-    const float inv = 1.0f / sqrtf(ss[r] * (1.0f / D) + d.rms_eps);
+    const float inv = rsqrtf(ss[r] * (1.0f / D) + d.rms_eps);
     float4 o;
-    o.x = yr[r].x * inv * nw.x * silu_f(zz[r].x);
-    o.y = yr[r].y * inv * nw.y * silu_f(zz[r].y);
-    o.z = yr[r].z * inv * nw.z * silu_f(zz[r].z);
-    o.w = yr[r].w * inv * nw.w * silu_f(zz[r].w);
+    o.x = yr[r].x * inv * nw.x * silu_fast(zz[r].x);
+    o.y = yr[r].y * inv * nw.y * silu_fast(zz[r].y);
+    o.z = yr[r].z * inv * nw.z * silu_fast(zz[r].z);
+    o.w = yr[r].w * inv * nw.w * silu_fast(zz[r].w);
     store4<OUT_BF16>(y, (size_t)(row0 + r) * D + c0, o);
   }
 }

@@ -177,15 +177,20 @@ __device__ __forceinline__ void split2(float x, uint16_t& hi, uint16_t& lo) {
   hi = __bfloat16_as_ushort(h);
   lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
 }
-// Split 8 consecutive fp32 values into two 16-byte chunks (hi, lo).
+// Split 8 consecutive fp32 values into two 16-byte chunks (hi, lo), two values per packed
+// round-to-nearest conversion.
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
-  uint16_t h[8], l[8];
+  uint32_t h[4], l[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) split2(x[i], h[i], l[i]);
-  hi = make_uint4(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16), h[4] | (uint32_t(h[5]) << 16),
-                  h[6] | (uint32_t(h[7]) << 16));
-  lo = make_uint4(l[0] | (uint32_t(l[1]) << 16), l[2] | (uint32_t(l[3]) << 16), l[4] | (uint32_t(l[5]) << 16),
-                  l[6] | (uint32_t(l[7]) << 16));
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+    h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[i] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 }  // namespace tc

@@ -92,6 +92,8 @@ size_t gdn_prefill_workspace_size(const gdn_dims_t* d);
  * Each sequence starts with a zero conv history and with its init_state.  Empty
  * sequences copy init_state (or zeros) to final_state.  T_tot == 0 writes final_state
  * only.  cu_seqlens' contents are not validated on the host (they stay on the device).
+ * bf16 inputs run on the tensor-core path, which needs T_tot / 64 + N + 1 <= 65535
+ * (about 4.19M packed tokens per call); larger calls return GDN_ERR_SHAPE.
  */
 int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
                 const float* a, const float* b, const float* A_log, const float* dt_bias,

@@ -17,6 +17,8 @@ def to_dev(x, device="cuda"):
 
 
 def run_prefill(inp, out_dtype=torch.float32, init_alias=False, **kw):
+    """Run gdn_prefill on generated inputs (numpy) through the binding; returns fp64 numpy
+    (y, final_state).  Extra keyword arguments go to gdn_prefill (e.g. workspace, q_scale)."""
     from gated_deltanet_token_b200 import gdn
 
     d = {n: to_dev(inp.get(n)) for n in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w",

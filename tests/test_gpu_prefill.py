@@ -117,3 +117,48 @@ def test_long_prefill_T262144_sampled_heads(oracle_mod):
     y, S = run_prefill(inp, torch.float32)
     sl = slice(*heads)
     check_bf16(y[:, sl], ref["y"][:, sl], S[:, sl], ref["final_state"][:, sl])
+
+
+# ---- the bf16 (tensor-core) path: head ratios, ragged lengths, SIMT cross-check ----------
+
+@pytest.mark.parametrize("ratio", [1, 2, 4])
+def test_head_ratios_bf16_tensor_core_path(oracle_mod, ratio):
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[77, 3, 130], h_qk=2, h_v=2 * ratio)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_bf16(y, ref["y"], S, ref["final_state"])
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 31, 32, 33, 63, 64, 65, 129])
+def test_short_lengths_bf16_tensor_core_path(oracle_mod, T):
+    inp = make_inputs("prefill_T4096_bf16", T=T, h_qk=4, h_v=8)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_bf16(y, ref["y"], S, ref["final_state"])
+
+
+def test_tensor_core_path_is_insensitive_to_stale_workspace(oracle_mod):
+    """The workspace is reused between calls: fill it with NaN bit patterns first and check
+    that nothing left in it reaches the results (rows past a chunk's length are rewritten)."""
+    from gated_deltanet_token_b200 import gdn
+
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[5, 70, 33], h_qk=2, h_v=4)
+    ref = _oracle(oracle_mod, inp)
+    T = inp["q"].shape[0]
+    dims = gdn.make_dims(3, T, 2, 4, gdn.GDN_DTYPE_BF16, gdn.GDN_DTYPE_F32)
+    ws = torch.full((gdn.gdn_prefill_workspace_size(dims),), 0xFF, dtype=torch.uint8, device="cuda")
+    y, S = run_prefill(inp, torch.float32, workspace=ws)
+    assert np.isfinite(y).all() and np.isfinite(S).all()
+    check_bf16(y, ref["y"], S, ref["final_state"])
+
+
+def test_tensor_core_and_fp32_paths_agree(monkeypatch):
+    """Both arithmetic paths of the bf16-input prefill (tensor cores with bf16 hi/lo products,
+    and fp32 FFMA) against each other, on the model head shapes."""
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[200, 64, 1])
+    y_tc, S_tc = run_prefill(inp, torch.float32)
+    monkeypatch.setenv("GDN_FORCE_SIMT", "1")
+    y_s, S_s = run_prefill(inp, torch.float32)
+    r = float(np.sqrt(np.mean(y_s ** 2)))
+    assert np.abs(y_tc - y_s).max() <= 2e-2 * r
+    assert np.linalg.norm(S_tc - S_s) / np.linalg.norm(S_s) <= 1e-2
