@@ -723,7 +723,7 @@ __global__ void __launch_bounds__(288, 1)
   uint8_t* s_lo = sm + PB_S_TILE;
   uint8_t* stage[2] = {sm + 2 * PB_S_TILE, sm + 2 * PB_S_TILE + PBStage::BYTES};
   __shared__ uint64_t mbar_ld[2];
-  __shared__ uint64_t mbar_mma;
+  __shared__ uint64_t mbar_mma[3];  // one per MMA round: each completes once per chunk
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
 
@@ -737,13 +737,17 @@ __global__ void __launch_bounds__(288, 1)
     s_abort = 0;
     tc::mbar_init(tc::smem_u32(&mbar_ld[0]), 1);
     tc::mbar_init(tc::smem_u32(&mbar_ld[1]), 1);
-    tc::mbar_init(tc::smem_u32(&mbar_mma), 1);
+    for (int q3 = 0; q3 < 3; ++q3) tc::mbar_init(tc::smem_u32(&mbar_mma[q3]), 1);
     tc::fence_mbar_init();
   }
   if (warp == 0) {
     tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // D_a 0..63, D_cd 64..127, D_e 128..191
     tc::tmem_relinquish();
   }
+  // barrier over the four warps that own TMEM lanes 0..63 (warps 0, 1, 4, 5)
+  auto named_bar_sync = [](int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+  };
   auto issue_load = [&](int c, int st) {
     const size_t gc = (size_t)gc0 + c;
     const uint32_t bar = tc::smem_u32(&mbar_ld[st]);
@@ -783,7 +787,7 @@ __global__ void __launch_bounds__(288, 1)
   constexpr uint32_t idesc_mn = tc::idesc_bf16(128, NV, 1, 1);
   const uint64_t d_s[2] = {tc::sdesc(tc::smem_u32(s_hi), 128, 16 * 128), tc::sdesc(tc::smem_u32(s_lo), 128, 16 * 128)};
 
-  uint32_t ph_ld[2] = {0, 0}, ph_mma = 0;
+  uint32_t ph_ld[2] = {0, 0}, ph_mma = 0;  // ph_mma: parity of this chunk's phase of each round barrier
   bool aborted = false;
   for (int c = 0; c < nchunks && !aborted; ++c) {
     const int st = c & 1;
@@ -819,11 +823,10 @@ __global__ void __launch_bounds__(288, 1)
         tc::umma_bf16(T_A, da[0] + ao, d_s[0] + bo, idesc_kn2, ks != 0);  // a_hi [s_hi | s_lo]
         tc::umma_bf16(T_A, da[1] + ao, d_s[0] + bo, idesc_kn, 1);         // a_lo s_hi
       }
-      tc::umma_commit(tc::smem_u32(&mbar_mma));
+      tc::umma_commit(tc::smem_u32(&mbar_mma[0]));
     }
     if (producer && lane == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);  // stage last read by chunk c-1
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
-    ph_mma ^= 1;
+    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     tc::tc_fence_after();
     float qs[NH];  // rows 64..127: e^{gamma_t} (Q S^T)[t][:]
     if (!producer) {
@@ -853,8 +856,7 @@ __global__ void __launch_bounds__(288, 1)
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
-    __syncthreads();
-    if (s_abort) { aborted = true; break; }
+    if (quarter < 2 && !producer) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 2: [U ; (M o QK^T) U] = [T;P] (128 x 64) x R (K = 64, N = nv) ----------------
     if (tid == 0) {
       tc::tc_fence_after();
@@ -866,10 +868,9 @@ __global__ void __launch_bounds__(288, 1)
         tc::umma_bf16(T_CD, da[0] + ao, db + bo, idesc_kn2, ks != 0);
         tc::umma_bf16(T_CD, da[1] + ao, db + bo, idesc_kn, 1);
       }
-      tc::umma_commit(tc::smem_u32(&mbar_mma));
+      tc::umma_commit(tc::smem_u32(&mbar_mma[1]));
     }
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
-    ph_mma ^= 1;
+    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     tc::tc_fence_after();
     if (!producer) {
       uint32_t r[16], r2[16];
@@ -903,8 +904,7 @@ __global__ void __launch_bounds__(288, 1)
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
-    __syncthreads();
-    if (s_abort) { aborted = true; break; }
+    if (quarter < 2 && !producer) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 3: K^T U-tilde: A = MN-major view of the K rows (M = 128 key comps, K = 64 tokens)
     if (tid == 0) {
       tc::tc_fence_after();
@@ -916,9 +916,9 @@ __global__ void __launch_bounds__(288, 1)
         tc::umma_bf16(T_E, da[0] + o, db + o, idesc_mn2, ks != 0);
         tc::umma_bf16(T_E, da[1] + o, db + o, idesc_mn, 1);
       }
-      tc::umma_commit(tc::smem_u32(&mbar_mma));
+      tc::umma_commit(tc::smem_u32(&mbar_mma[2]));
     }
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[2]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_mma ^= 1;
     tc::tc_fence_after();
     if (!producer) {
