@@ -28,17 +28,22 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // The bf16-input prefill runs its chunk contractions on tcgen05 (bf16 hi/lo products); the
 // fp32-input prefill keeps true fp32 FFMA.  GDN_FORCE_SIMT=1 in the environment sends bf16
-// inputs down the fp32 path too (for comparisons).
+// inputs down the fp32 path too, and GDN_NO_FUSED_NORM=1 keeps the output norm of the bf16
+// path in its own kernel (both for comparisons).
+int getenv_flag(const char* name) {
+  const char* f = getenv(name);
+  return f && f[0] == '1' ? 1 : 0;
+}
+
 bool use_tc(const gdn_dims_t* d) {
   if (d->in_dtype != GDN_DTYPE_BF16) return false;
-  const char* f = getenv("GDN_FORCE_SIMT");
-  return !(f && f[0] == '1');
+  return getenv_flag("GDN_FORCE_SIMT") == 0;
 }
 
 // Workspace of the prefill, carved from the caller's buffer in this order.
 struct WsLayout {
   size_t tab, seqc0, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
-  size_t kq, tp, gb, bv;  // tensor-core path
+  size_t kq, tp, gb, vs;  // tensor-core path
   int max_chunks;
   bool tc;
 };
@@ -61,7 +66,7 @@ WsLayout ws_layout_tc(const gdn_dims_t* d) {
   L.kq = take(MC * hq * KQ_BYTES);
   L.tp = take(MC * hv * TP_BYTES);
   L.gb = take(MC * hv * GB_FLOATS * 4);
-  L.bv = take(MC * hv * BV_BYTES);
+  L.vs = take(MC * hv * VS_BYTES);
   L.yraw = take(T * hv * D * 4);
   L.total = off;
   return L;
@@ -180,11 +185,45 @@ int configure_device() {
           cudaSuccess ||
       cudaFuncSetAttribute(k_chunkprep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_TC_SMEM) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(k_chunkscan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PB_TC_SMEM) !=
-          cudaSuccess)
+      cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_RAW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)PB_TC_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)PB_TC_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)PB_TC_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   done_mask.fetch_or(bit);
   return GDN_OK;
+}
+
+// Clusters of four phase-B CTAs (the slices of one value head) that fit on the device at
+// once, per device; 0 if the query failed (then the fused output norm is not used).
+int scan_clusters_per_wave() {
+  static int cached[64];
+  static std::atomic<uint64_t> known{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (known.load() & bit) return cached[dev & 63];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, D / TC_NV);
+  cfg.blockDim = dim3(288);
+  cfg.dynamicSmemBytes = PB_TC_SMEM;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 1;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = D / TC_NV;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_chunkscan_tc<PB_Y_BF16>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cached[dev & 63] = n;
+  known.fetch_or(bit);
+  return n;
 }
 
 template <bool IN_BF16>
@@ -273,16 +312,50 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
         const int grid = nitems < g_num_sms ? nitems : g_num_sms;
         k_prologue_tc<<<grid, 512, PRO_SMEM, s>>>(kd, tab, nitems, static_cast<const uint16_t*>(q),
                                                   static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
-                                                  b, conv_w, kq, F(L.bv));
+                                                  conv_w, kq, F(L.vs));
       }
       ProfScope p("chunk_prep_tc", s);
       k_chunkprep_tc<<<dim3(d->h_qk, L.max_chunks), 256, PA_TC_SMEM, s>>>(kd, tab, a, b, A_log, dt_bias, kq, tp,
                                                                           F(L.gb));
     }
+    // The output norm runs inside phase B (clusters of the four slices of a head) unless that
+    // would take more waves of CTAs than the unclustered launch.
+    const long units = (long)d->n_seqs * d->h_v;
+    const int per_wave = scan_clusters_per_wave();
+    const long waves_fused = per_wave > 0 ? (units + per_wave - 1) / per_wave : 0;
+    const long waves_plain = (units * (D / TC_NV) + g_num_sms - 1) / g_num_sms;
+    const bool fused = per_wave > 0 && waves_fused <= waves_plain && getenv_flag("GDN_NO_FUSED_NORM") == 0;
+    const dim3 grid(d->n_seqs, d->h_v, D / TC_NV);
+    if (fused) {
+      ProfScope p("chunk_scan_tc_norm", s);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(288);
+      cfg.dynamicSmemBytes = PB_TC_SMEM;
+      cfg.stream = s;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 1;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = D / TC_NV;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      const uint16_t* zb = static_cast<const uint16_t*>(z);
+      cudaError_t e = kd.out_bf16
+          ? cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_BF16>, kd, (const int*)cu_seqlens, (const int*)seqc0,
+                               (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
+                               init_state, F(L.yraw), final_state, zb, norm_w, y)
+          : cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_F32>, kd, (const int*)cu_seqlens, (const int*)seqc0,
+                               (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
+                               init_state, F(L.yraw), final_state, zb, norm_w, y);
+      if (e != cudaSuccess) return GDN_ERR_CUDA;
+      return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
     {
       ProfScope p("chunk_scan_tc", s);
-      k_chunkscan_tc<<<dim3(d->n_seqs, d->h_v, D / TC_NV), 288, PB_TC_SMEM, s>>>(
-          kd, cu_seqlens, seqc0, kq, tp, F(L.gb), F(L.bv), init_state, F(L.yraw), final_state);
+      k_chunkscan_tc<PB_Y_RAW><<<grid, 288, PB_TC_SMEM, s>>>(kd, cu_seqlens, seqc0, kq, tp, F(L.gb), F(L.vs),
+                                                             init_state, F(L.yraw), final_state, nullptr, nullptr,
+                                                             nullptr);
     }
     if (d->total_tokens > 0) {
       ProfScope p("epilogue", s);

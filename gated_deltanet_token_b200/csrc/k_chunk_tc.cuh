@@ -16,9 +16,11 @@
 // element, which the scale-invariant output norm amplifies on tokens with a small y_raw;
 // the split keeps the products at ~2^-17 relative error.
 //
-// Phase A (k_chunkprep_tc, parallel over chunks x QK heads): conv + SiLU + L2 norm of q, k;
-// the [K;Q] hi/lo tile (stored to the workspace with one bulk copy); [K;Q] K^T on tcgen05;
-// per value head: gates, gamma, A, M o QK^T, T = (I + A)^-1 (blocked 16 x 16 forward
+// Prologue (k_prologue_tc, persistent over (head group, half chunk) items): conv + SiLU of
+// q, k, v, L2 norm of q and k; writes the [K;Q] hi/lo operand tile of each (chunk, QK head)
+// and v as fp32 slices.
+// Phase A (k_chunkprep_tc, parallel over chunks x QK heads): [K;Q] K^T on tcgen05; per
+// value head: gates, gamma, A, M o QK^T, T = (I + A)^-1 (blocked 16 x 16 forward
 // substitution), P = (M o QK^T) T, and the [T;P] hi/lo tile.
 // Phase B (k_chunkscan_tc, sequential over one sequence's chunks, parallel over value
 // heads and 32-row slices of the state): the three MMA rounds above per chunk, with the
@@ -35,8 +37,8 @@ constexpr uint32_t KQ_BYTES = 2 * KQ_TILE;           // per (chunk, QK head)
 constexpr uint32_t TP_TILE = 128 * 64 * 2;           // one bf16 tile of [T;P]: 16 KB
 constexpr uint32_t TP_BYTES = 2 * TP_TILE;           // per (chunk, value head)
 constexpr uint32_t GB_FLOATS = 128;                  // gamma[64], beta[64] per (chunk, value head)
-constexpr uint32_t BV_SLICE = 64 * TC_NV * 4;        // beta * v (fp32) of one 32-column slice: 8 KB
-constexpr uint32_t BV_BYTES = 4 * BV_SLICE;          // per (chunk, value head)
+constexpr uint32_t VS_SLICE = 64 * TC_NV * 4;        // v after conv + SiLU (fp32), one 32-column slice: 8 KB
+constexpr uint32_t VS_BYTES = 4 * VS_SLICE;          // per (chunk, value head)
 constexpr uint32_t LBO128 = 2048;                    // K-direction core stride of 128-row tiles
 
 // Byte offset of element (r, k) in a K-major no-swizzle tile with 128 rows.
@@ -165,20 +167,22 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 }
 
 // ======================================================================================
-// Prologue of the tensor-core path (K1).  Persistent: each CTA walks work items (head group,
+// Prologue of the tensor-core path.  Persistent: each CTA walks work items (head group,
 // half chunk) with a stride of the grid size.  A group is up to 8 heads of one stream -- q,
 // k or value heads -- whose slices of a token row are contiguous (2 KB).  The next item's
 // 32 + 3 token rows and conv taps are bulk-copied into the other of two shared-memory stages
-// while the current item is computed, so loads overlap compute.  16 warps: warp w works on
-// head w % 8 of the group and on token blocks 16 (w / 8) .. + 15 of the half chunk.
+// while the current item is computed, so loads overlap compute; the 32 lanes of warp 0 issue
+// those copies together and leave the item's description in shared memory for the others.
+// 16 warps: warp w works on head w % 8 of the group and on tokens 16 (w / 8) .. + 15 of the
+// half chunk.
 //   q / k head j: rows 64..127 / 0..63 of the [K;Q] hi/lo tile of QK head j
-//   value head h: beta * v as four contiguous 32-column fp32 slices [4][64][32]
+//   value head h: v after conv and SiLU as four contiguous 32-column fp32 slices [4][64][32]
 // Width-4 causal conv and SiLU ("Qwen3.8-Flash-Next" technical report, Fig. 2; field
-// guide §02), L2 norm of q and k (Fig. 2), beta = sigmoid(b).  q/k lanes: token r = lane % 4,
-// 8-channel groups lane / 4 and lane / 4 + 8; the eight lanes of a token reduce the L2 norm
-// with three shuffles and consecutive lanes store consecutive 16-byte chunks.  Every row of
-// a used chunk slot is written (rows past the chunk's length as zeros): phase B multiplies
-// those K rows by zero weights, so stale workspace bits must not survive.
+// guide §02), L2 norm of q and k (Fig. 2).  q/k lanes: token r = lane % 4, 8-channel groups
+// lane / 4 and lane / 4 + 8; the eight lanes of a token reduce the L2 norm with three
+// shuffles and consecutive lanes store consecutive 16-byte chunks.  Every row of a used
+// chunk slot is written (rows past the chunk's length as zeros): phase B multiplies those K
+// rows by zero weights, so stale workspace bits must not survive.
 // ======================================================================================
 constexpr int PRO_HG = 8;                  // heads per work item
 constexpr int PRO_TOK = 32;                // tokens per work item (half a chunk)
@@ -187,11 +191,12 @@ constexpr uint32_t PRO_ROWS_BYTES = PRO_ROWS * PRO_HG * D * 2;
 constexpr uint32_t PRO_W_BYTES = PRO_HG * D * 16;
 constexpr uint32_t PRO_STAGE = PRO_ROWS_BYTES + PRO_W_BYTES;
 constexpr size_t PRO_SMEM = 2 * (size_t)PRO_STAGE;
+static_assert(PRO_ROWS <= 64, "two token rows per lane of the issuing warp");
 
 struct ProItem {
   ChunkEntry e;
   int chunk, tb0, stream, h0, nh, nheads;
-  size_t ch0;  // first conv channel of the group
+  int ch0;  // first conv channel of the group
 };
 
 __device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry* tab, int it, int ngroups) {
@@ -205,8 +210,7 @@ __device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry* tab
   w.nheads = w.stream == 2 ? d.h_v : hq;
   w.h0 = (w.stream == 2 ? grp - 2 * nqg : grp - w.stream * nqg) * PRO_HG;
   w.nh = min(PRO_HG, w.nheads - w.h0);
-  w.ch0 = w.stream == 0 ? (size_t)w.h0 * D : w.stream == 1 ? (size_t)(hq + w.h0) * D
-                                                           : (size_t)2 * hq * D + (size_t)w.h0 * D;
+  w.ch0 = w.stream == 0 ? w.h0 * D : w.stream == 1 ? (hq + w.h0) * D : 2 * hq * D + w.h0 * D;
   return w;
 }
 
@@ -214,15 +218,15 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
                                                         const uint16_t* __restrict__ q,
                                                         const uint16_t* __restrict__ k,
                                                         const uint16_t* __restrict__ v,
-                                                        const float* __restrict__ b,
                                                         const float* __restrict__ conv_w,
-                                                        uint8_t* __restrict__ kq_ws, float* __restrict__ bv_ws) {
+                                                        uint8_t* __restrict__ kq_ws, float* __restrict__ vs_ws) {
   const int hq = d.h_qk, hv = d.h_v;
   const int ngroups = 2 * ((hq + PRO_HG - 1) / PRO_HG) + (hv + PRO_HG - 1) / PRO_HG;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hw = warp & (PRO_HG - 1), tsplit = warp >> 3;
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t mbar[2];
+  __shared__ ProItem s_item[2];
   __shared__ int s_abort;
   if (tid == 0) {
     s_abort = 0;
@@ -231,44 +235,56 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     tc::fence_mbar_init();
   }
   __syncthreads();
-  // issue the copies of item `it` into stage `st` (thread 0); unused chunk slots copy nothing
+  // (warp 0, all lanes) describe item `it` in s_item[st] and issue its copies into stage
+  // `st`: lane l copies token rows l and l + 32.  Unused chunk slots copy nothing.
   auto issue = [&](int it, int st) -> bool {  // true if copies were issued
     const ProItem w = pro_item(d, tab, it, ngroups);
+    if (lane == 0) s_item[st] = w;
     if (w.e.len == 0) return false;
     const uint16_t* src = w.stream == 0 ? q : w.stream == 1 ? k : v;
     const uint32_t row_bytes = (uint32_t)w.nh * D * 2;
-    uint32_t bytes = (uint32_t)w.nh * D * 16;
-    for (int r = 0; r < PRO_ROWS; ++r) {
-      const int tcr = w.tb0 - 3 + r;
-      if (tcr < w.e.len && (long)w.e.t0 + tcr >= w.e.seq_start) bytes += row_bytes;
+    bool ok[2];
+    uint32_t mine = 0;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = lane + 32 * u, tcr = w.tb0 - 3 + r;
+      ok[u] = r < PRO_ROWS && tcr < w.e.len && (long)w.e.t0 + tcr >= w.e.seq_start;
+      mine += ok[u] ? row_bytes : 0u;
     }
+    const uint32_t bytes = __reduce_add_sync(0xffffffffu, mine) + (uint32_t)w.nh * D * 16;
     const uint32_t bar = tc::smem_u32(&mbar[st]);
-    uint8_t* base = sm + (size_t)st * PRO_STAGE;
-    tc::mbar_arrive_expect_tx(bar, bytes);
-    tc::bulk_g2s(tc::smem_u32(base + PRO_ROWS_BYTES), conv_w + w.ch0 * 4, (uint32_t)w.nh * D * 16, bar);
-    for (int r = 0; r < PRO_ROWS; ++r) {
-      const int tcr = w.tb0 - 3 + r;
-      const long tg = (long)w.e.t0 + tcr;
-      if (tcr < w.e.len && tg >= w.e.seq_start)
-        tc::bulk_g2s(tc::smem_u32(base) + r * row_bytes, src + ((size_t)tg * w.nheads + w.h0) * D, row_bytes, bar);
+    const uint32_t base = tc::smem_u32(sm + (size_t)st * PRO_STAGE);
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(bar, bytes);
+      tc::bulk_g2s(base + PRO_ROWS_BYTES, conv_w + (size_t)w.ch0 * 4, (uint32_t)w.nh * D * 16, bar);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = lane + 32 * u;
+      if (ok[u]) {
+        const long tg = (long)w.e.t0 + w.tb0 - 3 + r;
+        tc::bulk_g2s(base + r * row_bytes, src + ((size_t)tg * w.nheads + w.h0) * D, row_bytes, bar);
+      }
     }
     return true;
   };
-  bool pending[2] = {false, false};  // (thread 0) copies in flight per stage
-  if (tid == 0 && (int)blockIdx.x < nitems) pending[0] = issue(blockIdx.x, 0);
+  bool pending[2] = {false, false};  // (warp 0) copies in flight per stage
+  if (warp == 0 && (int)blockIdx.x < nitems) pending[0] = issue(blockIdx.x, 0);
+  __syncthreads();
   uint32_t parity[2] = {0, 0};
   int n = 0;
   for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
     const int st = n & 1;
-    const ProItem w = pro_item(d, tab, it, ngroups);
-    if (tid == 0 && it + (int)gridDim.x < nitems) pending[st ^ 1] = issue(it + gridDim.x, st ^ 1);
+    const ProItem w = s_item[st];
+    if (warp == 0 && it + (int)gridDim.x < nitems) pending[st ^ 1] = issue(it + gridDim.x, st ^ 1);
     if (w.e.len == 0) {
       __syncthreads();
       continue;
     }
     if (!tc::mbar_wait(tc::smem_u32(&mbar[st]), parity[st])) s_abort = 1;
     parity[st] ^= 1;
-    if (tid == 0) pending[st] = false;
+    if (warp == 0) pending[st] = false;
     __syncthreads();  // the abort decision is uniform
     if (s_abort) break;
     const uint8_t* base = sm + (size_t)st * PRO_STAGE;
@@ -344,16 +360,10 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
           const float4 t4 = wsm[c0 + c];
           wv[c][0] = t4.x; wv[c][1] = t4.y; wv[c][2] = t4.z; wv[c][3] = t4.w;
         }
-        float* out = bv_ws + ((size_t)w.chunk * hv + head) * (BV_BYTES / 4) + (size_t)(c0 / TC_NV) * (BV_SLICE / 4) +
+        float* out = vs_ws + ((size_t)w.chunk * hv + head) * (VS_BYTES / 4) + (size_t)(c0 / TC_NV) * (VS_SLICE / 4) +
                      (c0 % TC_NV);
 #pragma unroll 1
         for (int blk = tsplit * (PRO_TOK / 2); blk < (tsplit + 1) * (PRO_TOK / 2); blk += 8) {
-          float bt[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int t = tb0 + blk + i;
-            bt[i] = t < L ? __ldg(b + (size_t)(w.e.t0 + t) * hv + head) : 0.0f;
-          }
           uint2 x[11];  // raw bf16 of 4 channels, rows t - 3 .. t + 7
 #pragma unroll
           for (int p = 0; p < 11; ++p) {
@@ -367,13 +377,12 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int t = tb0 + blk + i;
-            const float beta = t < L ? sigmoid_fast(bt[i]) : 0.0f;
             float r4[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               const float acc = fmaf(wv[c][3], xv(i + 3, c),
                                      fmaf(wv[c][2], xv(i + 2, c), fmaf(wv[c][1], xv(i + 1, c), wv[c][0] * xv(i, c))));
-              r4[c] = beta * silu_fast(acc);
+              r4[c] = t < L ? silu_fast(acc) : 0.0f;
             }
             *reinterpret_cast<float4*>(out + t * TC_NV) = make_float4(r4[0], r4[1], r4[2], r4[3]);
           }
@@ -383,12 +392,10 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     tc::fence_proxy_async();
     __syncthreads();  // this stage is free for the item after next
   }
-  if (s_abort) {  // record, and let copies still in flight land (bounded) before leaving
-    if (tid == 0) {
-      atomicExch(&g_gdn_status, -7);
-      for (int q2 = 0; q2 < 2; ++q2)
-        if (pending[q2]) (void)tc::mbar_wait(tc::smem_u32(&mbar[q2]), parity[q2]);
-    }
+  if (s_abort && warp == 0) {  // record, and let copies still in flight land (bounded) before leaving
+    if (lane == 0) atomicExch(&g_gdn_status, -7);
+    for (int q2 = 0; q2 < 2; ++q2)
+      if (pending[q2]) (void)tc::mbar_wait(tc::smem_u32(&mbar[q2]), parity[q2]);
   }
 }
 
@@ -397,15 +404,23 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
 // ======================================================================================
 constexpr int PA_P = 68;  // pitch (floats) of the fp32 64 x 64 matrices of phase A
 constexpr uint32_t PA_MAT = 64 * PA_P * 4;
-// [0, 64K): [K;Q] tile (hi | lo); after [K;Q]K^T it holds the P operands: [Mq_a; Mq_b]
-// (K-major, 128 x 64) hi | lo and [T_a | T_b] (MN-major, K = 64, N = 128) hi | lo.  Then A and T
-// (fp32, one value head at a time) and the gates of the pair.
-constexpr uint32_t PA_OFF_A = 65536;
-constexpr uint32_t PA_OFF_T = PA_OFF_A + PA_MAT;
-constexpr uint32_t PA_OFF_G = PA_OFF_T + PA_MAT;
+// [0, 64K): the [K;Q] tile (hi | lo).  Once [K;Q]K^T is in TMEM the tile is dead and the
+// region holds the P operands, [Mq_a; Mq_b] (K-major, 128 x 64) hi | lo at [0, 32K) and
+// [T_a | T_b] (MN-major, K = 64, N = 128) hi | lo at [32K, 64K); the fp32 A matrices of both
+// heads of the pair alias [32K, 32K + 2 PA_MAT) until T is known.  Then the fp32 T matrices
+// of the pair and the gates.
+constexpr uint32_t PA_OFF_PA = 0;
+constexpr uint32_t PA_OFF_PB = 32768;
+constexpr uint32_t PA_OFF_A = 32768;
+constexpr uint32_t PA_OFF_T = PA_OFF_A + 2 * PA_MAT;
+constexpr uint32_t PA_OFF_G = PA_OFF_T + 2 * PA_MAT;
 constexpr size_t PA_TC_SMEM = PA_OFF_G + 4 * 64 * 4;
+static_assert(PA_OFF_T >= KQ_BYTES, "T and the gates lie past the [K;Q] tile");
 static_assert(PA_TC_SMEM <= 113 * 1024, "two phase-A CTAs per SM");
 
+// One CTA per (QK head j, chunk); value heads of QK head j in pairs (a, b), both heads of a
+// pair at once: A, M o QK^T, T = (I + A)^-1 and P = (M o QK^T) T.  Field guide §02 defines
+// the per-token steps these chunk quantities regroup.
 __global__ void __launch_bounds__(256, 2)
     k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
@@ -419,12 +434,12 @@ __global__ void __launch_bounds__(256, 2)
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* kq_hi = sm;
   uint8_t* kq_lo = sm + KQ_TILE;
-  uint8_t* pa_hi = sm;          // [Mq_a; Mq_b] operand (aliases the [K;Q] tile)
-  uint8_t* pa_lo = sm + 16384;
-  uint8_t* pb_hi = sm + 32768;  // [T_a | T_b] operand
-  uint8_t* pb_lo = sm + 49152;
-  float* Am = reinterpret_cast<float*>(sm + PA_OFF_A);
-  float* T = reinterpret_cast<float*>(sm + PA_OFF_T);
+  uint8_t* pa_hi = sm + PA_OFF_PA;  // [Mq_a; Mq_b] operand (aliases the [K;Q] tile)
+  uint8_t* pa_lo = pa_hi + 16384;
+  uint8_t* pb_hi = sm + PA_OFF_PB;  // [T_a | T_b] operand
+  uint8_t* pb_lo = pb_hi + 16384;
+  float* Am = reinterpret_cast<float*>(sm + PA_OFF_A);  // [2][64][PA_P]
+  float* Tm = reinterpret_cast<float*>(sm + PA_OFF_T);  // [2][64][PA_P]
   float* gs = reinterpret_cast<float*>(sm + PA_OFF_G);  // [2][64] gamma
   float* bs = gs + 128;                                 // [2][64] beta
   __shared__ uint64_t mbar;
@@ -503,20 +518,22 @@ __global__ void __launch_bounds__(256, 2)
     __syncthreads();
     aborted = s_abort != 0;
     if (aborted) break;
-    for (int hp = 0; hp < 2; ++hp) {
-      // A (fp32) and the Mq rows of the P operand, straight from the [K;Q]K^T accumulator:
-      // warp w reads TMEM lanes 32 (w % 4).. (rows 0..63 K K^T, 64..127 Q K^T), columns
-      // 32 (w / 4) .. + 31.
-      {
-        const int q4 = warp & 3, cbk = (warp >> 2) * 32;
-        const int t = (q4 * 32 + lane) & 63;
-        uint32_t r[32];
-        tc::tmem_ld32(tbase + ((uint32_t)(q4 * 32) << 16) + cbk, r);
-        tc::tmem_wait_ld();
+    // A (fp32) of both heads and the Mq rows of the P operand, straight from the [K;Q]K^T
+    // accumulator: warp w reads TMEM lanes 32 (w % 4).. (rows 0..63 K K^T, 64..127 Q K^T),
+    // columns 32 (w / 4) .. + 31.
+    {
+      const int q4 = warp & 3, cbk = (warp >> 2) * 32;
+      const int t = (q4 * 32 + lane) & 63;
+      uint32_t r[32];
+      tc::tmem_ld32(tbase + ((uint32_t)(q4 * 32) << 16) + cbk, r);
+      tc::tmem_wait_ld();
+#pragma unroll 1
+      for (int hp = 0; hp < 2; ++hp) {
         const float* g_ = gs + hp * 64;
         const float gt = g_[t];
         if (q4 < 2) {  // A[t][s] = beta_t e^{gamma_t - gamma_s} (k_t . k_s), s < t
           const float bt = bs[hp * 64 + t];
+          float* Ah = Am + hp * (64 * PA_P);
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
             float4 o;
@@ -526,7 +543,7 @@ __global__ void __launch_bounds__(256, 2)
               const int s_ = cbk + c4 * 4 + u;
               op[u] = s_ < t ? bt * __expf(gt - g_[s_]) * __uint_as_float(r[c4 * 4 + u]) : 0.0f;
             }
-            *reinterpret_cast<float4*>(Am + t * PA_P + cbk + c4 * 4) = o;
+            *reinterpret_cast<float4*>(Ah + t * PA_P + cbk + c4 * 4) = o;
           }
         } else {  // Mq[t][s] = e^{gamma_t - gamma_s} (q_t . k_s), s <= t  (mask before exp)
 #pragma unroll
@@ -544,93 +561,98 @@ __global__ void __launch_bounds__(256, 2)
           }
         }
       }
-      __syncthreads();
-      // T = (I + A)^-1 by 16 x 16 blocks: diagonal blocks by forward substitution (thread =
-      // block, column; rows of A read as float4) ...
-      if (tid < 64) {
-        const int blk = tid >> 4, c = tid & 15, o = blk * 16;
-        const float* Ab = Am + o * PA_P + o;
-        float* Tb = T + o * PA_P + o;
-        float x[16];
+    }
+    __syncthreads();
+    // T = (I + A)^-1 by 16 x 16 blocks: diagonal blocks by forward substitution (thread =
+    // head, block, column; rows of A read as float4) ...
+    if (tid < 128) {
+      const int hp = tid >> 6, blk = (tid >> 4) & 3, c = tid & 15, o = blk * 16;
+      const float* Ab = Am + hp * (64 * PA_P) + o * PA_P + o;
+      float* Tb = Tm + hp * (64 * PA_P) + o * PA_P + o;
+      float x[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          float ar[16];
+      for (int t = 0; t < 16; ++t) {
+        float ar[16];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(Ab + t * PA_P + q4 * 4);
-            ar[q4 * 4 + 0] = a4.x; ar[q4 * 4 + 1] = a4.y; ar[q4 * 4 + 2] = a4.z; ar[q4 * 4 + 3] = a4.w;
-          }
-          float v = (t == c) ? 1.0f : 0.0f;
-#pragma unroll
-          for (int r = 0; r < t; ++r) v = fmaf(-ar[r], x[r], v);
-          x[t] = v;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(Ab + t * PA_P + q4 * 4);
+          ar[q4 * 4 + 0] = a4.x; ar[q4 * 4 + 1] = a4.y; ar[q4 * 4 + 2] = a4.z; ar[q4 * 4 + 3] = a4.w;
         }
+        float v = (t == c) ? 1.0f : 0.0f;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) Tb[t * PA_P + c] = x[t];
+        for (int r = 0; r < t; ++r) v = fmaf(-ar[r], x[r], v);
+        x[t] = v;
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) Tb[t * PA_P + c] = x[t];
+    }
+    __syncthreads();
+    // ... then by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  Item = (head, block
+    // column bj, column quad, row rr); the 16 rows of a quad sit in one half-warp and share the
+    // rows of W = sum_k A_ik T_kj by shuffles.  Blocks above the diagonal are never read.
+    for (int dist = 1; dist < 4; ++dist) {
+      const int per_head = (4 - dist) * 64;
+      for (int g = tid; g < 2 * per_head; g += 256) {  // warp-uniform: per_head is a multiple of 64
+        const int hp = g >= per_head, i = g - hp * per_head;
+        const float* Ah = Am + hp * (64 * PA_P);
+        float* Th = Tm + hp * (64 * PA_P);
+        const int rr = i & 15, cq = ((i >> 4) & 3) * 4, bj = i >> 6, bi = bj + dist;
+        const int ti = bi * 16 + rr, tj = bj * 16 + cq;
+        float4 wv = make_float4(0, 0, 0, 0);
+        for (int kk = bj * 16; kk < bi * 16; kk += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(Ah + ti * PA_P + kk);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 tv = *reinterpret_cast<const float4*>(Th + (kk + u) * PA_P + tj);
+            wv.x = fmaf(av[u], tv.x, wv.x); wv.y = fmaf(av[u], tv.y, wv.y);
+            wv.z = fmaf(av[u], tv.z, wv.z); wv.w = fmaf(av[u], tv.w, wv.w);
+          }
+        }
+        float4 trow[4];  // T_ii row rr
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) trow[q4] = *reinterpret_cast<const float4*>(Th + ti * PA_P + bi * 16 + q4 * 4);
+        float4 res = make_float4(0, 0, 0, 0);
+        const int base = lane & 16;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float tv = m <= rr ? comp(trow[m >> 2], m & 3) : 0.0f;
+          const float w0 = __shfl_sync(0xffffffffu, wv.x, base + m);
+          const float w1 = __shfl_sync(0xffffffffu, wv.y, base + m);
+          const float w2 = __shfl_sync(0xffffffffu, wv.z, base + m);
+          const float w3 = __shfl_sync(0xffffffffu, wv.w, base + m);
+          res.x = fmaf(-tv, w0, res.x); res.y = fmaf(-tv, w1, res.y);
+          res.z = fmaf(-tv, w2, res.z); res.w = fmaf(-tv, w3, res.w);
+        }
+        *reinterpret_cast<float4*>(Th + ti * PA_P + tj) = res;
+      }
+      __syncthreads();
+    }
+    // T of both heads as columns hp * 64 .. of the MN-major B operand of P (over the dead A
+    // matrices), and the T rows of each head's [T;P] output tile (K-major, straight to the
+    // workspace); blocks above the diagonal are zeros.
+    for (int it = tid; it < 2 * 64 * 8; it += 256) {
+      const int hp = it >> 9, r = it & 63, s0 = ((it >> 6) & 7) * 8;
+      float tv[8];
+      if ((s0 >> 4) <= (r >> 4)) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) tv[c] = Tm[hp * (64 * PA_P) + r * PA_P + s0 + c];
       } else {
-        for (int idx = tid - 64; idx < 64 * 16; idx += 192) {  // zero blocks above the diagonal
-          const int t = idx >> 4, s4 = (idx & 15) * 4;
-          if ((s4 >> 4) > (t >> 4)) *reinterpret_cast<float4*>(T + t * PA_P + s4) = make_float4(0, 0, 0, 0);
-        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) tv[c] = 0.0f;
       }
-      __syncthreads();
-      // ... then by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  Item = (block column bj,
-      // column quad, row rr); the 16 rows of a quad sit in one half-warp and share the rows of
-      // W = sum_k A_ik T_kj by shuffles.
-      for (int dist = 1; dist < 4; ++dist) {
-        const int nitems = (4 - dist) * 64;
-        if ((tid & ~31) < nitems) {
-          const int rr = tid & 15, cq = ((tid >> 4) & 3) * 4, bj = tid >> 6, bi = bj + dist;
-          const int ti = bi * 16 + rr, tj = bj * 16 + cq;
-          float4 wv = make_float4(0, 0, 0, 0);
-          for (int kk = bj * 16; kk < bi * 16; kk += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(Am + ti * PA_P + kk);
-            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float4 tv = *reinterpret_cast<const float4*>(T + (kk + u) * PA_P + tj);
-              wv.x = fmaf(av[u], tv.x, wv.x); wv.y = fmaf(av[u], tv.y, wv.y);
-              wv.z = fmaf(av[u], tv.z, wv.z); wv.w = fmaf(av[u], tv.w, wv.w);
-            }
-          }
-          float4 trow[4];  // T_ii row rr
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) trow[q4] = *reinterpret_cast<const float4*>(T + ti * PA_P + bi * 16 + q4 * 4);
-          float4 res = make_float4(0, 0, 0, 0);
-          const int base = lane & 16;
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const float tv = m <= rr ? comp(trow[m >> 2], m & 3) : 0.0f;
-            const float w0 = __shfl_sync(0xffffffffu, wv.x, base + m);
-            const float w1 = __shfl_sync(0xffffffffu, wv.y, base + m);
-            const float w2 = __shfl_sync(0xffffffffu, wv.z, base + m);
-            const float w3 = __shfl_sync(0xffffffffu, wv.w, base + m);
-            res.x = fmaf(-tv, w0, res.x); res.y = fmaf(-tv, w1, res.y);
-            res.z = fmaf(-tv, w2, res.z); res.w = fmaf(-tv, w3, res.w);
-          }
-          *reinterpret_cast<float4*>(T + ti * PA_P + tj) = res;
-        }
-        __syncthreads();
+      uint4 hi, lo;
+      tc::split8(tv, hi, lo);
+      if (hp == 0 || gpair[1] != gpair[0]) {
+        uint8_t* out = tp_ws + ((size_t)chunk * hv + j * G + gpair[hp]) * TP_BYTES;
+        *reinterpret_cast<uint4*>(out + kmaj128(r, s0)) = hi;
+        *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(r, s0)) = lo;
       }
-      // T as columns hp * 64 .. of the MN-major B operand of P, and the T rows of the head's
-      // [T;P] output tile (K-major, straight to the workspace)
-      for (int it = tid; it < 64 * 8; it += 256) {
-        const int r = it & 63, s0 = (it >> 6) * 8;
-        float tv[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) tv[c] = T[r * PA_P + s0 + c];
-        uint4 hi, lo;
-        tc::split8(tv, hi, lo);
-        const uint32_t boff = mnmaj(r, (hp * 64 + s0) >> 3, 64);
-        *reinterpret_cast<uint4*>(pb_hi + boff) = hi;
-        *reinterpret_cast<uint4*>(pb_lo + boff) = lo;
-        if (hp == 0 || gpair[1] != gpair[0]) {
-          uint8_t* out = tp_ws + ((size_t)chunk * hv + j * G + gpair[hp]) * TP_BYTES;
-          *reinterpret_cast<uint4*>(out + kmaj128(r, s0)) = hi;
-          *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(r, s0)) = lo;
-        }
-      }
-      __syncthreads();  // A and T are reused by the next head
+      // the operand overwrites A: every thread must be past its last read of A (the
+      // barrier above) -- and T lies outside the operand, so the reads here are safe
+      const uint32_t boff = mnmaj(r, (hp * 64 + s0) >> 3, 64);
+      *reinterpret_cast<uint4*>(pb_hi + boff) = hi;
+      *reinterpret_cast<uint4*>(pb_lo + boff) = lo;
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
@@ -690,25 +712,40 @@ struct PBStage {  // byte offsets inside one input stage
   static constexpr uint32_t KQ = 0;
   static constexpr uint32_t TP = KQ_BYTES;
   static constexpr uint32_t GB = KQ_BYTES + TP_BYTES;
-  static constexpr uint32_t BV = GB + GB_FLOATS * 4;  // beta * v slice; later the R / U-tilde tile
-  static constexpr uint32_t BYTES = BV + BV_SLICE;
+  static constexpr uint32_t VS = GB + GB_FLOATS * 4;  // v slice; later the R / U-tilde tile
+  static constexpr uint32_t BYTES = VS + VS_SLICE;
 };
 constexpr uint32_t PB_S_TILE = 128 * TC_NV * 2;  // S^T operand (K = 128, N = nv), one of hi/lo
 constexpr uint32_t PB_R_TILE = 64 * TC_NV * 2;   // R / U-tilde operand (K = 64, N = nv): 4 KB
 constexpr size_t PB_TC_SMEM = 2 * (size_t)PB_S_TILE + 2 * (size_t)PBStage::BYTES;
-static_assert(2 * PB_R_TILE == BV_SLICE, "the R / U-tilde tile reuses the beta * v slot");
+static_assert(2 * PB_R_TILE == VS_SLICE, "the R / U-tilde tile reuses the v slot");
+
+// Output modes of phase B: y before the output norm to the workspace (a separate epilogue
+// follows), or the gated RMS norm fused in, with a bf16 or an fp32 y.
+enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 
 // One CTA per (sequence, value head, 32-row state slice); 9 warps: warp w < 8 serves TMEM lane
 // quarter w % 4 and columns 16 (w / 4) .. 16 (w / 4) + 15 of the slice; warp 8 issues the
 // bulk copies of the next chunk.  Each product a b is taken as a_hi [b_hi | b_lo] (one MMA of
 // width 2 nv: the lo tile follows the hi tile at the operand's N stride) plus a_lo b_hi; the
 // epilogue adds the two column halves.
+//
+// Fused output norm (YM != PB_Y_RAW; launched as clusters of the four slices of a value
+// head): the norm of y_t over the head's 128 components ("Qwen3.8-Flash-Next" technical
+// report, Fig. 2: RMS norm of each head's output, gated by SiLU(z)) needs the sums of squares
+// of all four slices.  Each slice adds its two 16-column halves through shared memory, stores
+// the per-token sum into the three other CTAs of the cluster and arrives on their mbarrier;
+// the y values wait in registers and are normalised at the start of the next chunk, while the
+// first MMA round runs, so the exchange stays off the chunk-to-chunk chain.
+template <int YM>
 __global__ void __launch_bounds__(288, 1)
     k_chunkscan_tc(Dims d, const int* __restrict__ cu, const int* __restrict__ seq_chunk0,
                    const uint8_t* __restrict__ kq_ws, const uint8_t* __restrict__ tp_ws,
-                   const float* __restrict__ gb_ws, const float* __restrict__ bv_ws,
-                   const float* init_state, float* __restrict__ y_raw, float* final_state) {
+                   const float* __restrict__ gb_ws, const float* __restrict__ vs_ws,
+                   const float* init_state, float* __restrict__ y_raw, float* final_state,
+                   const uint16_t* __restrict__ z, const float* __restrict__ norm_w, void* __restrict__ y) {
   constexpr int NV = TC_NV, NH = NV / 2;
+  constexpr bool FUSED = YM != PB_Y_RAW;
   const int n = blockIdx.x, h = blockIdx.y, sl = blockIdx.z, i0 = sl * NV;
   const int hq = d.h_qk, hv = d.h_v, G = hv / hq, j = h / G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -726,6 +763,13 @@ __global__ void __launch_bounds__(288, 1)
   __shared__ uint64_t mbar_mma[3];  // one per MMA round: each completes once per chunk
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
+  // fused norm: sums of squares from the three other slices, [chunk parity][peer][token]; the
+  // local hand-off of a token's second column half; one arrival barrier per chunk parity
+  __shared__ float red[FUSED ? 2 * 3 * 64 : 1];
+  __shared__ float handoff[FUSED ? 64 : 1];
+  __shared__ uint64_t red_bar[2];
+  const bool yth = FUSED && !producer && quarter >= 2;  // holds y rows (tokens) of the chunk
+  const int rank = FUSED ? (int)tc::cluster_ctarank() : 0;
 
   // state: thread holds S[i0 + cb + i][row] (row = key component), i < 16
   float S[NH];
@@ -738,6 +782,10 @@ __global__ void __launch_bounds__(288, 1)
     tc::mbar_init(tc::smem_u32(&mbar_ld[0]), 1);
     tc::mbar_init(tc::smem_u32(&mbar_ld[1]), 1);
     for (int q3 = 0; q3 < 3; ++q3) tc::mbar_init(tc::smem_u32(&mbar_mma[q3]), 1);
+    if (FUSED) {
+      tc::mbar_init(tc::smem_u32(&red_bar[0]), 3 * 64);  // 64 sending threads in each peer
+      tc::mbar_init(tc::smem_u32(&red_bar[1]), 3 * 64);
+    }
     tc::fence_mbar_init();
   }
   if (warp == 0) {
@@ -756,7 +804,7 @@ __global__ void __launch_bounds__(288, 1)
     tc::bulk_g2s(dst + PBStage::KQ, kq_ws + (gc * hq + j) * KQ_BYTES, KQ_BYTES, bar);
     tc::bulk_g2s(dst + PBStage::TP, tp_ws + (gc * hv + h) * TP_BYTES, TP_BYTES, bar);
     tc::bulk_g2s(dst + PBStage::GB, gb_ws + (gc * hv + h) * GB_FLOATS, GB_FLOATS * 4, bar);
-    tc::bulk_g2s(dst + PBStage::BV, bv_ws + (gc * hv + h) * (BV_BYTES / 4) + (size_t)sl * (BV_SLICE / 4), BV_SLICE,
+    tc::bulk_g2s(dst + PBStage::VS, vs_ws + (gc * hv + h) * (VS_BYTES / 4) + (size_t)sl * (VS_SLICE / 4), VS_SLICE,
                  bar);
   };
   // S^T operand: thread writes its row (K index = row) for its 16 columns, MN-major
@@ -774,6 +822,7 @@ __global__ void __launch_bounds__(288, 1)
   tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
+  if (FUSED) tc::cluster_sync();  // peers started; their barriers are initialised
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -789,11 +838,60 @@ __global__ void __launch_bounds__(288, 1)
 
   uint32_t ph_ld[2] = {0, 0}, ph_mma = 0;  // ph_mma: parity of this chunk's phase of each round barrier
   bool aborted = false;
+  // fused norm, y threads: the previous chunk's y row (token y_tok, or -1) and its z
+  float yv[NH], own = 0.0f;
+  uint4 zr[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  int y_tok = -1;
+  uint32_t red_ph[2] = {0, 0};
+  // normalise and store the y row held from the chunk with parity `buf`
+  auto finish = [&](int buf) -> bool {
+    const int t = row & 63;
+    const bool ok = tc::mbar_wait_cluster(tc::smem_u32(&red_bar[buf]), red_ph[buf]);
+    red_ph[buf] ^= 1;
+    if (!ok) return false;
+    float tot = 0.0f;  // the same order in every slice: identical norms
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+      tot += rr == rank ? (cb == 0 ? own : handoff[t]) : red[(buf * 3 + (rr < rank ? rr : rr - 1)) * 64 + t];
+    if (y_tok >= 0) {
+      const float inv = rsqrtf(tot * (1.0f / D) + d.rms_eps);
+      const float4* nw4 = reinterpret_cast<const float4*>(norm_w + i0 + cb);
+      const uint32_t zw[8] = {zr[0].x, zr[0].y, zr[0].z, zr[0].w, zr[1].x, zr[1].y, zr[1].z, zr[1].w};
+      float o[NH];
+#pragma unroll
+      for (int q4 = 0; q4 < NH / 4; ++q4) {
+        const float4 w4 = __ldg(nw4 + q4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = q4 * 4 + u;
+          const float zv = bf2f(i & 1 ? zw[i >> 1] >> 16 : zw[i >> 1] & 0xffffu);
+          o[i] = yv[i] * inv * comp(w4, u) * silu_fast(zv);
+        }
+      }
+      const size_t base = ((size_t)y_tok * hv + h) * D + i0 + cb;
+      if (YM == PB_Y_BF16) {
+        uint32_t pw[NH / 2];
+#pragma unroll
+        for (int i = 0; i < NH; i += 2) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i], o[i + 1]);
+          pw[i >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        uint4* yp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + base);
+        yp[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        yp[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      } else {
+        float4* yp = reinterpret_cast<float4*>(static_cast<float*>(y) + base);
+#pragma unroll
+        for (int q4 = 0; q4 < NH / 4; ++q4) yp[q4] = make_float4(o[q4 * 4], o[q4 * 4 + 1], o[q4 * 4 + 2], o[q4 * 4 + 3]);
+      }
+    }
+    return true;
+  };
   for (int c = 0; c < nchunks && !aborted; ++c) {
     const int st = c & 1;
     const int t0 = ts + c * CH, L = min(CH, te - t0);
     uint8_t* sg = stage[st];
-    uint8_t* r_hi = sg + PBStage::BV;
+    uint8_t* r_hi = sg + PBStage::VS;
     uint8_t* r_lo = r_hi + PB_R_TILE;
     const uint32_t kq0 = tc::smem_u32(sg + PBStage::KQ), tp0 = tc::smem_u32(sg + PBStage::TP);
     if (!producer && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
@@ -801,13 +899,13 @@ __global__ void __launch_bounds__(288, 1)
     const float* gsm = reinterpret_cast<const float*>(sg + PBStage::GB);
     const float gL = gsm[L - 1];
     const int t = row & 63;
-    float bvr[NH];  // beta * v of token row t (rows 0..63 only), read before the slot is reused
+    float vr[NH];  // v of token row t (rows 0..63 only), read before the slot is reused
     if (quarter < 2) {
-      const float4* bv = reinterpret_cast<const float4*>(sg + PBStage::BV) + (t * NV + cb) / 4;
+      const float4* vp = reinterpret_cast<const float4*>(sg + PBStage::VS) + (t * NV + cb) / 4;
 #pragma unroll
       for (int q4 = 0; q4 < NH / 4; ++q4) {
-        const float4 x = bv[q4];
-        bvr[q4 * 4 + 0] = x.x; bvr[q4 * 4 + 1] = x.y; bvr[q4 * 4 + 2] = x.z; bvr[q4 * 4 + 3] = x.w;
+        const float4 x = vp[q4];
+        vr[q4 * 4 + 0] = x.x; vr[q4 * 4 + 1] = x.y; vr[q4 * 4 + 2] = x.z; vr[q4 * 4 + 3] = x.w;
       }
     }
     const float eg = t < L ? __expf(gsm[t]) : 0.0f;
@@ -826,6 +924,7 @@ __global__ void __launch_bounds__(288, 1)
       tc::umma_commit(tc::smem_u32(&mbar_mma[0]));
     }
     if (producer && lane == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);  // stage last read by chunk c-1
+    if (yth && c > 0 && !finish((c - 1) & 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     tc::tc_fence_after();
     float qs[NH];  // rows 64..127: e^{gamma_t} (Q S^T)[t][:]
@@ -836,11 +935,11 @@ __global__ void __launch_bounds__(288, 1)
       tc::tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
-      if (quarter < 2) {  // R[t][i] = beta_t v[t][i] - beta_t e^{gamma_t} (K S^T)[t][i]
-        const float be = t < L ? gsm[64 + t] * eg : 0.0f;
+      if (quarter < 2) {  // R[t][i] = beta_t (v[t][i] - e^{gamma_t} (K S^T)[t][i])
+        const float bt = t < L ? gsm[64 + t] : 0.0f;
         float rr[NH];
 #pragma unroll
-        for (int i = 0; i < NH; ++i) rr[i] = t < L ? fmaf(-be, __uint_as_float(r[i]), bvr[i]) : 0.0f;
+        for (int i = 0; i < NH; ++i) rr[i] = t < L ? bt * fmaf(-eg, __uint_as_float(r[i]), vr[i]) : 0.0f;
 #pragma unroll
         for (int q8 = 0; q8 < 2; ++q8) {
           uint4 hi, lo;
@@ -892,14 +991,43 @@ __global__ void __launch_bounds__(288, 1)
           *reinterpret_cast<uint4*>(r_hi + off) = hi;
           *reinterpret_cast<uint4*>(r_lo + off) = lo;
         }
-      } else if (t < L) {  // Y = e^gamma Q S^T + (M o QK^T) U
-        float4* yr = reinterpret_cast<float4*>(y_raw + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
+      } else if (!FUSED) {  // Y = e^gamma Q S^T + (M o QK^T) U
+        if (t < L) {
+          float4* yr = reinterpret_cast<float4*>(y_raw + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
 #pragma unroll
-        for (int q4 = 0; q4 < NH / 4; ++q4)
-          yr[q4] = make_float4(qs[q4 * 4 + 0] + __uint_as_float(r[q4 * 4 + 0]),
-                               qs[q4 * 4 + 1] + __uint_as_float(r[q4 * 4 + 1]),
-                               qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]),
-                               qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]));
+          for (int q4 = 0; q4 < NH / 4; ++q4)
+            yr[q4] = make_float4(qs[q4 * 4 + 0] + __uint_as_float(r[q4 * 4 + 0]),
+                                 qs[q4 * 4 + 1] + __uint_as_float(r[q4 * 4 + 1]),
+                                 qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]),
+                                 qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]));
+        }
+      } else {  // the same y, kept until the four slices' sums of squares are in
+        float p = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NH; ++i) {
+          yv[i] = t < L ? qs[i] + __uint_as_float(r[i]) : 0.0f;
+          p = fmaf(yv[i], yv[i], p);
+        }
+        y_tok = t < L ? t0 + t : -1;
+        if (t < L) {
+          const uint4* zp = reinterpret_cast<const uint4*>(z + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
+          zr[0] = __ldg(zp);
+          zr[1] = __ldg(zp + 1);
+        }
+        const int buf = c & 1;
+        if (cb != 0) handoff[t] = p;
+        named_bar_sync(quarter, 64);  // warps (2, 6) and (3, 7): the two halves of a token
+        if (cb == 0) {
+          own = p + handoff[t];
+          handoff[t] = own;
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            if (rr == rank) continue;
+            const int slot = rank < rr ? rank : rank - 1;  // this slice's slot in peer rr
+            tc::st_cluster_f32(tc::mapa(tc::smem_u32(&red[(buf * 3 + slot) * 64 + t]), (uint32_t)rr), own);
+            tc::mbar_arrive_remote(tc::mapa(tc::smem_u32(&red_bar[buf]), (uint32_t)rr));
+          }
+        }
       }
     }
     tc::fence_proxy_async();
@@ -936,6 +1064,7 @@ __global__ void __launch_bounds__(288, 1)
     __syncthreads();
     if (s_abort) { aborted = true; break; }
   }
+  if (!aborted && yth && nchunks > 0 && !finish((nchunks - 1) & 1)) atomicExch(&g_gdn_status, -7);
   if (!aborted && !producer) {
 #pragma unroll
     for (int i = 0; i < NH; ++i) final_state[sbase + (size_t)(cb + i) * D + row] = S[i];
@@ -943,6 +1072,7 @@ __global__ void __launch_bounds__(288, 1)
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tbase, 256);
+  if (FUSED) tc::cluster_sync();  // no CTA leaves while a peer may still write to it
 }
 
 }  // namespace gdn

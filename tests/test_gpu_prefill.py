@@ -162,3 +162,22 @@ def test_tensor_core_and_fp32_paths_agree(monkeypatch):
     r = float(np.sqrt(np.mean(y_s ** 2)))
     assert np.abs(y_tc - y_s).max() <= 2e-2 * r
     assert np.linalg.norm(S_tc - S_s) / np.linalg.norm(S_s) <= 1e-2
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_fused_output_norm_matches_separate_epilogue(oracle_mod, monkeypatch, out_dtype):
+    """The gated RMS norm fused into the state pass (clusters of the four slices of a head
+    exchange their sums of squares) against the same norm in its own kernel, and both
+    against the oracle; lengths include empty sequences and partial chunks."""
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[0, 130, 1, 64, 0, 77], h_qk=4, h_v=8)
+    ref = _oracle(oracle_mod, inp)
+    y_f, S_f = run_prefill(inp, out_dtype)
+    monkeypatch.setenv("GDN_NO_FUSED_NORM", "1")
+    y_e, S_e = run_prefill(inp, out_dtype)
+    is_bf16 = out_dtype == torch.bfloat16
+    check_bf16(y_f, ref["y"], S_f, ref["final_state"], y_is_bf16=is_bf16)
+    check_bf16(y_e, ref["y"], S_e, ref["final_state"], y_is_bf16=is_bf16)
+    assert np.array_equal(S_f, S_e)
+    r = float(np.sqrt(np.mean(ref["y"] ** 2)))
+    tol = 1e-5 * r if out_dtype == torch.float32 else 2.0 ** -8 * np.abs(ref["y"]).max()
+    assert np.abs(y_f - y_e).max() <= tol
