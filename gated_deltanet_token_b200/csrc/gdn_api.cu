@@ -207,7 +207,7 @@ int scan_clusters_per_wave() {
   if (known.load() & bit) return cached[dev & 63];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, 1, D / TC_NV);
-  cfg.blockDim = dim3(288);
+  cfg.blockDim = dim3(384);
   cfg.dynamicSmemBytes = PB_TC_SMEM;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
@@ -330,7 +330,7 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
       ProfScope p("chunk_scan_tc_norm", s);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = grid;
-      cfg.blockDim = dim3(288);
+      cfg.blockDim = dim3(384);
       cfg.dynamicSmemBytes = PB_TC_SMEM;
       cfg.stream = s;
       cudaLaunchAttribute attr;

@@ -724,25 +724,30 @@ static_assert(2 * PB_R_TILE == VS_SLICE, "the R / U-tilde tile reuses the v slot
 // follows), or the gated RMS norm fused in, with a bf16 or an fp32 y.
 enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 
-// One CTA per (sequence, value head, 32-row state slice); 9 warps: warp w < 8 serves TMEM lane
-// quarter w % 4 and columns 16 (w / 4) .. 16 (w / 4) + 15 of the slice; warp 8 issues the
+// One CTA per (sequence, value head, 32-row state slice).  Warps 0..7 ("workers") serve TMEM
+// lane quarter w % 4 and columns 16 (w / 4) .. 16 (w / 4) + 15 of the slice; warp 8 issues the
 // bulk copies of the next chunk.  Each product a b is taken as a_hi [b_hi | b_lo] (one MMA of
 // width 2 nv: the lo tile follows the hi tile at the operand's N stride) plus a_lo b_hi; the
 // epilogue adds the two column halves.
+
 //
-// Fused output norm (YM != PB_Y_RAW; launched as clusters of the four slices of a value
-// head): the norm of y_t over the head's 128 components ("Qwen3.8-Flash-Next" technical
-// report, Fig. 2: RMS norm of each head's output, gated by SiLU(z)) needs the sums of squares
-// of all four slices.  Each slice adds its two 16-column halves through shared memory, stores
-// the per-token sum into the three other CTAs of the cluster and arrives on their mbarrier;
-// the y values wait in registers and are normalised at the start of the next chunk, while the
-// first MMA round runs, so the exchange stays off the chunk-to-chunk chain.
+// Fused output norm (YM != PB_Y_RAW; clusters of the four slices of a value head; 12 warps):
+// warps 10 and 11 own TMEM lanes 64..127, i.e. the 64 tokens' y rows, and take the whole y
+// path, so the workers only carry the state chain.  The norm of y_t over the head's 128
+// components ("Qwen3.8-Flash-Next" technical report, Fig. 2: RMS norm of each head's output,
+// gated by SiLU(z)) needs the sums of squares of all four slices: each norm thread stores its
+// token's sum into the three other CTAs of the cluster as one 32-bit word whose two low bits
+// carry a chunk tag (the value is the flag: no fence or barrier between CTAs).  Its y row
+// waits in registers and is normalised in the next chunk, while that chunk's second MMA
+// round runs.  Every slice sums the
+// same four tag-stripped words in rank order, so all four use the same norm.  Warp 9 idles.
 template <int YM>
-__global__ void __launch_bounds__(288, 1)
+__global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     k_chunkscan_tc(Dims d, const int* __restrict__ cu, const int* __restrict__ seq_chunk0,
                    const uint8_t* __restrict__ kq_ws, const uint8_t* __restrict__ tp_ws,
                    const float* __restrict__ gb_ws, const float* __restrict__ vs_ws,
-                   const float* init_state, float* __restrict__ y_raw, float* final_state,
+                   const float* init_state, float* __restrict__ y_raw,
+                   float* final_state,
                    const uint16_t* __restrict__ z, const float* __restrict__ norm_w, void* __restrict__ y) {
   constexpr int NV = TC_NV, NH = NV / 2;
   constexpr bool FUSED = YM != PB_Y_RAW;
@@ -750,7 +755,9 @@ __global__ void __launch_bounds__(288, 1)
   const int hq = d.h_qk, hv = d.h_v, G = hv / hq, j = h / G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, cb = ((warp >> 2) & 1) * NH;
-  const bool producer = warp == 8;
+  const bool worker = warp < 8, producer = warp == 8;
+  const bool normw = FUSED && warp >= 10;  // y rows of tokens 32 (warp - 10) + lane
+  const bool rwarp = worker && quarter < 2;  // token rows 0..63: R and U-tilde
   const int row = quarter * 32 + lane;  // TMEM lane: accumulator row
   const int ts = cu ? cu[n] : 0, te = cu ? cu[n + 1] : d.total_tokens;
   const int nchunks = te > ts ? (te - ts + CH - 1) / CH : 0;
@@ -763,29 +770,27 @@ __global__ void __launch_bounds__(288, 1)
   __shared__ uint64_t mbar_mma[3];  // one per MMA round: each completes once per chunk
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
-  // fused norm: sums of squares from the three other slices, [chunk parity][peer][token]; the
-  // local hand-off of a token's second column half; one arrival barrier per chunk parity
-  __shared__ float red[FUSED ? 2 * 3 * 64 : 1];
-  __shared__ float handoff[FUSED ? 64 : 1];
-  __shared__ uint64_t red_bar[2];
-  const bool yth = FUSED && !producer && quarter >= 2;  // holds y rows (tokens) of the chunk
+  // fused norm: tagged sums of squares from the three other slices, [chunk parity][peer][token]
+  __shared__ uint32_t red[FUSED ? 2 * 3 * 64 : 1];
   const int rank = FUSED ? (int)tc::cluster_ctarank() : 0;
 
-  // state: thread holds S[i0 + cb + i][row] (row = key component), i < 16
-  float S[NH];
+  if (FUSED && tc::cluster_nctarank() != D / NV) {  // launched without its clusters: no exchange
+    if (tid == 0) atomicExch(&g_gdn_status, -6);
+    return;
+  }
+  // keep: a worker's state S[i0 + cb + i][row] (row = key component) in keep[0..15]; a norm
+  // thread's pending y row in keep[0..31] (one register array serves both roles)
+  float keep[NV];
+  float* S = keep;
   const size_t sbase = (((size_t)n * hv + h) * D + i0) * D;
 #pragma unroll
-  for (int i = 0; i < NH; ++i) S[i] = (init_state && !producer) ? init_state[sbase + (size_t)(cb + i) * D + row] : 0.0f;
+  for (int i = 0; i < NH; ++i) S[i] = (init_state && worker) ? init_state[sbase + (size_t)(cb + i) * D + row] : 0.0f;
 
   if (tid == 0) {
     s_abort = 0;
     tc::mbar_init(tc::smem_u32(&mbar_ld[0]), 1);
     tc::mbar_init(tc::smem_u32(&mbar_ld[1]), 1);
     for (int q3 = 0; q3 < 3; ++q3) tc::mbar_init(tc::smem_u32(&mbar_mma[q3]), 1);
-    if (FUSED) {
-      tc::mbar_init(tc::smem_u32(&red_bar[0]), 3 * 64);  // 64 sending threads in each peer
-      tc::mbar_init(tc::smem_u32(&red_bar[1]), 3 * 64);
-    }
     tc::fence_mbar_init();
   }
   if (warp == 0) {
@@ -796,11 +801,12 @@ __global__ void __launch_bounds__(288, 1)
   auto named_bar_sync = [](int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
   };
+  // (producer warp, lane 0) copies of chunk c into stage st
   auto issue_load = [&](int c, int st) {
     const size_t gc = (size_t)gc0 + c;
     const uint32_t bar = tc::smem_u32(&mbar_ld[st]);
-    tc::mbar_arrive_expect_tx(bar, PBStage::BYTES);
     const uint32_t dst = tc::smem_u32(stage[st]);
+    tc::mbar_arrive_expect_tx(bar, PBStage::BYTES);
     tc::bulk_g2s(dst + PBStage::KQ, kq_ws + (gc * hq + j) * KQ_BYTES, KQ_BYTES, bar);
     tc::bulk_g2s(dst + PBStage::TP, tp_ws + (gc * hv + h) * TP_BYTES, TP_BYTES, bar);
     tc::bulk_g2s(dst + PBStage::GB, gb_ws + (gc * hv + h) * GB_FLOATS, GB_FLOATS * 4, bar);
@@ -818,11 +824,13 @@ __global__ void __launch_bounds__(288, 1)
       *reinterpret_cast<uint4*>(s_lo + off) = lo;
     }
   };
-  if (!producer) write_s_tile();
+  if (worker) write_s_tile();
+  if (FUSED)
+    for (int i = tid; i < 2 * 3 * 64; i += blockDim.x) red[i] = 3u;  // tag 3: no chunk yet
   tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
-  if (FUSED) tc::cluster_sync();  // peers started; their barriers are initialised
+  if (FUSED) tc::cluster_sync();  // peers started; their exchange words are initialised
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -838,51 +846,62 @@ __global__ void __launch_bounds__(288, 1)
 
   uint32_t ph_ld[2] = {0, 0}, ph_mma = 0;  // ph_mma: parity of this chunk's phase of each round barrier
   bool aborted = false;
-  // fused norm, y threads: the previous chunk's y row (token y_tok, or -1) and its z
-  float yv[NH], own = 0.0f;
-  uint4 zr[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  // fused norm, norm threads: the previous chunk's y row (in keep, token y_tok, or -1)
+  float* yv = keep;
+  float own = 0.0f;
   int y_tok = -1;
-  uint32_t red_ph[2] = {0, 0};
-  // normalise and store the y row held from the chunk with parity `buf`
-  auto finish = [&](int buf) -> bool {
-    const int t = row & 63;
-    const bool ok = tc::mbar_wait_cluster(tc::smem_u32(&red_bar[buf]), red_ph[buf]);
-    red_ph[buf] ^= 1;
-    if (!ok) return false;
-    float tot = 0.0f;  // the same order in every slice: identical norms
+  auto untag = [](uint32_t w) { return __uint_as_float(w & ~3u); };
+  const uint32_t t_norm = tbase + ((uint32_t)(64 + 32 * (warp & 1)) << 16);  // norm warps: lanes 64.. / 96..
+  // normalise and store the y row held from chunk cy (bounded wait for the peers' words)
+  auto finish = [&](int cy) -> bool {
+    const int t = row & 63, buf = cy & 1;
+    const uint32_t tag = (uint32_t)(cy >> 1) & 3u;
+    const uint32_t a0 = tc::smem_u32(&red[(buf * 3) * 64 + t]);
+    uint32_t w[3];
+    uint64_t t_start = 0;
+    for (;;) {
+#pragma unroll
+      for (int p = 0; p < 3; ++p) w[p] = tc::ld_volatile_shared(a0 + p * 64 * 4);
+      if ((w[0] & 3u) == tag && (w[1] & 3u) == tag && (w[2] & 3u) == tag) break;
+      __nanosleep(64);
+      uint64_t now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t_start == 0) t_start = now;
+      else if (now - t_start > 2000000000ull) return false;
+    }
+    float tot = 0.0f;  // the same words in the same order in every slice: identical norms
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr)
-      tot += rr == rank ? (cb == 0 ? own : handoff[t]) : red[(buf * 3 + (rr < rank ? rr : rr - 1)) * 64 + t];
+      tot += rr == rank ? own : untag(rr < rank ? w[rr < 3 ? rr : 2] : w[rr > 0 ? rr - 1 : 0]);
     if (y_tok >= 0) {
       const float inv = rsqrtf(tot * (1.0f / D) + d.rms_eps);
-      const float4* nw4 = reinterpret_cast<const float4*>(norm_w + i0 + cb);
-      const uint32_t zw[8] = {zr[0].x, zr[0].y, zr[0].z, zr[0].w, zr[1].x, zr[1].y, zr[1].z, zr[1].w};
-      float o[NH];
+      const float4* nw4 = reinterpret_cast<const float4*>(norm_w + i0);
+      const size_t base = ((size_t)y_tok * hv + h) * D + i0;
+      const uint4* zp = reinterpret_cast<const uint4*>(z + base);  // prefetched into L2 at round 2
 #pragma unroll
-      for (int q4 = 0; q4 < NH / 4; ++q4) {
-        const float4 w4 = __ldg(nw4 + q4);
+      for (int g8 = 0; g8 < NV / 8; ++g8) {  // 8 columns at a time
+        const uint4 zq = __ldg(zp + g8);
+        const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+        const float4 wa = __ldg(nw4 + 2 * g8), wb = __ldg(nw4 + 2 * g8 + 1);
+        float o[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = q4 * 4 + u;
-          const float zv = bf2f(i & 1 ? zw[i >> 1] >> 16 : zw[i >> 1] & 0xffffu);
-          o[i] = yv[i] * inv * comp(w4, u) * silu_fast(zv);
+        for (int u = 0; u < 8; ++u) {
+          const float zv = bf2f(u & 1 ? zw[u >> 1] >> 16 : zw[u >> 1] & 0xffffu);
+          o[u] = yv[g8 * 8 + u] * inv * comp(u < 4 ? wa : wb, u & 3) * silu_fast(zv);
         }
-      }
-      const size_t base = ((size_t)y_tok * hv + h) * D + i0 + cb;
-      if (YM == PB_Y_BF16) {
-        uint32_t pw[NH / 2];
+        if (YM == PB_Y_BF16) {
+          uint32_t pw[4];
 #pragma unroll
-        for (int i = 0; i < NH; i += 2) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i], o[i + 1]);
-          pw[i >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+          for (int u = 0; u < 8; u += 2) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[u], o[u + 1]);
+            pw[u >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + base)[g8] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        } else {
+          float4* yp = reinterpret_cast<float4*>(static_cast<float*>(y) + base) + 2 * g8;
+          yp[0] = make_float4(o[0], o[1], o[2], o[3]);
+          yp[1] = make_float4(o[4], o[5], o[6], o[7]);
         }
-        uint4* yp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + base);
-        yp[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-        yp[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-      } else {
-        float4* yp = reinterpret_cast<float4*>(static_cast<float*>(y) + base);
-#pragma unroll
-        for (int q4 = 0; q4 < NH / 4; ++q4) yp[q4] = make_float4(o[q4 * 4], o[q4 * 4 + 1], o[q4 * 4 + 2], o[q4 * 4 + 3]);
       }
     }
     return true;
@@ -894,13 +913,13 @@ __global__ void __launch_bounds__(288, 1)
     uint8_t* r_hi = sg + PBStage::VS;
     uint8_t* r_lo = r_hi + PB_R_TILE;
     const uint32_t kq0 = tc::smem_u32(sg + PBStage::KQ), tp0 = tc::smem_u32(sg + PBStage::TP);
-    if (!producer && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    if ((worker || normw) && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_ld[st] ^= 1;
     const float* gsm = reinterpret_cast<const float*>(sg + PBStage::GB);
     const float gL = gsm[L - 1];
     const int t = row & 63;
-    float vr[NH];  // v of token row t (rows 0..63 only), read before the slot is reused
-    if (quarter < 2) {
+    float vr[NH];  // R threads: v of token row t, read before the slot is reused
+    if (rwarp) {
       const float4* vp = reinterpret_cast<const float4*>(sg + PBStage::VS) + (t * NV + cb) / 4;
 #pragma unroll
       for (int q4 = 0; q4 < NH / 4; ++q4) {
@@ -924,11 +943,10 @@ __global__ void __launch_bounds__(288, 1)
       tc::umma_commit(tc::smem_u32(&mbar_mma[0]));
     }
     if (producer && lane == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);  // stage last read by chunk c-1
-    if (yth && c > 0 && !finish((c - 1) & 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     tc::tc_fence_after();
-    float qs[NH];  // rows 64..127: e^{gamma_t} (Q S^T)[t][:]
-    if (!producer) {
+    float qs[FUSED ? NV : NH];  // y rows: e^{gamma_t} (Q S^T)[t][:] (workers: 16 columns, norm warps: 32)
+    if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
       tc::tmem_ld16(t_a, r);
       tc::tmem_ld16(t_a + NV, r2);
@@ -952,10 +970,21 @@ __global__ void __launch_bounds__(288, 1)
 #pragma unroll
         for (int i = 0; i < NH; ++i) qs[i] = eg * __uint_as_float(r[i]);
       }
+    } else if (normw) {  // all 32 columns of the token's y row, 16 at a time
+#pragma unroll
+      for (int h16 = 0; h16 < 2; ++h16) {
+        uint32_t r[16], r2[16];
+        tc::tmem_ld16(t_norm + 16 * h16, r);
+        tc::tmem_ld16(t_norm + NV + 16 * h16, r2);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) qs[16 * h16 + i] = eg * (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
+      }
+      if (c > 0 && !finish(c - 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }  // while round 2 runs
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
-    if (quarter < 2 && !producer) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
+    if (rwarp) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 2: [U ; (M o QK^T) U] = [T;P] (128 x 64) x R (K = 64, N = nv) ----------------
     if (tid == 0) {
       tc::tc_fence_after();
@@ -971,7 +1000,7 @@ __global__ void __launch_bounds__(288, 1)
     }
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     tc::tc_fence_after();
-    if (!producer) {
+    if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
       tc::tmem_ld16(t_cd, r);
       tc::tmem_ld16(t_cd + NV, r2);
@@ -991,48 +1020,46 @@ __global__ void __launch_bounds__(288, 1)
           *reinterpret_cast<uint4*>(r_hi + off) = hi;
           *reinterpret_cast<uint4*>(r_lo + off) = lo;
         }
-      } else if (!FUSED) {  // Y = e^gamma Q S^T + (M o QK^T) U
-        if (t < L) {
-          float4* yr = reinterpret_cast<float4*>(y_raw + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
+      } else if (t < L) {  // Y = e^gamma Q S^T + (M o QK^T) U, before the output norm
+        float4* yr = reinterpret_cast<float4*>(y_raw + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
 #pragma unroll
-          for (int q4 = 0; q4 < NH / 4; ++q4)
-            yr[q4] = make_float4(qs[q4 * 4 + 0] + __uint_as_float(r[q4 * 4 + 0]),
-                                 qs[q4 * 4 + 1] + __uint_as_float(r[q4 * 4 + 1]),
-                                 qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]),
-                                 qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]));
-        }
-      } else {  // the same y, kept until the four slices' sums of squares are in
-        float p = 0.0f;
+        for (int q4 = 0; q4 < NH / 4; ++q4)
+          yr[q4] = make_float4(qs[q4 * 4 + 0] + __uint_as_float(r[q4 * 4 + 0]),
+                               qs[q4 * 4 + 1] + __uint_as_float(r[q4 * 4 + 1]),
+                               qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]),
+                               qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]));
+      }
+    } else if (normw) {  // the same y, kept until the four slices' sums of squares are in
+      float p = 0.0f;
 #pragma unroll
-        for (int i = 0; i < NH; ++i) {
-          yv[i] = t < L ? qs[i] + __uint_as_float(r[i]) : 0.0f;
-          p = fmaf(yv[i], yv[i], p);
-        }
-        y_tok = t < L ? t0 + t : -1;
-        if (t < L) {
-          const uint4* zp = reinterpret_cast<const uint4*>(z + ((size_t)(t0 + t) * hv + h) * D + i0 + cb);
-          zr[0] = __ldg(zp);
-          zr[1] = __ldg(zp + 1);
-        }
-        const int buf = c & 1;
-        if (cb != 0) handoff[t] = p;
-        named_bar_sync(quarter, 64);  // warps (2, 6) and (3, 7): the two halves of a token
-        if (cb == 0) {
-          own = p + handoff[t];
-          handoff[t] = own;
+      for (int h16 = 0; h16 < 2; ++h16) {
+        uint32_t r[16], r2[16];
+        tc::tmem_ld16(t_norm + 2 * NV + 16 * h16, r);
+        tc::tmem_ld16(t_norm + 3 * NV + 16 * h16, r2);
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int rr = 0; rr < 4; ++rr) {
-            if (rr == rank) continue;
-            const int slot = rank < rr ? rank : rank - 1;  // this slice's slot in peer rr
-            tc::st_cluster_f32(tc::mapa(tc::smem_u32(&red[(buf * 3 + slot) * 64 + t]), (uint32_t)rr), own);
-            tc::mbar_arrive_remote(tc::mapa(tc::smem_u32(&red_bar[buf]), (uint32_t)rr));
-          }
+        for (int i = 0; i < 16; ++i) {
+          const int k = 16 * h16 + i;
+          yv[k] = t < L ? qs[k] + (__uint_as_float(r[i]) + __uint_as_float(r2[i])) : 0.0f;
+          p = fmaf(yv[k], yv[k], p);
         }
       }
+      y_tok = t < L ? t0 + t : -1;
+      const int buf = c & 1;
+      const uint32_t word = (__float_as_uint(p) & ~3u) | ((uint32_t)(c >> 1) & 3u);
+      own = untag(word);
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        if (rr == rank) continue;
+        const int slot = rank < rr ? rank : rank - 1;  // this slice's slot in peer rr
+        tc::st_cluster_u32(tc::mapa(tc::smem_u32(&red[(buf * 3 + slot) * 64 + t]), (uint32_t)rr), word);
+      }
+      if (t < L)  // z of this row, read by the norm at the next chunk's start
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(z + ((size_t)(t0 + t) * hv + h) * D + i0));
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
-    if (quarter < 2 && !producer) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
+    if (rwarp) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 3: K^T U-tilde: A = MN-major view of the K rows (M = 128 key comps, K = 64 tokens)
     if (tid == 0) {
       tc::tc_fence_after();
@@ -1049,7 +1076,7 @@ __global__ void __launch_bounds__(288, 1)
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[2]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_mma ^= 1;
     tc::tc_fence_after();
-    if (!producer) {
+    if (worker) {
       uint32_t r[16], r2[16];
       tc::tmem_ld16(t_e, r);
       tc::tmem_ld16(t_e + NV, r2);
@@ -1064,8 +1091,8 @@ __global__ void __launch_bounds__(288, 1)
     __syncthreads();
     if (s_abort) { aborted = true; break; }
   }
-  if (!aborted && yth && nchunks > 0 && !finish((nchunks - 1) & 1)) atomicExch(&g_gdn_status, -7);
-  if (!aborted && !producer) {
+  if (!aborted && normw && nchunks > 0 && !finish(nchunks - 1)) atomicExch(&g_gdn_status, -7);
+  if (!aborted && worker) {
 #pragma unroll
     for (int i = 0; i < NH; ++i) final_state[sbase + (size_t)(cb + i) * D + row] = S[i];
   }

@@ -125,8 +125,9 @@ const char* gdn_status_string(int code);
 
 /*
  * Synchronises `stream`, then returns and clears the library's device status word for
- * the current device: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a bounded device-side wait
- * gave up since the last read.  Returns GDN_ERR_CUDA if the synchronisation fails.
+ * the current device: GDN_OK, GDN_ERR_DEVICE_TIMEOUT if a bounded device-side wait gave up
+ * since the last read, or GDN_ERR_CUDA if a kernel found its launch shape inconsistent and
+ * did nothing.  Returns GDN_ERR_CUDA also if the synchronisation fails.
  */
 int gdn_read_device_status(gdn_stream_t stream);
 
