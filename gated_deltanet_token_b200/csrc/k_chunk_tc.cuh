@@ -199,12 +199,16 @@ struct ProItem {
   int ch0;  // first conv channel of the group
 };
 
-__device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry* tab, int it, int ngroups) {
+// Chunk slot of work item `it`.
+__device__ __forceinline__ int pro_chunk(int it, int ngroups) { return (it / ngroups) >> 1; }
+
+// Work item `it`, given its chunk-table entry e = tab[pro_chunk(it, ngroups)].
+__device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry& e, int it, int ngroups) {
   ProItem w;
   const int grp = it % ngroups, hc = it / ngroups;
   w.chunk = hc >> 1;
   w.tb0 = (hc & 1) * PRO_TOK;
-  w.e = tab[w.chunk];
+  w.e = e;
   const int hq = d.h_qk, nqg = (hq + PRO_HG - 1) / PRO_HG;
   w.stream = grp < nqg ? 0 : grp < 2 * nqg ? 1 : 2;
   w.nheads = w.stream == 2 ? d.h_v : hq;
@@ -235,10 +239,11 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     tc::fence_mbar_init();
   }
   __syncthreads();
-  // (warp 0, all lanes) describe item `it` in s_item[st] and issue its copies into stage
-  // `st`: lane l copies token rows l and l + 32.  Unused chunk slots copy nothing.
-  auto issue = [&](int it, int st) -> bool {  // true if copies were issued
-    const ProItem w = pro_item(d, tab, it, ngroups);
+  // (warp 0, all lanes) describe item `it` (chunk-table entry e) in s_item[st] and issue its
+  // copies into stage `st`: lane l copies token rows l and l + 32.  Unused chunk slots copy
+  // nothing.
+  auto issue = [&](int it, const ChunkEntry& e, int st) -> bool {  // true if copies were issued
+    const ProItem w = pro_item(d, e, it, ngroups);
     if (lane == 0) s_item[st] = w;
     if (w.e.len == 0) return false;
     const uint16_t* src = w.stream == 0 ? q : w.stream == 1 ? k : v;
@@ -270,14 +275,24 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     return true;
   };
   bool pending[2] = {false, false};  // (warp 0) copies in flight per stage
-  if (warp == 0 && (int)blockIdx.x < nitems) pending[0] = issue(blockIdx.x, 0);
+  // warp 0 reads the table entry of the item after the one it issues next, one item ahead, so
+  // that the load's latency hides behind the current item's work
+  const int g = gridDim.x;
+  ChunkEntry e_next{};
+  if (warp == 0 && (int)blockIdx.x < nitems) {
+    pending[0] = issue(blockIdx.x, tab[pro_chunk(blockIdx.x, ngroups)], 0);
+    if ((int)blockIdx.x + g < nitems) e_next = tab[pro_chunk(blockIdx.x + g, ngroups)];
+  }
   __syncthreads();
   uint32_t parity[2] = {0, 0};
   int n = 0;
   for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
     const int st = n & 1;
     const ProItem w = s_item[st];
-    if (warp == 0 && it + (int)gridDim.x < nitems) pending[st ^ 1] = issue(it + gridDim.x, st ^ 1);
+    if (warp == 0 && it + g < nitems) {
+      pending[st ^ 1] = issue(it + g, e_next, st ^ 1);
+      if (it + 2 * g < nitems) e_next = tab[pro_chunk(it + 2 * g, ngroups)];
+    }
     if (w.e.len == 0) {
       __syncthreads();
       continue;
@@ -414,7 +429,8 @@ constexpr uint32_t PA_OFF_PB = 32768;
 constexpr uint32_t PA_OFF_A = 32768;
 constexpr uint32_t PA_OFF_T = PA_OFF_A + 2 * PA_MAT;
 constexpr uint32_t PA_OFF_G = PA_OFF_T + 2 * PA_MAT;
-constexpr size_t PA_TC_SMEM = PA_OFF_G + 4 * 64 * 4;
+constexpr uint32_t PA_OFF_W = PA_OFF_G + 4 * 64 * 4;  // [16 half-warps][16 rows] float4 scratch
+constexpr size_t PA_TC_SMEM = PA_OFF_W + 16 * 16 * 16;
 static_assert(PA_OFF_T >= KQ_BYTES, "T and the gates lie past the [K;Q] tile");
 static_assert(PA_TC_SMEM <= 113 * 1024, "two phase-A CTAs per SM");
 
@@ -442,6 +458,7 @@ __global__ void __launch_bounds__(256, 2)
   float* Tm = reinterpret_cast<float*>(sm + PA_OFF_T);  // [2][64][PA_P]
   float* gs = reinterpret_cast<float*>(sm + PA_OFF_G);  // [2][64] gamma
   float* bs = gs + 128;                                 // [2][64] beta
+  float4* wsc = reinterpret_cast<float4*>(sm + PA_OFF_W) + (tid >> 4) * 16;  // this half-warp's rows
   __shared__ uint64_t mbar;
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
@@ -589,7 +606,8 @@ __global__ void __launch_bounds__(256, 2)
     __syncthreads();
     // ... then by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  Item = (head, block
     // column bj, column quad, row rr); the 16 rows of a quad sit in one half-warp and share the
-    // rows of W = sum_k A_ik T_kj by shuffles.  Blocks above the diagonal are never read.
+    // rows of W = sum_k A_ik T_kj through shared memory.  Blocks above the diagonal are never
+    // read.
     for (int dist = 1; dist < 4; ++dist) {
       const int per_head = (4 - dist) * 64;
       for (int g = tid; g < 2 * per_head; g += 256) {  // warp-uniform: per_head is a multiple of 64
@@ -612,18 +630,17 @@ __global__ void __launch_bounds__(256, 2)
         float4 trow[4];  // T_ii row rr
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) trow[q4] = *reinterpret_cast<const float4*>(Th + ti * PA_P + bi * 16 + q4 * 4);
+        wsc[rr] = wv;
+        __syncwarp();
         float4 res = make_float4(0, 0, 0, 0);
-        const int base = lane & 16;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
           const float tv = m <= rr ? comp(trow[m >> 2], m & 3) : 0.0f;
-          const float w0 = __shfl_sync(0xffffffffu, wv.x, base + m);
-          const float w1 = __shfl_sync(0xffffffffu, wv.y, base + m);
-          const float w2 = __shfl_sync(0xffffffffu, wv.z, base + m);
-          const float w3 = __shfl_sync(0xffffffffu, wv.w, base + m);
-          res.x = fmaf(-tv, w0, res.x); res.y = fmaf(-tv, w1, res.y);
-          res.z = fmaf(-tv, w2, res.z); res.w = fmaf(-tv, w3, res.w);
+          const float4 w = wsc[m];
+          res.x = fmaf(-tv, w.x, res.x); res.y = fmaf(-tv, w.y, res.y);
+          res.z = fmaf(-tv, w.z, res.z); res.w = fmaf(-tv, w.w, res.w);
         }
+        __syncwarp();  // the rows are read before the next item of this half-warp writes them
         *reinterpret_cast<float4*>(Th + ti * PA_P + tj) = res;
       }
       __syncthreads();
