@@ -6,6 +6,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cudaTypedefs.h>
+
 #include <atomic>
 #include <type_traits>
 
@@ -165,6 +167,37 @@ Dims kdims(const gdn_dims_t* d) {
 
 int g_num_sms = 148;  // SM count of the current device (set by configure_device)
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+  if (f) return f;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !p)
+    return nullptr;
+  f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  fn.store(f);
+  return f;
+}
+
+// Tensor map of a bf16 stream [T][nheads][128] for the prologue's box of 128 channels x
+// PRO_HG heads x PRO_ROWS tokens (elements outside the tensor read as zeros).
+int make_stream_map(CUtensorMap* m, const void* x, int T, int nheads) {
+  memset(m, 0, sizeof(*m));
+  PFN_cuTensorMapEncodeTiled_v12000 f = encode_tiled();
+  if (!f) return GDN_ERR_CUDA;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)nheads, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)nheads * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)PRO_HG, (cuuint32_t)PRO_ROWS};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GDN_OK : GDN_ERR_CUDA;
+}
+
 // Opt the large-shared-memory kernels in once per device.
 int configure_device() {
   static std::atomic<uint64_t> done_mask{0};
@@ -310,9 +343,12 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
         const int ngroups = 2 * ((d->h_qk + PRO_HG - 1) / PRO_HG) + (d->h_v + PRO_HG - 1) / PRO_HG;
         const int nitems = ngroups * 2 * L.max_chunks;
         const int grid = nitems < g_num_sms ? nitems : g_num_sms;
-        k_prologue_tc<<<grid, 512, PRO_SMEM, s>>>(kd, tab, nitems, static_cast<const uint16_t*>(q),
-                                                  static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
-                                                  conv_w, kq, F(L.vs));
+        CUtensorMap tm_q, tm_k, tm_v;
+        if (make_stream_map(&tm_q, q, d->total_tokens, d->h_qk) != GDN_OK ||
+            make_stream_map(&tm_k, k, d->total_tokens, d->h_qk) != GDN_OK ||
+            make_stream_map(&tm_v, v, d->total_tokens, d->h_v) != GDN_OK)
+          return GDN_ERR_CUDA;
+        k_prologue_tc<<<grid, 512, PRO_SMEM, s>>>(kd, tab, nitems, tm_q, tm_k, tm_v, conv_w, kq, F(L.vs));
       }
       ProfScope p("chunk_prep_tc", s);
       k_chunkprep_tc<<<dim3(d->h_qk, L.max_chunks), 256, PA_TC_SMEM, s>>>(kd, tab, a, b, A_log, dt_bias, kq, tp,

@@ -26,6 +26,8 @@
 // heads and 32-row slices of the state): the three MMA rounds above per chunk, with the
 // next chunk's tiles bulk-copied into a second stage while the current one computes.
 #pragma once
+#include <cuda.h>
+
 #include "gdn_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -171,8 +173,11 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 // half chunk) with a stride of the grid size.  A group is up to 8 heads of one stream -- q,
 // k or value heads -- whose slices of a token row are contiguous (2 KB).  The next item's
 // 32 + 3 token rows and conv taps are bulk-copied into the other of two shared-memory stages
-// while the current item is computed, so loads overlap compute; the 32 lanes of warp 0 issue
-// those copies together and leave the item's description in shared memory for the others.
+// while the current item is computed, so loads overlap compute: one 3-D tensor copy of the box
+// (128 channels x 8 heads x 35 tokens; heads past the stream's count and tokens outside the
+// tensor read as zeros, tokens of a neighbouring sequence are skipped by the conv) and one
+// bulk copy of the taps.  Warp 0 issues them and leaves the item's description in shared
+// memory for the others.
 // 16 warps: warp w works on head w % 8 of the group and on tokens 16 (w / 8) .. + 15 of the
 // half chunk.
 //   q / k head j: rows 64..127 / 0..63 of the [K;Q] hi/lo tile of QK head j
@@ -191,7 +196,7 @@ constexpr uint32_t PRO_ROWS_BYTES = PRO_ROWS * PRO_HG * D * 2;
 constexpr uint32_t PRO_W_BYTES = PRO_HG * D * 16;
 constexpr uint32_t PRO_STAGE = PRO_ROWS_BYTES + PRO_W_BYTES;
 constexpr size_t PRO_SMEM = 2 * (size_t)PRO_STAGE;
-static_assert(PRO_ROWS <= 64, "two token rows per lane of the issuing warp");
+static_assert(PRO_ROWS <= 256 && PRO_HG <= 256, "tensor-copy box limits");
 
 struct ProItem {
   ChunkEntry e;
@@ -219,9 +224,9 @@ __device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry& e, 
 }
 
 __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab, int nitems,
-                                                        const uint16_t* __restrict__ q,
-                                                        const uint16_t* __restrict__ k,
-                                                        const uint16_t* __restrict__ v,
+                                                        const __grid_constant__ CUtensorMap tm_q,
+                                                        const __grid_constant__ CUtensorMap tm_k,
+                                                        const __grid_constant__ CUtensorMap tm_v,
                                                         const float* __restrict__ conv_w,
                                                         uint8_t* __restrict__ kq_ws, float* __restrict__ vs_ws) {
   const int hq = d.h_qk, hv = d.h_v;
@@ -232,6 +237,10 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
   __shared__ uint64_t mbar[2];
   __shared__ ProItem s_item[2];
   __shared__ int s_abort;
+  if ((tc::smem_u32(sm) & 127u) != 0) {  // tensor copies need 128-byte aligned destinations
+    if (tid == 0) atomicExch(&g_gdn_status, -6);
+    return;
+  }
   if (tid == 0) {
     s_abort = 0;
     tc::mbar_init(tc::smem_u32(&mbar[0]), 1);
@@ -239,47 +248,26 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     tc::fence_mbar_init();
   }
   __syncthreads();
-  // (warp 0, all lanes) describe item `it` (chunk-table entry e) in s_item[st] and issue its
-  // copies into stage `st`: lane l copies token rows l and l + 32.  Unused chunk slots copy
-  // nothing.
+  // (warp 0, lane 0) describe item `it` (chunk-table entry e) in s_item[st] and issue its
+  // copies into stage `st`.  Unused chunk slots copy nothing.
   auto issue = [&](int it, const ChunkEntry& e, int st) -> bool {  // true if copies were issued
     const ProItem w = pro_item(d, e, it, ngroups);
-    if (lane == 0) s_item[st] = w;
+    s_item[st] = w;
     if (w.e.len == 0) return false;
-    const uint16_t* src = w.stream == 0 ? q : w.stream == 1 ? k : v;
-    const uint32_t row_bytes = (uint32_t)w.nh * D * 2;
-    bool ok[2];
-    uint32_t mine = 0;
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int r = lane + 32 * u, tcr = w.tb0 - 3 + r;
-      ok[u] = r < PRO_ROWS && tcr < w.e.len && (long)w.e.t0 + tcr >= w.e.seq_start;
-      mine += ok[u] ? row_bytes : 0u;
-    }
-    const uint32_t bytes = __reduce_add_sync(0xffffffffu, mine) + (uint32_t)w.nh * D * 16;
     const uint32_t bar = tc::smem_u32(&mbar[st]);
     const uint32_t base = tc::smem_u32(sm + (size_t)st * PRO_STAGE);
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(bar, bytes);
-      tc::bulk_g2s(base + PRO_ROWS_BYTES, conv_w + (size_t)w.ch0 * 4, (uint32_t)w.nh * D * 16, bar);
-    }
-    __syncwarp();
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int r = lane + 32 * u;
-      if (ok[u]) {
-        const long tg = (long)w.e.t0 + w.tb0 - 3 + r;
-        tc::bulk_g2s(base + r * row_bytes, src + ((size_t)tg * w.nheads + w.h0) * D, row_bytes, bar);
-      }
-    }
+    tc::mbar_arrive_expect_tx(bar, PRO_ROWS_BYTES + (uint32_t)w.nh * D * 16);
+    tc::bulk_g2s(base + PRO_ROWS_BYTES, conv_w + (size_t)w.ch0 * 4, (uint32_t)w.nh * D * 16, bar);
+    const CUtensorMap* tm = w.stream == 0 ? &tm_q : w.stream == 1 ? &tm_k : &tm_v;
+    tc::tma_load_3d(base, tm, 0, w.h0, w.e.t0 + w.tb0 - 3, bar);  // rows t - 3 .. of the half chunk
     return true;
   };
-  bool pending[2] = {false, false};  // (warp 0) copies in flight per stage
+  bool pending[2] = {false, false};  // (thread 0) copies in flight per stage
   // warp 0 reads the table entry of the item after the one it issues next, one item ahead, so
   // that the load's latency hides behind the current item's work
   const int g = gridDim.x;
   ChunkEntry e_next{};
-  if (warp == 0 && (int)blockIdx.x < nitems) {
+  if (tid == 0 && (int)blockIdx.x < nitems) {
     pending[0] = issue(blockIdx.x, tab[pro_chunk(blockIdx.x, ngroups)], 0);
     if ((int)blockIdx.x + g < nitems) e_next = tab[pro_chunk(blockIdx.x + g, ngroups)];
   }
@@ -289,7 +277,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
   for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
     const int st = n & 1;
     const ProItem w = s_item[st];
-    if (warp == 0 && it + g < nitems) {
+    if (tid == 0 && it + g < nitems) {
       pending[st ^ 1] = issue(it + g, e_next, st ^ 1);
       if (it + 2 * g < nitems) e_next = tab[pro_chunk(it + 2 * g, ngroups)];
     }
@@ -299,7 +287,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     }
     if (!tc::mbar_wait(tc::smem_u32(&mbar[st]), parity[st])) s_abort = 1;
     parity[st] ^= 1;
-    if (warp == 0) pending[st] = false;
+    if (tid == 0) pending[st] = false;
     __syncthreads();  // the abort decision is uniform
     if (s_abort) break;
     const uint8_t* base = sm + (size_t)st * PRO_STAGE;
@@ -334,7 +322,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
 #pragma unroll
             for (int tap = 0; tap < 4; ++tap) {
               if (!okt[tap]) continue;
-              const uint4 x = *reinterpret_cast<const uint4*>(hrow + (size_t)(blk + r + tap) * nh * D + cg);
+              const uint4 x = *reinterpret_cast<const uint4*>(hrow + (size_t)(blk + r + tap) * PRO_HG * D + cg);
               const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
               for (int c = 0; c < 8; ++c)
@@ -383,7 +371,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
 #pragma unroll
           for (int p = 0; p < 11; ++p) {
             const int rr = blk + p;
-            x[p] = row_ok(rr) ? *reinterpret_cast<const uint2*>(hrow + (size_t)rr * nh * D + c0) : make_uint2(0, 0);
+            x[p] = row_ok(rr) ? *reinterpret_cast<const uint2*>(hrow + (size_t)rr * PRO_HG * D + c0) : make_uint2(0, 0);
           }
           auto xv = [&](int p, int c) {
             const uint32_t wd = c < 2 ? x[p].x : x[p].y;
@@ -407,8 +395,8 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     tc::fence_proxy_async();
     __syncthreads();  // this stage is free for the item after next
   }
-  if (s_abort && warp == 0) {  // record, and let copies still in flight land (bounded) before leaving
-    if (lane == 0) atomicExch(&g_gdn_status, -7);
+  if (s_abort && tid == 0) {  // record, and let copies still in flight land (bounded) before leaving
+    atomicExch(&g_gdn_status, -7);
     for (int q2 = 0; q2 < 2; ++q2)
       if (pending[q2]) (void)tc::mbar_wait(tc::smem_u32(&mbar[q2]), parity[q2]);
   }

@@ -1,5 +1,5 @@
 // tc_ptx.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core path: mbarriers, bulk
-// (1-D TMA) copies, cluster (distributed shared memory) stores, tcgen05
+// (1-D TMA) and tensor copies, cluster (distributed shared memory) stores, tcgen05
 // allocation / MMA / commit / TMEM loads, and the shared-memory matrix descriptors.  No
 // cluster multicast is used anywhere.
 //
@@ -95,6 +95,17 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// 3-D tiled tensor copy global -> shared (no multicast), completion counted in bytes on
+// `bar`.  `tmap` is the address of a __grid_constant__ CUtensorMap kernel parameter; (x, y, z)
+// is the box origin in elements (x * element size must be a multiple of 16 bytes; the other
+// coordinates may be negative or past the end: those elements read as zeros).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
 }
 // shared -> global, tracked by the issuing thread's bulk groups.
