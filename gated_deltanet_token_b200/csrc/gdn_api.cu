@@ -330,11 +330,16 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
   int* seqc0 = reinterpret_cast<int*>(ws + L.seqc0);
   const Dims kd = kdims(d);
 
-  {
+  // One sequence without cu_seqlens: the tensor-core kernels compute the trivial tile map
+  // themselves (no table, no launch).
+  const bool need_map = !L.tc || cu_seqlens != nullptr;
+  if (need_map) {
     ProfScope p("tilemap", s);
     k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0);
   }
   if (L.tc) {
+    const ChunkEntry* tabc = need_map ? tab : nullptr;
+    const int* seqc0c = need_map ? seqc0 : nullptr;
     uint8_t* kq = reinterpret_cast<uint8_t*>(ws + L.kq);
     uint8_t* tp = reinterpret_cast<uint8_t*>(ws + L.tp);
     if (d->total_tokens > 0) {
@@ -348,10 +353,10 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
             make_stream_map(&tm_k, k, d->total_tokens, d->h_qk) != GDN_OK ||
             make_stream_map(&tm_v, v, d->total_tokens, d->h_v) != GDN_OK)
           return GDN_ERR_CUDA;
-        k_prologue_tc<<<grid, 512, PRO_SMEM, s>>>(kd, tab, nitems, tm_q, tm_k, tm_v, conv_w, kq, F(L.vs));
+        k_prologue_tc<<<grid, PRO_THREADS, PRO_SMEM, s>>>(kd, tabc, nitems, tm_q, tm_k, tm_v, conv_w, kq, F(L.vs));
       }
       ProfScope p("chunk_prep_tc", s);
-      k_chunkprep_tc<<<dim3(d->h_qk, L.max_chunks), 256, PA_TC_SMEM, s>>>(kd, tab, a, b, A_log, dt_bias, kq, tp,
+      k_chunkprep_tc<<<dim3(d->h_qk, L.max_chunks), 256, PA_TC_SMEM, s>>>(kd, tabc, a, b, A_log, dt_bias, kq, tp,
                                                                           F(L.gb));
     }
     // The output norm runs inside phase B (clusters of the four slices of a head) unless that
@@ -378,10 +383,10 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
       cfg.numAttrs = 1;
       const uint16_t* zb = static_cast<const uint16_t*>(z);
       cudaError_t e = kd.out_bf16
-          ? cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_BF16>, kd, (const int*)cu_seqlens, (const int*)seqc0,
+          ? cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_BF16>, kd, (const int*)cu_seqlens, seqc0c,
                                (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
                                init_state, F(L.yraw), final_state, zb, norm_w, y)
-          : cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_F32>, kd, (const int*)cu_seqlens, (const int*)seqc0,
+          : cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_F32>, kd, (const int*)cu_seqlens, seqc0c,
                                (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
                                init_state, F(L.yraw), final_state, zb, norm_w, y);
       if (e != cudaSuccess) return GDN_ERR_CUDA;
@@ -389,7 +394,7 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     }
     {
       ProfScope p("chunk_scan_tc", s);
-      k_chunkscan_tc<PB_Y_RAW><<<grid, 288, PB_TC_SMEM, s>>>(kd, cu_seqlens, seqc0, kq, tp, F(L.gb), F(L.vs),
+      k_chunkscan_tc<PB_Y_RAW><<<grid, 288, PB_TC_SMEM, s>>>(kd, cu_seqlens, seqc0c, kq, tp, F(L.gb), F(L.vs),
                                                              init_state, F(L.yraw), final_state, nullptr, nullptr,
                                                              nullptr);
     }

@@ -25,6 +25,18 @@ struct __align__(16) ChunkEntry {
   int seq_start;  // first packed token of the sequence (conv history stops there)
 };
 
+// Entry c of the tile map.  With no table (tab == nullptr: one sequence of `total` tokens)
+// the entry is computed: chunk c covers tokens 64 c .. 64 c + 63 of sequence 0.
+__device__ __forceinline__ ChunkEntry chunk_entry(const ChunkEntry* tab, int total, int c) {
+  if (tab) return tab[c];
+  ChunkEntry e;
+  e.seq = 0;
+  e.t0 = c * 64;
+  e.len = min(64, max(0, total - c * 64));
+  e.seq_start = 0;
+  return e;
+}
+
 __device__ __forceinline__ float bf2f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
 __device__ __forceinline__ uint16_t f2bf(float f) {

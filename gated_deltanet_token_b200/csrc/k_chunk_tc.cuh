@@ -192,6 +192,8 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 constexpr int PRO_HG = 8;                  // heads per work item
 constexpr int PRO_TOK = 32;                // tokens per work item (half a chunk)
 constexpr int PRO_ROWS = PRO_TOK + 3;      // with the conv history
+constexpr int PRO_TSPLIT = 2;              // warps per head of an item (token ranges of 16)
+constexpr int PRO_THREADS = PRO_HG * PRO_TSPLIT * 32;
 constexpr uint32_t PRO_ROWS_BYTES = PRO_ROWS * PRO_HG * D * 2;
 constexpr uint32_t PRO_W_BYTES = PRO_HG * D * 16;
 constexpr uint32_t PRO_STAGE = PRO_ROWS_BYTES + PRO_W_BYTES;
@@ -223,7 +225,7 @@ __device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry& e, 
   return w;
 }
 
-__global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab, int nitems,
+__global__ void __launch_bounds__(PRO_THREADS, 1) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab, int nitems,
                                                         const __grid_constant__ CUtensorMap tm_q,
                                                         const __grid_constant__ CUtensorMap tm_k,
                                                         const __grid_constant__ CUtensorMap tm_v,
@@ -268,8 +270,8 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
   const int g = gridDim.x;
   ChunkEntry e_next{};
   if (tid == 0 && (int)blockIdx.x < nitems) {
-    pending[0] = issue(blockIdx.x, tab[pro_chunk(blockIdx.x, ngroups)], 0);
-    if ((int)blockIdx.x + g < nitems) e_next = tab[pro_chunk(blockIdx.x + g, ngroups)];
+    pending[0] = issue(blockIdx.x, chunk_entry(tab, d.total_tokens, pro_chunk(blockIdx.x, ngroups)), 0);
+    if ((int)blockIdx.x + g < nitems) e_next = chunk_entry(tab, d.total_tokens, pro_chunk(blockIdx.x + g, ngroups));
   }
   __syncthreads();
   uint32_t parity[2] = {0, 0};
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
     const ProItem w = s_item[st];
     if (tid == 0 && it + g < nitems) {
       pending[st ^ 1] = issue(it + g, e_next, st ^ 1);
-      if (it + 2 * g < nitems) e_next = tab[pro_chunk(it + 2 * g, ngroups)];
+      if (it + 2 * g < nitems) e_next = chunk_entry(tab, d.total_tokens, pro_chunk(it + 2 * g, ngroups));
     }
     if (w.e.len == 0) {
       __syncthreads();
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
         uint8_t* tile = kq_ws + ((size_t)w.chunk * hq + head) * KQ_BYTES;
         const float scale = w.stream == 0 ? d.q_scale : 1.0f;
 #pragma unroll 1
-        for (int blk = tsplit * (PRO_TOK / 2); blk < (tsplit + 1) * (PRO_TOK / 2); blk += 4) {
+        for (int blk = tsplit * (PRO_TOK / PRO_TSPLIT); blk < (tsplit + 1) * (PRO_TOK / PRO_TSPLIT); blk += 4) {
           const int t = tb0 + blk + r;  // chunk-relative token
           float acc[2][8];
           bool okt[4];
@@ -314,19 +316,21 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
 #pragma unroll
           for (int gi = 0; gi < 2; ++gi) {
             const int cg = (g0 + 8 * gi) * 8;
-            float4 w4[8];  // the group's 8 channels x 4 taps
-#pragma unroll
-            for (int c = 0; c < 8; ++c) w4[c] = wsm[cg + c];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[gi][c] = 0.0f;
+            uint32_t xw[4][4];  // the four tap rows' 8 channels (bf16 pairs); zero outside the sequence
 #pragma unroll
             for (int tap = 0; tap < 4; ++tap) {
-              if (!okt[tap]) continue;
-              const uint4 x = *reinterpret_cast<const uint4*>(hrow + (size_t)(blk + r + tap) * PRO_HG * D + cg);
-              const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+              const uint4 x = okt[tap] ? *reinterpret_cast<const uint4*>(hrow + (size_t)(blk + r + tap) * PRO_HG * D + cg)
+                                       : make_uint4(0, 0, 0, 0);
+              xw[tap][0] = x.x; xw[tap][1] = x.y; xw[tap][2] = x.z; xw[tap][3] = x.w;
+            }
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                acc[gi][c] = fmaf(comp(w4[c], tap), bf2f(c & 1 ? wd[c >> 1] >> 16 : wd[c >> 1] & 0xffffu), acc[gi][c]);
+            for (int c = 0; c < 8; ++c) {
+              const float4 w4 = wsm[cg + c];  // channel cg + c, taps 0..3
+              float a_ = 0.0f;
+#pragma unroll
+              for (int tap = 0; tap < 4; ++tap)
+                a_ = fmaf(comp(w4, tap), bf2f(c & 1 ? xw[tap][c >> 1] >> 16 : xw[tap][c >> 1] & 0xffffu), a_);
+              acc[gi][c] = a_;
             }
           }
           float ss0 = 0.0f, ss1 = 0.0f;
@@ -366,7 +370,7 @@ __global__ void __launch_bounds__(512, 1) k_prologue_tc(Dims d, const ChunkEntry
         float* out = vs_ws + ((size_t)w.chunk * hv + head) * (VS_BYTES / 4) + (size_t)(c0 / TC_NV) * (VS_SLICE / 4) +
                      (c0 % TC_NV);
 #pragma unroll 1
-        for (int blk = tsplit * (PRO_TOK / 2); blk < (tsplit + 1) * (PRO_TOK / 2); blk += 8) {
+        for (int blk = tsplit * (PRO_TOK / PRO_TSPLIT); blk < (tsplit + 1) * (PRO_TOK / PRO_TSPLIT); blk += 8) {
           uint2 x[11];  // raw bf16 of 4 channels, rows t - 3 .. t + 7
 #pragma unroll
           for (int p = 0; p < 11; ++p) {
@@ -431,7 +435,7 @@ __global__ void __launch_bounds__(256, 2)
                    const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
                    uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
   const int chunk = blockIdx.y;  // head-fastest grid: concurrent CTAs read adjacent tiles
-  const ChunkEntry e = tab[chunk];
+  const ChunkEntry e = chunk_entry(tab, d.total_tokens, chunk);
   if (e.len == 0) return;
   const int j = blockIdx.x, hq = d.h_qk, hv = d.h_v, G = hv / hq, L = e.len;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -766,7 +770,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   const int row = quarter * 32 + lane;  // TMEM lane: accumulator row
   const int ts = cu ? cu[n] : 0, te = cu ? cu[n + 1] : d.total_tokens;
   const int nchunks = te > ts ? (te - ts + CH - 1) / CH : 0;
-  const int gc0 = seq_chunk0[n];
+  const int gc0 = seq_chunk0 ? seq_chunk0[n] : 0;
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* s_hi = sm;
   uint8_t* s_lo = sm + PB_S_TILE;
