@@ -746,10 +746,12 @@ enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 // components ("Qwen3.8-Flash-Next" technical report, Fig. 2: RMS norm of each head's output,
 // gated by SiLU(z)) needs the sums of squares of all four slices: each norm thread stores its
 // token's sum into the three other CTAs of the cluster as one 32-bit word whose two low bits
-// carry a chunk tag (the value is the flag: no fence or barrier between CTAs).  Its y row
-// waits in registers and is normalised in the next chunk, while that chunk's second MMA
-// round runs.  Every slice sums the
-// same four tag-stripped words in rank order, so all four use the same norm.  Warp 9 idles.
+// carry a chunk tag (the value is the flag: no fence or barrier between CTAs), then waits for
+// the peers' words and normalises its y row.  The norm warps stay out of the workers' chunk
+// barriers: they arrive on an mbarrier once they are done with a chunk's TMEM rows and stage,
+// and thread 0 waits for that before the next chunk's first MMA round, so the exchange never
+// holds up the state chain.  Every slice sums the same four tag-stripped words in rank order,
+// so all four use the same norm.  Warp 9 idles.
 template <int YM>
 __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     k_chunkscan_tc(Dims d, const int* __restrict__ cu, const int* __restrict__ seq_chunk0,
@@ -779,6 +781,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   __shared__ uint64_t mbar_mma[3];  // one per MMA round: each completes once per chunk
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
+  __shared__ uint64_t norm_done;  // fused norm: the norm warps are done with a chunk (64 arrivals)
   // fused norm: tagged sums of squares from the three other slices, [chunk parity][peer][token]
   __shared__ uint32_t red[FUSED ? 2 * 3 * 64 : 1];
   const int rank = FUSED ? (int)tc::cluster_ctarank() : 0;
@@ -800,6 +803,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     tc::mbar_init(tc::smem_u32(&mbar_ld[0]), 1);
     tc::mbar_init(tc::smem_u32(&mbar_ld[1]), 1);
     for (int q3 = 0; q3 < 3; ++q3) tc::mbar_init(tc::smem_u32(&mbar_mma[q3]), 1);
+    if (FUSED) tc::mbar_init(tc::smem_u32(&norm_done), 64);
     tc::fence_mbar_init();
   }
   if (warp == 0) {
@@ -809,6 +813,11 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   // barrier over the four warps that own TMEM lanes 0..63 (warps 0, 1, 4, 5)
   auto named_bar_sync = [](int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+  };
+  // the chunk barrier: every warp but the norm warps
+  auto loop_sync = [&]() {
+    if (FUSED) named_bar_sync(2, 320);
+    else __syncthreads();
   };
   // (producer warp, lane 0) copies of chunk c into stage st
   auto issue_load = [&](int c, int st) {
@@ -915,14 +924,73 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     }
     return true;
   };
-  for (int c = 0; c < nchunks && !aborted; ++c) {
+  // ---- fused norm: the y rows, one chunk behind nothing but the two MMA rounds they read ----
+  if (normw) {
+    const int t = row & 63;
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c & 1;
+      const int t0 = ts + c * CH, L = min(CH, te - t0);
+      const float* gsm = reinterpret_cast<const float*>(stage[st] + PBStage::GB);
+      bool ok = tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st]);
+      ph_ld[st] ^= 1;
+      const float eg = (ok && t < L) ? __expf(gsm[t]) : 0.0f;
+      float qs[NV];  // e^{gamma_t} (Q S^T)[t][:], all 32 columns of the slice, 16 at a time
+      ok = ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma);
+      tc::tc_fence_after();
+      if (ok) {
+#pragma unroll
+        for (int h16 = 0; h16 < 2; ++h16) {
+          uint32_t r[16], r2[16];
+          tc::tmem_ld16(t_norm + 16 * h16, r);
+          tc::tmem_ld16(t_norm + NV + 16 * h16, r2);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) qs[16 * h16 + i] = eg * (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
+        }
+      }
+      ok = ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma);
+      ph_mma ^= 1;
+      tc::tc_fence_after();
+      if (ok) {  // Y = e^gamma Q S^T + (M o QK^T) U, and this slice's sum of squares to the peers
+        float p = 0.0f;
+#pragma unroll
+        for (int h16 = 0; h16 < 2; ++h16) {
+          uint32_t r[16], r2[16];
+          tc::tmem_ld16(t_norm + 2 * NV + 16 * h16, r);
+          tc::tmem_ld16(t_norm + 3 * NV + 16 * h16, r2);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k = 16 * h16 + i;
+            yv[k] = t < L ? qs[k] + (__uint_as_float(r[i]) + __uint_as_float(r2[i])) : 0.0f;
+            p = fmaf(yv[k], yv[k], p);
+          }
+        }
+        y_tok = t < L ? t0 + t : -1;
+        const int buf = c & 1;
+        const uint32_t word = (__float_as_uint(p) & ~3u) | ((uint32_t)(c >> 1) & 3u);
+        own = untag(word);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          if (rr == rank) continue;
+          const int slot = rank < rr ? rank : rank - 1;  // this slice's slot in peer rr
+          tc::st_cluster_u32(tc::mapa(tc::smem_u32(&red[(buf * 3 + slot) * 64 + t]), (uint32_t)rr), word);
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(tc::smem_u32(&norm_done));  // this chunk's TMEM rows and stage are read
+      if (!ok || !finish(c)) { s_abort = 1; atomicExch(&g_gdn_status, -7); break; }
+      if (s_abort) break;
+    }
+  }
+  for (int c = 0; c < nchunks && !aborted && !normw; ++c) {
     const int st = c & 1;
     const int t0 = ts + c * CH, L = min(CH, te - t0);
     uint8_t* sg = stage[st];
     uint8_t* r_hi = sg + PBStage::VS;
     uint8_t* r_lo = r_hi + PB_R_TILE;
     const uint32_t kq0 = tc::smem_u32(sg + PBStage::KQ), tp0 = tc::smem_u32(sg + PBStage::TP);
-    if ((worker || normw) && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    if (worker && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     ph_ld[st] ^= 1;
     const float* gsm = reinterpret_cast<const float*>(sg + PBStage::GB);
     const float gL = gsm[L - 1];
@@ -937,7 +1005,13 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       }
     }
     const float eg = t < L ? __expf(gsm[t]) : 0.0f;
-    __syncthreads();
+    // the norm warps are done with the previous chunk's TMEM rows and stage before this
+    // chunk's first round overwrites the one and the producer reloads the other
+    if (FUSED && tid == 0 && c > 0 && !tc::mbar_wait(tc::smem_u32(&norm_done), (uint32_t)(c - 1) & 1u)) {
+      s_abort = 1;
+      atomicExch(&g_gdn_status, -7);
+    }
+    loop_sync();
     if (s_abort) { aborted = true; break; }
     // ---- round 1: [K S^T ; Q S^T] = [K;Q] (128 x 128) x S^T (K = 128, N = nv) -------------
     if (tid == 0) {
@@ -954,7 +1028,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     if (producer && lane == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);  // stage last read by chunk c-1
     if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
     tc::tc_fence_after();
-    float qs[FUSED ? NV : NH];  // y rows: e^{gamma_t} (Q S^T)[t][:] (workers: 16 columns, norm warps: 32)
+    float qs[NH];  // y rows (separate-epilogue mode): e^{gamma_t} (Q S^T)[t][:]
     if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
       tc::tmem_ld16(t_a, r);
@@ -979,17 +1053,6 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
 #pragma unroll
         for (int i = 0; i < NH; ++i) qs[i] = eg * __uint_as_float(r[i]);
       }
-    } else if (normw) {  // all 32 columns of the token's y row, 16 at a time
-#pragma unroll
-      for (int h16 = 0; h16 < 2; ++h16) {
-        uint32_t r[16], r2[16];
-        tc::tmem_ld16(t_norm + 16 * h16, r);
-        tc::tmem_ld16(t_norm + NV + 16 * h16, r2);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) qs[16 * h16 + i] = eg * (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
-      }
-      if (c > 0 && !finish(c - 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }  // while round 2 runs
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
@@ -1038,33 +1101,6 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
                                qs[q4 * 4 + 2] + __uint_as_float(r[q4 * 4 + 2]),
                                qs[q4 * 4 + 3] + __uint_as_float(r[q4 * 4 + 3]));
       }
-    } else if (normw) {  // the same y, kept until the four slices' sums of squares are in
-      float p = 0.0f;
-#pragma unroll
-      for (int h16 = 0; h16 < 2; ++h16) {
-        uint32_t r[16], r2[16];
-        tc::tmem_ld16(t_norm + 2 * NV + 16 * h16, r);
-        tc::tmem_ld16(t_norm + 3 * NV + 16 * h16, r2);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k = 16 * h16 + i;
-          yv[k] = t < L ? qs[k] + (__uint_as_float(r[i]) + __uint_as_float(r2[i])) : 0.0f;
-          p = fmaf(yv[k], yv[k], p);
-        }
-      }
-      y_tok = t < L ? t0 + t : -1;
-      const int buf = c & 1;
-      const uint32_t word = (__float_as_uint(p) & ~3u) | ((uint32_t)(c >> 1) & 3u);
-      own = untag(word);
-#pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        if (rr == rank) continue;
-        const int slot = rank < rr ? rank : rank - 1;  // this slice's slot in peer rr
-        tc::st_cluster_u32(tc::mapa(tc::smem_u32(&red[(buf * 3 + slot) * 64 + t]), (uint32_t)rr), word);
-      }
-      if (t < L)  // z of this row, read by the norm at the next chunk's start
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(z + ((size_t)(t0 + t) * hv + h) * D + i0));
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
@@ -1097,10 +1133,9 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     }
     tc::fence_proxy_async();
     tc::tc_fence_before();
-    __syncthreads();
+    loop_sync();
     if (s_abort) { aborted = true; break; }
   }
-  if (!aborted && normw && nchunks > 0 && !finish(nchunks - 1)) atomicExch(&g_gdn_status, -7);
   if (!aborted && worker) {
 #pragma unroll
     for (int i = 0; i < NH; ++i) final_state[sbase + (size_t)(cb + i) * D + row] = S[i];
