@@ -13,6 +13,7 @@ sides, timed with CUDA events on the launching stream.  Inputs rotate over three
 copies (3 x 97 MiB > 126 MB L2) so no step starts with its inputs in L2.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py --configs      # one JSON line per workload: GPU time and the oracle beside it
 Multi-GPU: launched with torch.distributed.run, one rank per GPU; every rank runs its own
 full workload (weak scaling, no data-path collective: the mixer shards by sequence/head).
 """
@@ -54,6 +55,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     p.add_argument("--decode-steps", type=int, default=None)
+    p.add_argument("--configs", action="store_true",
+                   help="time every workload (GPU and the oracle on a bounded sample) instead of the bench step")
     return p.parse_args(argv)
 
 
@@ -466,10 +469,117 @@ def gpu_arm(args):
     return 0
 
 
+def configs_table(args):
+    """`--configs`: for each workload, the GPU time of one call (median over repeats, inputs
+    resident) and the oracle's tokens/s on the host cores for a bounded token sample."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from gated_deltanet_token_b200 import gdn
+    from gated_deltanet_token_b200.inputs import WORKLOADS, make_inputs
+
+    oracle.build()
+    cores = cpu_cores()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+
+    def dev_t(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if a.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        return t.to(dev)
+
+    def gpu_time(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    def oracle_rate(inp, kind, sample_tokens):
+        sub = dict(inp)
+        if kind == "prefill":
+            cu = inp.get("cu_seqlens")
+            if cu is not None:  # the first sequences, up to the sample size
+                keep = int(np.searchsorted(cu, sample_tokens, side="right"))
+                keep = max(1, min(keep, len(cu) - 1))
+                sub["cu_seqlens"] = cu[:keep + 1]
+                T = int(cu[keep])
+            else:
+                T = min(sample_tokens, inp["q"].shape[0])
+            for n in ("q", "k", "v", "z", "a", "b"):
+                sub[n] = inp[n][:T]
+            if sub.get("init_state") is not None and cu is not None:
+                sub["init_state"] = inp["init_state"][:len(sub["cu_seqlens"]) - 1]
+            t0 = time.perf_counter()
+            oracle.prefill(sub, n_threads=cores, want_state=True)
+            return T / (time.perf_counter() - t0), f"first {T} tokens"
+        t0 = time.perf_counter()
+        oracle.decode(sub, n_threads=cores)
+        N = inp["q"].shape[0]
+        return N / (time.perf_counter() - t0), f"all {N} sequences, one step"
+
+    for name in WORKLOADS:
+        inp = make_inputs(name)
+        spec = inp["spec"]
+        hq, hv = spec["h_qk"], spec["h_v"]
+        d = {n: dev_t(inp.get(n)) for n in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w",
+                                            "norm_w", "init_state", "state", "conv_state")}
+        if spec["kind"] == "prefill":
+            T = spec["T"]
+            cu = inp.get("cu_seqlens")
+            cu_t = None if cu is None else torch.from_numpy(cu.astype(np.int32)).to(dev)
+            odt = torch.float32 if spec["dtype"] == "f32" else torch.bfloat16
+            dims = gdn.make_dims(spec["n_seqs"], T, hq, hv, gdn.GDN_DTYPE_F32 if spec["dtype"] == "f32"
+                                 else gdn.GDN_DTYPE_BF16, gdn.GDN_DTYPE_F32 if odt == torch.float32
+                                 else gdn.GDN_DTYPE_BF16)
+            ws = torch.empty(gdn.gdn_prefill_workspace_size(dims), dtype=torch.uint8, device=dev)
+            y = torch.empty((T, hv, 128), dtype=odt, device=dev)
+            fs = torch.empty((spec["n_seqs"], hv, 128, 128), dtype=torch.float32, device=dev)
+
+            def call():
+                gdn.gdn_prefill(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                                d["conv_w"], d["norm_w"], d["init_state"], cu_t, out_dtype=odt, y=y,
+                                final_state=fs, workspace=ws)
+            ms = gpu_time(call, 5 if T > 100000 else 20)
+            units = T
+            rate, sample = oracle_rate(inp, "prefill", 1024 if hv >= 32 else T)
+            del ws, y, fs
+        else:
+            N = spec["n_seqs"]
+            yd = torch.empty((N, hv, 128), dtype=torch.bfloat16, device=dev)
+
+            def call():
+                gdn.gdn_decode(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                               d["conv_w"], d["norm_w"], d["conv_state"], d["state"], out_dtype=torch.bfloat16,
+                               y=yd)
+            ms = gpu_time(call, 20)
+            units = N
+            rate, sample = oracle_rate(inp, "decode", N)
+        print(json.dumps({"workload": name, "kind": spec["kind"], "tokens": units, "gpu_ms": ms,
+                          "gpu_tok_s": units / (ms / 1e3), "oracle_tok_s": rate, "oracle_threads": cores,
+                          "oracle_sample": sample, "speedup": units / (ms / 1e3) / rate}), flush=True)
+        del d
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return reference_arm(args)
+    if args.configs:
+        return configs_table(args)
     return gpu_arm(args)
 
 

@@ -737,7 +737,9 @@ enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 // lane quarter w % 4 and columns 16 (w / 4) .. 16 (w / 4) + 15 of the slice; warp 8 issues the
 // bulk copies of the next chunk.  Each product a b is taken as a_hi [b_hi | b_lo] (one MMA of
 // width 2 nv: the lo tile follows the hi tile at the operand's N stride) plus a_lo b_hi; the
-// epilogue adds the two column halves.
+// epilogue adds the two column halves.  (These small-N MMAs are bound by reading the A tile
+// from shared memory, so two MMAs per k-step beat three of width nv.)  One barrier per chunk,
+// at its start, orders the S tile, the stage reuse and the abort decision.
 
 //
 // Fused output norm (YM != PB_Y_RAW; clusters of the four slices of a value head; 12 warps):
@@ -1131,10 +1133,8 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       for (int i = 0; i < NH; ++i) S[i] = fmaf(eL, S[i], __uint_as_float(r[i]) + __uint_as_float(r2[i]));
       write_s_tile();
     }
-    tc::fence_proxy_async();
+    tc::fence_proxy_async();  // the next chunk's start barrier publishes the S tile
     tc::tc_fence_before();
-    loop_sync();
-    if (s_abort) { aborted = true; break; }
   }
   if (!aborted && worker) {
 #pragma unroll
