@@ -58,7 +58,8 @@ __device__ __forceinline__ uint32_t mnmaj(int k, int nb, int K) {
 // point gdn_selftest_tc).  case 0: A K-major 128x128, B = first 64 rows of A (K-major);
 // case 1: A K-major 128x128, B MN-major K=128 N=32; case 2: A K-major 128x64, B MN-major
 // K=64 N=32; case 3: A = transpose of rows 0..63 of a K-major 128-row tile (MN-major
-// view), B MN-major K=64 N=32.  out[0] = max |D - ref|, out[1] = max |ref|.
+// view), B MN-major K=64 N=32; case 4: as case 1 with A copied into TMEM first (tcgen05.cp)
+// and read from there by the MMA.  out[0] = max |D - ref|, out[1] = max |ref|.
 // ======================================================================================
 __device__ __forceinline__ float st_val(uint32_t i, uint32_t salt) {
   uint32_t x = i * 2654435761u ^ (salt * 0x9E3779B9u + 0x85EBCA6Bu);
@@ -70,7 +71,7 @@ __device__ __forceinline__ float st_val(uint32_t i, uint32_t salt) {
 template <int CASE>
 __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   constexpr int N = CASE == 0 ? 64 : 32;
-  constexpr int K = (CASE == 0 || CASE == 1) ? 128 : 64;
+  constexpr int K = (CASE == 0 || CASE == 1 || CASE == 4) ? 128 : 64;
   constexpr int ROWS_A = 128;  // rows of the physical A tile (case 3: the 128-row tile)
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* Ahi = sm;
@@ -82,8 +83,8 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int a_cols = CASE == 3 ? 128 : K;  // K-major physical columns of the A tile
   // logical A[m][k] and B[k][n]
-  auto Aval = [&](int m, int k) { return CASE == 3 ? st_val(k * 128 + m, 11u) : st_val(m * 1024 + k, 1u + CASE); };
-  auto Bval = [&](int k, int n) { return CASE == 0 ? Aval(n, k) : st_val(k * 64 + n, 7u + CASE); };
+  auto Aval = [&](int m, int k) { return CASE == 3 ? st_val(k * 128 + m, 11u) : st_val(m * 1024 + k, 1u + CASE % 4); };
+  auto Bval = [&](int k, int n) { return CASE == 0 ? Aval(n, k) : st_val(k * 64 + n, 7u + CASE % 4); };
   // physical A tile (K-major, 128 rows): case 3 stores X[s][j] = A[j][s] at (r = s, k = j)
   for (int idx = tid; idx < ROWS_A * a_cols; idx += 128) {
     const int r = idx / a_cols, c = idx % a_cols;
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
     tc::fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(&tslot), 64);
+    tc::tmem_alloc(tc::smem_u32(&tslot), CASE == 4 ? 256 : 64);
     tc::tmem_relinquish();
   }
   tc::fence_proxy_async();
@@ -116,7 +117,30 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
-  if (tid == 0) {
+  bool ok = true;
+  if (CASE == 4) {  // A hi -> TMEM columns 64.., A lo -> 128.., then read by the MMA from there
+    if (tid == 0) {
+      for (int ks = 0; ks < K / 16; ++ks) {
+        tc::tmem_cp_128x256b(tbase + 64 + ks * 8, tc::sdesc(tc::smem_u32(Ahi) + ks * 2 * LBO128, LBO128, 128));
+        tc::tmem_cp_128x256b(tbase + 128 + ks * 8, tc::sdesc(tc::smem_u32(Alo) + ks * 2 * LBO128, LBO128, 128));
+      }
+      tc::umma_commit(tc::smem_u32(&mbar));
+    }
+    ok = tc::mbar_wait(tc::smem_u32(&mbar), 0);
+    tc::tc_fence_after();
+  }
+  if (tid == 0 && CASE == 4 && ok) {
+    constexpr uint32_t idesc = tc::idesc_bf16(128, N, 0, 1);
+    const uint32_t b0[2] = {tc::smem_u32(Bhi), tc::smem_u32(Blo)};
+    for (int ks = 0; ks < K / 16; ++ks)
+      for (int term = 0; term < 3; ++term) {
+        const uint32_t at = tbase + (term == 2 ? 128 : 64) + ks * 8;
+        const uint64_t bd = tc::sdesc(b0[term == 1] + ks * 2 * 128, 128, (K / 8) * 128);
+        tc::umma_bf16_ts(tbase, at, bd, idesc, (ks | term) != 0);
+      }
+    tc::umma_commit(tc::smem_u32(&mbar));
+  }
+  if (tid == 0 && CASE != 4) {
     constexpr uint32_t idesc = tc::idesc_bf16(128, N, CASE == 3 ? 1 : 0, CASE == 0 ? 0 : 1);
     const uint32_t a0[2] = {tc::smem_u32(Ahi), tc::smem_u32(Alo)};
     const uint32_t b0[2] = {CASE == 0 ? tc::smem_u32(Ahi) : tc::smem_u32(Bhi),
@@ -134,7 +158,7 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
     }
     tc::umma_commit(tc::smem_u32(&mbar));
   }
-  const bool ok = tc::mbar_wait(tc::smem_u32(&mbar), 0);
+  ok = ok && tc::mbar_wait(tc::smem_u32(&mbar), CASE == 4 ? 1 : 0);
   tc::tc_fence_after();
   const int m = warp * 32 + lane;
   float err = 0.0f, mag = 0.0f;
@@ -165,7 +189,7 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   atomicMax(reinterpret_cast<int*>(out + 1), __float_as_int(mag));
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tbase, 64);
+  if (warp == 0) tc::tmem_dealloc(tbase, CASE == 4 ? 256 : 64);
 }
 
 // ======================================================================================
