@@ -498,7 +498,7 @@ int gdn_profile_read(gdn_kernel_time_t* out, int max_entries) {
 
 int gdn_selftest_tc(int case_id, float* out2) {
   if (!out2) return GDN_ERR_NULL;
-  if (case_id < 0 || case_id > 4) return GDN_ERR_SHAPE;
+  if (case_id < 0 || case_id > 5) return GDN_ERR_SHAPE;
   float zero[2] = {0.0f, 0.0f};
   if (cudaMemcpyToSymbol(g_selftest_out, zero, sizeof zero) != cudaSuccess) return GDN_ERR_CUDA;
   float* dptr = nullptr;
@@ -522,9 +522,13 @@ int gdn_selftest_tc(int case_id, float* out2) {
       e = cudaFuncSetAttribute(k_selftest_umma<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e == cudaSuccess) k_selftest_umma<3><<<1, 128, smem>>>(dptr);
       break;
-    default:
+    case 4:
       e = cudaFuncSetAttribute(k_selftest_umma<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e == cudaSuccess) k_selftest_umma<4><<<1, 128, smem>>>(dptr);
+      break;
+    default:
+      e = cudaFuncSetAttribute(k_selftest_umma<5>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_selftest_umma<5><<<1, 128, smem>>>(dptr);
   }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
     return GDN_ERR_CUDA;

@@ -59,7 +59,9 @@ __device__ __forceinline__ uint32_t mnmaj(int k, int nb, int K) {
 // case 1: A K-major 128x128, B MN-major K=128 N=32; case 2: A K-major 128x64, B MN-major
 // K=64 N=32; case 3: A = transpose of rows 0..63 of a K-major 128-row tile (MN-major
 // view), B MN-major K=64 N=32; case 4: as case 1 with A copied into TMEM first (tcgen05.cp)
-// and read from there by the MMA.  out[0] = max |D - ref|, out[1] = max |ref|.
+// and read from there by the MMA; case 5: M = 64 from rows 64..127 of the 128-row A tile, B
+// MN-major K=128 N=32, the result read from TMEM lanes 0..15 of each 32-lane quarter.
+// out[0] = max |D - ref|, out[1] = max |ref|.
 // ======================================================================================
 __device__ __forceinline__ float st_val(uint32_t i, uint32_t salt) {
   uint32_t x = i * 2654435761u ^ (salt * 0x9E3779B9u + 0x85EBCA6Bu);
@@ -71,7 +73,8 @@ __device__ __forceinline__ float st_val(uint32_t i, uint32_t salt) {
 template <int CASE>
 __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   constexpr int N = CASE == 0 ? 64 : 32;
-  constexpr int K = (CASE == 0 || CASE == 1 || CASE == 4) ? 128 : 64;
+  constexpr int K = (CASE == 0 || CASE == 1 || CASE == 4 || CASE == 5) ? 128 : 64;
+  constexpr int M = CASE == 5 ? 64 : 128;
   constexpr int ROWS_A = 128;  // rows of the physical A tile (case 3: the 128-row tile)
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* Ahi = sm;
@@ -83,12 +86,15 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int a_cols = CASE == 3 ? 128 : K;  // K-major physical columns of the A tile
   // logical A[m][k] and B[k][n]
-  auto Aval = [&](int m, int k) { return CASE == 3 ? st_val(k * 128 + m, 11u) : st_val(m * 1024 + k, 1u + CASE % 4); };
+  // case 5: logical row m of A is physical row 64 + m
+  auto Aval = [&](int m, int k) {
+    return CASE == 3 ? st_val(k * 128 + m, 11u) : st_val((m + (CASE == 5 ? 64 : 0)) * 1024 + k, 1u + CASE % 4);
+  };
   auto Bval = [&](int k, int n) { return CASE == 0 ? Aval(n, k) : st_val(k * 64 + n, 7u + CASE % 4); };
   // physical A tile (K-major, 128 rows): case 3 stores X[s][j] = A[j][s] at (r = s, k = j)
   for (int idx = tid; idx < ROWS_A * a_cols; idx += 128) {
     const int r = idx / a_cols, c = idx % a_cols;
-    float v = CASE == 3 ? (r < 64 ? Aval(c, r) : 0.0f) : Aval(r, c);
+    float v = CASE == 3 ? (r < 64 ? Aval(c, r) : 0.0f) : CASE == 5 ? st_val(r * 1024 + c, 2u) : Aval(r, c);
     uint16_t h, l;
     tc::split2(v, h, l);
     *reinterpret_cast<uint16_t*>(Ahi + kmaj128(r, c)) = h;
@@ -141,7 +147,7 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
     tc::umma_commit(tc::smem_u32(&mbar));
   }
   if (tid == 0 && CASE != 4) {
-    constexpr uint32_t idesc = tc::idesc_bf16(128, N, CASE == 3 ? 1 : 0, CASE == 0 ? 0 : 1);
+    constexpr uint32_t idesc = tc::idesc_bf16(M, N, CASE == 3 ? 1 : 0, CASE == 0 ? 0 : 1);
     const uint32_t a0[2] = {tc::smem_u32(Ahi), tc::smem_u32(Alo)};
     const uint32_t b0[2] = {CASE == 0 ? tc::smem_u32(Ahi) : tc::smem_u32(Bhi),
                             CASE == 0 ? tc::smem_u32(Alo) : tc::smem_u32(Blo)};
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
     for (int ks = 0; ks < K / 16; ++ks) {
       for (int term = 0; term < 3; ++term) {
         const int ai = term == 2 ? 1 : 0, bi = term == 1 ? 1 : 0;
-        const uint64_t ad = tc::sdesc(a0[ai] + ks * 2 * a_lbo, a_lbo, a_sbo);
+        const uint64_t ad = tc::sdesc(a0[ai] + ks * 2 * a_lbo + (CASE == 5 ? 8 * 128 : 0), a_lbo, a_sbo);
         const uint64_t bd = tc::sdesc(b0[bi] + ks * 2 * b_lbo, b_lbo, b_sbo);
         tc::umma_bf16(tbase, ad, bd, idesc, (ks | term) != 0);
       }
@@ -160,14 +166,15 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
   }
   ok = ok && tc::mbar_wait(tc::smem_u32(&mbar), CASE == 4 ? 1 : 0);
   tc::tc_fence_after();
-  const int m = warp * 32 + lane;
+  const int m = CASE == 5 ? warp * 16 + (lane & 15) : warp * 32 + lane;  // row held by this lane
+  const bool holds = CASE != 5 || lane < 16;  // M = 64: lanes 16..31 of a quarter hold no row
   float err = 0.0f, mag = 0.0f;
   if (ok) {
     for (int n0 = 0; n0 < N; n0 += 32) {
       uint32_t r[32];
-      tc::tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + n0, r);
+      tc::tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + n0, r);  // the whole warp loads
       tc::tmem_wait_ld();
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < 32 && holds; ++c) {
         const int n = n0 + c;
         float ref = 0.0f;
         for (int kk = 0; kk < K; ++kk) {
@@ -705,7 +712,8 @@ __global__ void __launch_bounds__(256, 2)
                         db[term == 1] + (uint64_t)((ks * 256) >> 4), idesc, (ks | term) != 0);
       tc::umma_commit(tc::smem_u32(&mbar));
     }
-    const bool ok = tc::mbar_wait(tc::smem_u32(&mbar), mma_phase);
+    // warp-uniform, so that the warp-collective TMEM loads below run on every lane or none
+    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&mbar), mma_phase));
     mma_phase ^= 1;
     if (!ok) atomicExch(&g_gdn_status, -7);
     tc::tc_fence_after();
@@ -957,11 +965,12 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       const int st = c & 1;
       const int t0 = ts + c * CH, L = min(CH, te - t0);
       const float* gsm = reinterpret_cast<const float*>(stage[st] + PBStage::GB);
-      bool ok = tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st]);
+      // warp-uniform, so that the warp-collective TMEM loads run on every lane or none
+      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st]));
       ph_ld[st] ^= 1;
       const float eg = (ok && t < L) ? __expf(gsm[t]) : 0.0f;
       float qs[NV];  // e^{gamma_t} (Q S^T)[t][:], all 32 columns of the slice, 16 at a time
-      ok = ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma);
+      ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma));
       tc::tc_fence_after();
       if (ok) {
 #pragma unroll
@@ -974,7 +983,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
           for (int i = 0; i < 16; ++i) qs[16 * h16 + i] = eg * (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
         }
       }
-      ok = ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma);
+      ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma));
       ph_mma ^= 1;
       tc::tc_fence_after();
       if (ok) {  // Y = e^gamma Q S^T + (M o QK^T) U, and this slice's sum of squares to the peers

@@ -188,7 +188,8 @@ int gdn_prefill_noalloc(const gdn_dims_t* d, const void* q, const void* k, const
  * Diagnostic: runs one tcgen05 operand-layout case of the bf16 tensor-core path on fixed
  * synthetic tiles (case 0: K-major A and B, 128x64x128; 1: K-major A, MN-major B, 128x32x128;
  * 2: K-major A, MN-major B, 128x32x64; 3: MN-major A and B, 128x32x64; 4: as 1 with A copied
- * into tensor memory and read from there), each product in
+ * into tensor memory and read from there; 5: 64x32x128 from the lower half of a 128-row A
+ * tile), each product in
  * three bf16 hi/lo terms, and compares with the same products on CUDA cores.  Writes
  * out2[0] = max |difference|, out2[1] = max |reference| (host memory).  Synchronous;
  * allocates nothing.  Returns GDN_OK, GDN_ERR_NULL, GDN_ERR_SHAPE (bad case) or GDN_ERR_CUDA.

@@ -7,7 +7,7 @@ from gated_deltanet_token_b200 import gdn
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("case", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("case", [0, 1, 2, 3, 4, 5])
 def test_tc_layout_case(case):
     err, mag = gdn.gdn_selftest_tc(case)
     assert mag > 0.1
