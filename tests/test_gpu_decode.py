@@ -55,3 +55,12 @@ def test_prefill_then_decode_matches_longer_prefill(oracle_mod):
     ref = oracle_mod.prefill(full)
     assert np.abs(y[0] - ref["y"][T]).max() <= 1e-4
     assert np.linalg.norm(S[0] - ref["final_state"][0]) / np.linalg.norm(ref["final_state"][0]) <= 1e-4
+
+
+def test_decode_norm_weights(oracle_mod):
+    """A non-trivial norm_w (every component different) through the decode step's output norm."""
+    inp = make_inputs("decode_N256_bf16", n_seqs=7, h_qk=2, h_v=4, dtype="f32")
+    inp["norm_w"] = np.random.default_rng(6).uniform(0.5, 1.5, inp["norm_w"].shape).astype(np.float32)
+    ref = oracle_mod.decode(inp)
+    y, S, _ = run_decode(inp, torch.float32)
+    check_fp32(y, ref["y"], S, ref["state"])

@@ -181,3 +181,36 @@ def test_fused_output_norm_matches_separate_epilogue(oracle_mod, monkeypatch, ou
     r = float(np.sqrt(np.mean(ref["y"] ** 2)))
     tol = 1e-5 * r if out_dtype == torch.float32 else 2.0 ** -8 * np.abs(ref["y"]).max()
     assert np.abs(y_f - y_e).max() <= tol
+
+
+def _random_norm_w(inp, seed=5):
+    inp["norm_w"] = np.random.default_rng(seed).uniform(0.5, 1.5, inp["norm_w"].shape).astype(np.float32)
+    return inp
+
+
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_norm_weights_bf16_path(oracle_mod, monkeypatch, fused, out_dtype):
+    """A non-trivial norm_w (every component different) through the fused output norm and
+    through the separate epilogue: a wrong component index in either shows up here."""
+    inp = _random_norm_w(make_inputs("varlen8_prefill_bf16", lengths=[70, 1, 130], h_qk=4, h_v=8))
+    ref = _oracle(oracle_mod, inp)
+    if not fused:
+        monkeypatch.setenv("GDN_NO_FUSED_NORM", "1")
+    y, S = run_prefill(inp, out_dtype)
+    check_bf16(y, ref["y"], S, ref["final_state"], y_is_bf16=out_dtype == torch.bfloat16)
+
+
+def test_norm_weights_fp32_path(oracle_mod):
+    inp = _random_norm_w(make_inputs("tiny_prefill_fp32"))
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_fp32(y, ref["y"], S, ref["final_state"])
+
+
+def test_q_scale_bf16_path(oracle_mod):
+    """q_scale on the tensor-core path (the prologue scales the normalised query)."""
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[90, 40], h_qk=2, h_v=4)
+    ref = oracle_mod.prefill(inp, q_scale=0.7)
+    y, S = run_prefill(inp, torch.float32, q_scale=0.7)
+    check_bf16(y, ref["y"], S, ref["final_state"])
