@@ -19,12 +19,13 @@
 // Prologue (k_prologue_tc, persistent over (head group, half chunk) items): conv + SiLU of
 // q, k, v, L2 norm of q and k; writes the [K;Q] hi/lo operand tile of each (chunk, QK head)
 // and v as fp32 slices.
-// Phase A (k_chunkprep_tc, parallel over chunks x QK heads): [K;Q] K^T on tcgen05; per
-// value head: gates, gamma, A, M o QK^T, T = (I + A)^-1 (blocked 16 x 16 forward
-// substitution), P = (M o QK^T) T, and the [T;P] hi/lo tile.
+// Phase A (k_chunkprep_tc, parallel over chunks x QK heads): [K;Q] K^T on tcgen05; for both
+// value heads of a pair at once: gates, gamma, A, M o QK^T, T = (I + A)^-1 (blocked 16 x 16
+// forward substitution), P = (M o QK^T) T, and the [T;P] hi/lo tiles.
 // Phase B (k_chunkscan_tc, sequential over one sequence's chunks, parallel over value
 // heads and 32-row slices of the state): the three MMA rounds above per chunk, with the
-// next chunk's tiles bulk-copied into a second stage while the current one computes.
+// next chunk's tiles bulk-copied into a second stage while the current one computes, and
+// (by default) the gated output norm fused in.
 #pragma once
 #include <cuda.h>
 
@@ -771,8 +772,9 @@ enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 // width 2 nv: the lo tile follows the hi tile at the operand's N stride) plus a_lo b_hi; the
 // epilogue adds the two column halves.  (These small-N MMAs are bound by reading the A tile
 // from shared memory, so two MMAs per k-step beat three of width nv.)  One barrier per chunk,
-// at its start, orders the S tile, the stage reuse and the abort decision.
-
+// at its start, orders the S tile, the stage reuse and the abort decision; a named barrier
+// over the warps that own TMEM lanes 0..63 (warps 0, 1, 4, 5) hands R and U-tilde to the MMA
+// thread between rounds.
 //
 // Fused output norm (YM != PB_Y_RAW; clusters of the four slices of a value head; 12 warps):
 // warps 10 and 11 own TMEM lanes 64..127, i.e. the 64 tokens' y rows, and take the whole y
@@ -844,7 +846,8 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // D_a 0..63, D_cd 64..127, D_e 128..191
     tc::tmem_relinquish();
   }
-  // barrier over the four warps that own TMEM lanes 0..63 (warps 0, 1, 4, 5)
+  // named barrier over a subset of the warps (id 1: the R / U-tilde writers, id 2: all but
+  // the norm warps)
   auto named_bar_sync = [](int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
   };
