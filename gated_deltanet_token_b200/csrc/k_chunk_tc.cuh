@@ -466,7 +466,10 @@ __global__ void __launch_bounds__(256, 2)
                    const float* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
                    uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
-  const int chunk = blockIdx.y;  // head-fastest grid: concurrent CTAs read adjacent tiles
+  // head-fastest grid, chunks from the last: the prologue writes its tiles in chunk order, so
+  // the ones it wrote last are still in L2 when they are read here first, and the early
+  // chunks' [T;P] tiles (written here last) are in L2 when phase B starts on them
+  const int chunk = gridDim.y - 1 - blockIdx.y;
   const ChunkEntry e = chunk_entry(tab, d.total_tokens, chunk);
   if (e.len == 0) return;
   const int j = blockIdx.x, hq = d.h_qk, hv = d.h_v, G = hv / hq, L = e.len;
