@@ -10,7 +10,10 @@ reported under "decode" as state GB/s against the measured HBM copy bandwidth.
 
 Timing: W untimed warm-up steps, then K steps between a barrier + cuda synchronize on both
 sides, timed with CUDA events on the launching stream.  Inputs rotate over three device
-copies (3 x 97 MiB > 126 MB L2) so no step starts with its inputs in L2.
+copies (3 x 97 MiB > 126 MB L2) so no step starts with its inputs in L2.  A second pass of
+the same K steps brackets every kernel with CUDA events for the per-kernel durations of the
+roofline.  "e2e" runs the public call on inputs copied in from pinned host memory and results
+copied back every step, pipelined over three streams.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
   python bench.py --configs      # one JSON line per workload: GPU time and the oracle beside it
@@ -332,8 +335,6 @@ def gpu_arm(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.2)
-    gdn.gdn_profile_enable(True)
-    gdn.gdn_profile_read()
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -344,14 +345,23 @@ def gpu_arm(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    prof = gdn.gdn_profile_read()
-    gdn.gdn_profile_enable(False)
     ms_local = e0.elapsed_time(e1)
     ms = max_over_ranks(ms_local, dev)
     ms_per_step = ms / args.steps
     tokens_all = sum_over_ranks(float(T * args.steps), dev)
     value = tokens_all / (ms / 1e3) / 1e6
-    launches = sum(v[0] for v in prof.values())
+    # The same K steps again with every kernel bracketed by CUDA events on the call's stream:
+    # the per-kernel durations of the roofline.  (The events order the kernels strictly, so the
+    # launch overlap between them is absent from this pass and its step time is not reported.)
+    gdn.gdn_profile_enable(True)
+    gdn.gdn_profile_read()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    prof = gdn.gdn_profile_read()
+    gdn.gdn_profile_enable(False)
+    launches = sum(v[0] for v in prof.values())  # the same launches as the timed steps
 
     # --- roofline of the dominant kernel ------------------------------------------------------
     dom = max(prof.items(), key=lambda kv: kv[1][1])
@@ -416,35 +426,61 @@ def gpu_arm(args):
     del dd
 
     # --- end to end through the public call with host buffers ----------------------------------
+    # Every step copies its own inputs in from pinned host memory and its y and final state back
+    # out.  Three streams (host->device copies, the prefill, device->host copies) and two buffer
+    # slots let step i+1's inputs cross the host link while step i computes and step i-1's
+    # results return, as a serving loop would run them.
     host = {n: to_dev(inp[n], "cpu").pin_memory() for n in names}
-    dbuf = {n: torch.empty_like(host[n], device=dev) for n in names}
-    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    fs_host = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    n_slots = 2
+    dbuf = [{n: torch.empty_like(host[n], device=dev) for n in names} for _ in range(n_slots)]
+    ys = [torch.empty_like(y) for _ in range(n_slots)]
+    fss = [torch.empty_like(fs) for _ in range(n_slots)]
+    y_host = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(n_slots)]
+    fs_host = [torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True) for _ in range(n_slots)]
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(n_slots)]   # the slot's inputs are on the device
+    ev_run = [torch.cuda.Event() for _ in range(n_slots)]  # the slot's prefill has finished
+    ev_out = [torch.cuda.Event() for _ in range(n_slots)]  # the slot's results are on the host
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = y.numel() * y.element_size() + fs.numel() * fs.element_size()
+    torch.cuda.synchronize()
 
-    def e2e_step():
-        for n in names:
-            dbuf[n].copy_(host[n], non_blocking=True)
-        gdn.gdn_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["z"], dbuf["a"], dbuf["b"], params["A_log"],
+    def e2e_step(i):
+        k = i % n_slots
+        b = dbuf[k]
+        s_in.wait_event(ev_run[k])  # the prefill two steps back is done with this slot's inputs
+        with torch.cuda.stream(s_in):
+            for n in names:
+                b[n].copy_(host[n], non_blocking=True)
+        ev_in[k].record(s_in)
+        s_run.wait_event(ev_in[k])
+        s_run.wait_event(ev_out[k])  # this slot's results of two steps back are on the host
+        gdn.gdn_prefill(b["q"], b["k"], b["v"], b["z"], b["a"], b["b"], params["A_log"],
                         params["dt_bias"], params["conv_w"], params["norm_w"], None, None,
-                        out_dtype=torch.bfloat16, y=y, final_state=fs, workspace=ws)
-        y_host.copy_(y, non_blocking=True)
-        fs_host.copy_(fs, non_blocking=True)
+                        out_dtype=torch.bfloat16, y=ys[k], final_state=fss[k], workspace=ws, stream=s_run)
+        ev_run[k].record(s_run)
+        s_out.wait_event(ev_run[k])
+        with torch.cuda.stream(s_out):
+            y_host[k].copy_(ys[k], non_blocking=True)
+            fs_host[k].copy_(fss[k], non_blocking=True)
+        ev_out[k].record(s_out)
 
     e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)  # every step's work follows its input copies on s_in
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(s_out)  # ... and ends with its result copies on s_out
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_val = sum_over_ranks(float(T * e2e_steps), dev) / (e2e_ms / 1e3) / 1e6
+    # the results that came back equal those of the device-resident timed steps (same inputs)
+    last = (e2e_steps - 1) % n_slots
+    e2e_match = bool(torch.equal(y_host[last], y.cpu()) and torch.equal(fs_host[last], fs.cpu()))
 
     # --- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only ---------------------
     cpu = None
@@ -468,7 +504,8 @@ def gpu_arm(args):
                    "l2": f"{n_sets} rotating input sets of 97 MiB (> 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof, "cpu_baseline": cpu,
-        "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipeline": "3 streams, 2 slots", "matches_device": e2e_match},
         "gpu_launches": launches, "clocks": clk, "decode": decode,
     }
     print(json.dumps(out), flush=True)

@@ -10,6 +10,7 @@
 
 #include <atomic>
 #include <type_traits>
+#include <utility>
 
 #include "gdn.h"
 #include "gdn_common.cuh"
@@ -130,6 +131,37 @@ struct ProfScope {
   ProfScope(const char* name, cudaStream_t st) : i(prof_begin(name, st)), s(st) {}
   ~ProfScope() { prof_end(i, s); }
 };
+
+// Launches a tensor-core prefill kernel with programmatic dependent launch: its CTAs may
+// become resident while the previous kernel on the stream drains, and wait in
+// griddepcontrol.wait (their first statement) until it has completed.  GDN_NO_PDL=1 gives plain
+// stream order.  cluster_z > 1 adds a (1, 1, cluster_z) cluster shape.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_z,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (getenv_flag("GDN_NO_PDL") == 0) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster_z > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = (unsigned)cluster_z;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -353,11 +385,14 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
             make_stream_map(&tm_k, k, d->total_tokens, d->h_qk) != GDN_OK ||
             make_stream_map(&tm_v, v, d->total_tokens, d->h_v) != GDN_OK)
           return GDN_ERR_CUDA;
-        k_prologue_tc<<<grid, PRO_THREADS, PRO_SMEM, s>>>(kd, tabc, nitems, tm_q, tm_k, tm_v, conv_w, kq, F(L.vs));
+        if (launch_dep(k_prologue_tc, dim3(grid), dim3(PRO_THREADS), PRO_SMEM, s, 1, kd, tabc, nitems, tm_q, tm_k,
+                       tm_v, conv_w, kq, F(L.vs)) != cudaSuccess)
+          return GDN_ERR_CUDA;
       }
       ProfScope p("chunk_prep_tc", s);
-      k_chunkprep_tc<<<dim3(d->h_qk, L.max_chunks), 256, PA_TC_SMEM, s>>>(kd, tabc, a, b, A_log, dt_bias, kq, tp,
-                                                                          F(L.gb));
+      if (launch_dep(k_chunkprep_tc, dim3(d->h_qk, L.max_chunks), dim3(256), PA_TC_SMEM, s, 1, kd, tabc, a, b, A_log,
+                     dt_bias, (const uint8_t*)kq, tp, F(L.gb)) != cudaSuccess)
+        return GDN_ERR_CUDA;
     }
     // The output norm runs inside phase B (clusters of the four slices of a head) unless that
     // would take more waves of CTAs than the unclustered launch.
@@ -369,34 +404,21 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     const dim3 grid(d->n_seqs, d->h_v, D / TC_NV);
     if (fused) {
       ProfScope p("chunk_scan_tc_norm", s);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = grid;
-      cfg.blockDim = dim3(384);
-      cfg.dynamicSmemBytes = PB_TC_SMEM;
-      cfg.stream = s;
-      cudaLaunchAttribute attr;
-      attr.id = cudaLaunchAttributeClusterDimension;
-      attr.val.clusterDim.x = 1;
-      attr.val.clusterDim.y = 1;
-      attr.val.clusterDim.z = D / TC_NV;
-      cfg.attrs = &attr;
-      cfg.numAttrs = 1;
       const uint16_t* zb = static_cast<const uint16_t*>(z);
-      cudaError_t e = kd.out_bf16
-          ? cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_BF16>, kd, (const int*)cu_seqlens, seqc0c,
-                               (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
-                               init_state, F(L.yraw), final_state, zb, norm_w, y)
-          : cudaLaunchKernelEx(&cfg, k_chunkscan_tc<PB_Y_F32>, kd, (const int*)cu_seqlens, seqc0c,
-                               (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
-                               init_state, F(L.yraw), final_state, zb, norm_w, y);
+      cudaError_t e = launch_dep(kd.out_bf16 ? k_chunkscan_tc<PB_Y_BF16> : k_chunkscan_tc<PB_Y_F32>, grid, dim3(384),
+                                 PB_TC_SMEM, s, D / TC_NV, kd, (const int*)cu_seqlens, seqc0c, (const uint8_t*)kq,
+                                 (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs), init_state,
+                                 F(L.yraw), final_state, zb, norm_w, y);
       if (e != cudaSuccess) return GDN_ERR_CUDA;
       return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
     }
     {
       ProfScope p("chunk_scan_tc", s);
-      k_chunkscan_tc<PB_Y_RAW><<<grid, 288, PB_TC_SMEM, s>>>(kd, cu_seqlens, seqc0c, kq, tp, F(L.gb), F(L.vs),
-                                                             init_state, F(L.yraw), final_state, nullptr, nullptr,
-                                                             nullptr);
+      if (launch_dep(k_chunkscan_tc<PB_Y_RAW>, grid, dim3(288), PB_TC_SMEM, s, 1, kd, (const int*)cu_seqlens, seqc0c,
+                     (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
+                     init_state, F(L.yraw), final_state, (const uint16_t*)nullptr, (const float*)nullptr,
+                     (void*)nullptr) != cudaSuccess)
+        return GDN_ERR_CUDA;
     }
     if (d->total_tokens > 0) {
       ProfScope p("epilogue", s);

@@ -263,6 +263,8 @@ __global__ void __launch_bounds__(PRO_THREADS, 1) k_prologue_tc(Dims d, const Ch
                                                         const __grid_constant__ CUtensorMap tm_v,
                                                         const float* __restrict__ conv_w,
                                                         uint8_t* __restrict__ kq_ws, float* __restrict__ vs_ws) {
+  tc::grid_dep_wait();  // all earlier work on the stream (the inputs, the last call's use of the workspace) is done
+  tc::grid_dep_launch_dependents();
   const int hq = d.h_qk, hv = d.h_v;
   const int ngroups = 2 * ((hq + PRO_HG - 1) / PRO_HG) + (hv + PRO_HG - 1) / PRO_HG;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -466,6 +468,8 @@ __global__ void __launch_bounds__(256, 2)
                    const float* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
                    uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
+  tc::grid_dep_wait();  // the prologue's tiles are complete
+  tc::grid_dep_launch_dependents();
   // head-fastest grid, chunks from the last: the prologue writes its tiles in chunk order, so
   // the ones it wrote last are still in L2 when they are read here first, and the early
   // chunks' [T;P] tiles (written here last) are in L2 when phase B starts on them
@@ -799,6 +803,8 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
                    const float* init_state, float* __restrict__ y_raw,
                    float* final_state,
                    const uint16_t* __restrict__ z, const float* __restrict__ norm_w, void* __restrict__ y) {
+  tc::grid_dep_wait();  // phase A's tiles and gates are complete
+  tc::grid_dep_launch_dependents();
   constexpr int NV = TC_NV, NH = NV / 2;
   constexpr bool FUSED = YM != PB_Y_RAW;
   const int n = blockIdx.x, h = blockIdx.y, sl = blockIdx.z, i0 = sl * NV;

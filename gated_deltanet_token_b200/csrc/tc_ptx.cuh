@@ -23,6 +23,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------------
+// grid_dep_wait: the calling thread waits until the grids this launch depends on have completed
+// and their memory operations are visible (at once when the launch carried no such dependency).
+// Every thread calls it before its first global memory access.
+// grid_dep_launch_dependents: this CTA no longer holds back the launch of the next dependent
+// grid, whose CTAs may then take free SM resources and wait in their own grid_dep_wait.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- mbarriers ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
