@@ -121,7 +121,7 @@ def test_long_prefill_T262144_sampled_heads(oracle_mod):
 
 # ---- the bf16 (tensor-core) path: head ratios, ragged lengths, SIMT cross-check ----------
 
-@pytest.mark.parametrize("ratio", [1, 2, 4])
+@pytest.mark.parametrize("ratio", [1, 2, 3, 4, 8])
 def test_head_ratios_bf16_tensor_core_path(oracle_mod, ratio):
     inp = make_inputs("varlen8_prefill_bf16", lengths=[77, 3, 130], h_qk=2, h_v=2 * ratio)
     ref = _oracle(oracle_mod, inp)
