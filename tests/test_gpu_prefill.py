@@ -214,3 +214,43 @@ def test_q_scale_bf16_path(oracle_mod):
     ref = oracle_mod.prefill(inp, q_scale=0.7)
     y, S = run_prefill(inp, torch.float32, q_scale=0.7)
     check_bf16(y, ref["y"], S, ref["final_state"])
+
+
+def test_back_to_back_calls_chain_the_state(oracle_mod):
+    """Three prefill calls queued on one stream with no synchronisation between them, sharing one
+    workspace, each reading the state the previous one wrote into the same buffer
+    (init_state aliases final_state).  The kernels of a call may become resident while the
+    previous call's kernels drain, so this checks that every read still follows the write it
+    depends on: each segment's y and the final state match the oracle run segment by segment."""
+    from gated_deltanet_token_b200 import gdn
+    from tests._helpers import to_dev
+
+    lens = [300, 200, 130]
+    segs = [make_inputs("prefill_T4096_bf16", seed=10 + i, T=L, h_qk=4, h_v=8, init_state=True)
+            for i, L in enumerate(lens)]
+    for sg in segs[1:]:  # one layer: the same parameters in every segment
+        for nm in ("A_log", "dt_bias", "conv_w", "norm_w"):
+            sg[nm] = segs[0][nm]
+    par = {nm: to_dev(segs[0][nm]) for nm in ("A_log", "dt_bias", "conv_w", "norm_w")}
+    dims = gdn.make_dims(1, max(lens), 4, 8, gdn.GDN_DTYPE_BF16, gdn.GDN_DTYPE_F32)
+    ws = torch.empty(gdn.gdn_prefill_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    state = to_dev(segs[0]["init_state"]).clone()
+    dev_in = [{nm: to_dev(sg[nm]) for nm in ("q", "k", "v", "z", "a", "b")} for sg in segs]
+    torch.cuda.synchronize()
+    ys = []
+    for t in dev_in:  # queued back to back
+        y, _ = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["z"], t["a"], t["b"], par["A_log"], par["dt_bias"],
+                               par["conv_w"], par["norm_w"], state, None, out_dtype=torch.float32,
+                               final_state=state, workspace=ws)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert gdn.gdn_read_device_status() == 0
+    init = segs[0]["init_state"].astype(np.float32)
+    for sg, y in zip(segs, ys):  # the oracle, segment by segment, each from the last one's state
+        sg = dict(sg)
+        sg["init_state"] = init
+        ref = _oracle(oracle_mod, sg)
+        init = ref["final_state"].astype(np.float32)
+        check_bf16(y.float().cpu().numpy().astype(np.float64), ref["y"], ref["final_state"], ref["final_state"])
+    check_bf16(ys[-1].float().cpu().numpy().astype(np.float64), ref["y"], state.cpu().numpy().astype(np.float64),
+               ref["final_state"])
