@@ -173,10 +173,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def source_sha() -> str:
+# The source files each measured kernel is compiled from (its own header and what it includes).
+# Launch configurations live in gdn_api.cu; a change there is re-captured with the kernel's.
+KERNEL_SOURCES = {
+    "prologue_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
+    "chunk_prep_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
+    "chunk_scan_tc_norm": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
+    "decode": ("k_decode.cuh", "gdn_common.cuh"),
+    "chunk_phaseB_simt": ("k_chunk_simt.cuh", "gdn_common.cuh"),
+}
+
+
+def source_sha(files=None) -> str:
+    """Hash of the named kernel source files (default: every file of csrc/)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_token_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -184,14 +196,14 @@ def source_sha() -> str:
 
 def ncu_traffic(kernel: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
-    kernel sources changed since those counters were taken."""
+    kernel's source files changed since those counters were taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(kernel)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("src_sha") != source_sha():
+    if not rec or kernel not in KERNEL_SOURCES or rec.get("src_sha") != source_sha(KERNEL_SOURCES[kernel]):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -327,6 +327,7 @@ const char* gdn_status_string(int code) {
     case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
     case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT";
+    case GDN_ERR_INDEX: return "GDN_ERR_INDEX";
     default: return "GDN_ERR_UNKNOWN";
   }
 }
@@ -453,10 +454,11 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
-               const float* a, const float* b, const float* A_log, const float* dt_bias,
-               const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
-               gdn_stream_t stream) {
+// One decode step, on per-sequence state (slots == nullptr) or on pool slots.
+static int decode_impl(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+                const float* a, const float* b, const float* A_log, const float* dt_bias,
+                const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+                const int32_t* slots, int n_slots, gdn_stream_t stream) {
   int rc = check_dims(d, true);
   if (rc != GDN_OK) return rc;
   const void* ptrs[] = {q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y};
@@ -471,16 +473,60 @@ int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v,
   ProfScope p("decode", s);
   if (kd.in_bf16 && kd.out_bf16)
     k_decode<true, true><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
-                                              conv_state, state, y);
+                                              conv_state, state, y, slots, n_slots);
   else if (kd.in_bf16)
     k_decode<true, false><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
-                                               conv_state, state, y);
+                                               conv_state, state, y, slots, n_slots);
   else if (kd.out_bf16)
     k_decode<false, true><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
-                                               conv_state, state, y);
+                                               conv_state, state, y, slots, n_slots);
   else
     k_decode<false, false><<<grid, 256, 0, s>>>(kd, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w,
-                                                conv_state, state, y);
+                                                conv_state, state, y, slots, n_slots);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+               const float* a, const float* b, const float* A_log, const float* dt_bias,
+               const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+               gdn_stream_t stream) {
+  return decode_impl(d, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y, nullptr, 0,
+                     stream);
+}
+
+int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+                     const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     const float* conv_w, const float* norm_w, void* conv_state_pool, float* state_pool,
+                     int32_t n_slots, const int32_t* slot_ids, void* y, gdn_stream_t stream) {
+  if (!slot_ids) return GDN_ERR_NULL;
+  if (!aligned16(slot_ids)) return GDN_ERR_ALIGN;
+  if (n_slots < 1) return GDN_ERR_SHAPE;
+  return decode_impl(d, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state_pool, state_pool, y,
+                     slot_ids, n_slots, stream);
+}
+
+int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, const void* v,
+                           const int32_t* cu_seqlens, void* conv_state, gdn_stream_t stream) {
+  const int rc = check_dims(d, false);
+  if (rc != GDN_OK) return rc;
+  if (!conv_state) return GDN_ERR_NULL;
+  if (d->total_tokens > 0 && (!q || !k || !v)) return GDN_ERR_NULL;
+  if (!cu_seqlens && d->n_seqs != 1) return GDN_ERR_NULL;
+  const void* ptrs[] = {q, k, v, cu_seqlens, conv_state};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Dims kd = kdims(d);
+  const dim3 grid(d->n_seqs, 3);
+  ProfScope p("conv_state_out", s);
+  if (kd.in_bf16)
+    k_conv_state_out<uint16_t><<<grid, 256, 0, s>>>(kd, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                                    static_cast<const uint16_t*>(v), cu_seqlens,
+                                                    static_cast<uint16_t*>(conv_state));
+  else
+    k_conv_state_out<float><<<grid, 256, 0, s>>>(kd, static_cast<const float*>(q), static_cast<const float*>(k),
+                                                 static_cast<const float*>(v), cu_seqlens,
+                                                 static_cast<float*>(conv_state));
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

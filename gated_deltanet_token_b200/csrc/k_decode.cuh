@@ -8,6 +8,10 @@
 // using y_i = alpha (S q)_i + e (k . q), so each 512-byte state row is read once and
 // written once.  Dot products are warp-shuffle reductions over the row's 128 entries (four
 // per lane).  Last, y is RMS-normalised per value head and gated by SiLU(z).
+//
+// With `slots`, sequence n's state and conv history live in pool slot slots[n] (a resident
+// state pool, as a serving loop keeps one); a negative slot marks a padding entry that reads
+// and writes nothing, and a slot past the pool sets the device status and skips the entry.
 #pragma once
 #include "gdn_common.cuh"
 
@@ -24,9 +28,19 @@ __global__ void __launch_bounds__(256) k_decode(Dims d, const void* __restrict__
                                                 const float* __restrict__ dt_bias,
                                                 const float* __restrict__ conv_w,
                                                 const float* __restrict__ norm_w, void* conv_state,
-                                                float* state, void* __restrict__ y) {
+                                                float* state, void* __restrict__ y,
+                                                const int32_t* __restrict__ slots, int n_slots) {
   using E = typename std::conditional<BF16, uint16_t, float>::type;
   const int n = blockIdx.x, j = blockIdx.y;
+  int slot = n;
+  if (slots) {
+    slot = slots[n];
+    if (slot < 0) return;  // padding entry
+    if (slot >= n_slots) {
+      if (threadIdx.x == 0) atomicExch(&g_gdn_status, -8);
+      return;
+    }
+  }
   const int hq = d.h_qk, hv = d.h_v, G = hv / hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t cconv = (size_t)(2 * hq + hv) * D;
@@ -37,7 +51,7 @@ __global__ void __launch_bounds__(256) k_decode(Dims d, const void* __restrict__
   __shared__ float alpha_s[8], beta_s[8];
 
   // conv + SiLU over this CTA's channels, and the conv-history shift (raw values, bit-exact)
-  E* cs = static_cast<E*>(conv_state) + (size_t)n * 3 * cconv;
+  E* cs = static_cast<E*>(conv_state) + (size_t)slot * 3 * cconv;
   const int nch = 2 * D + G * D;
   for (int c = tid; c < nch; c += blockDim.x) {
     size_t ch;
@@ -91,7 +105,7 @@ __global__ void __launch_bounds__(256) k_decode(Dims d, const void* __restrict__
 
   // state rows: G * 128 rows, an equal contiguous share per warp, DEC_ROWS in flight
   const int rows_per_warp = G * D / 8;
-  const size_t state0 = ((size_t)n * hv + (size_t)j * G) * D * D;
+  const size_t state0 = ((size_t)slot * hv + (size_t)j * G) * D * D;
   for (int r0 = warp * rows_per_warp; r0 < (warp + 1) * rows_per_warp; r0 += DEC_ROWS) {
     float4 s[DEC_ROWS];
 #pragma unroll
@@ -127,6 +141,37 @@ __global__ void __launch_bounds__(256) k_decode(Dims d, const void* __restrict__
     o.z = yv.z * inv * nw.z * silu_f(zz.z);
     o.w = yv.w * inv * nw.w * silu_f(zz.w);
     store4<OUT_BF16>(y, off, o);
+  }
+}
+
+// The decode step's conv history after a prefill: the raw (pre-conv) q | k | v channels of
+// each sequence's last three tokens, row r = token te - 3 + r, in the conv_state layout
+// [N][3][C_conv].  Rows before the sequence's first token are zeros, as the prefill's own
+// history starts at zero.  One CTA per (sequence, row); 16-byte copies.  A cu_seqlens entry
+// outside [0, T_tot] or decreasing sets the device status and writes zeros.
+template <typename E>
+__global__ void __launch_bounds__(256) k_conv_state_out(Dims d, const E* __restrict__ q, const E* __restrict__ k,
+                                                        const E* __restrict__ v, const int* __restrict__ cu,
+                                                        E* __restrict__ out) {
+  const int n = blockIdx.x, r = blockIdx.y;
+  int ts = cu ? cu[n] : 0, te = cu ? cu[n + 1] : d.total_tokens;
+  if (ts < 0 || te < ts || te > d.total_tokens) {
+    if (threadIdx.x == 0) atomicExch(&g_gdn_status, -8);
+    ts = te = 0;
+  }
+  const int t = te - 3 + r;
+  const size_t cq = (size_t)d.h_qk * D, cv = (size_t)d.h_v * D, cconv = 2 * cq + cv;
+  constexpr int V = 16 / sizeof(E);  // elements per 16-byte copy (never straddles a stream)
+  uint4* o = reinterpret_cast<uint4*>(out + ((size_t)n * 3 + r) * cconv);
+  for (size_t c = (size_t)threadIdx.x * V; c < cconv; c += (size_t)blockDim.x * V) {
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= ts) {
+      const E* src = c < cq ? q + (size_t)t * cq + c
+                   : c < 2 * cq ? k + (size_t)t * cq + (c - cq)
+                                : v + (size_t)t * cv + (c - 2 * cq);
+      x = *reinterpret_cast<const uint4*>(src);
+    }
+    o[c / V] = x;
   }
 }
 

@@ -14,6 +14,7 @@ import os
 import torch
 
 GDN_OK = 0
+GDN_ERR_INDEX = -8
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -63,6 +64,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill_noalloc.argtypes = [dp] + [vp] * 14 + [vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode.argtypes = [dp] + [vp] * 13 + [vp]
+        L.gdn_decode_slots.restype = ctypes.c_int
+        L.gdn_decode_slots.argtypes = [dp] + [vp] * 12 + [ctypes.c_int32, vp, vp, vp]
+        L.gdn_prefill_conv_state.restype = ctypes.c_int
+        L.gdn_prefill_conv_state.argtypes = [dp] + [vp] * 5 + [vp]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_read_device_status.restype = ctypes.c_int
@@ -222,4 +227,50 @@ def gdn_decode(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, sta
                           _ptr(state), _ptr(y), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode")
+    return y
+
+
+def gdn_prefill_conv_state(q, k, v, cu_seqlens=None, *, conv_state=None, stream=None):
+    """The decode conv history after a prefill over the same packed q, k, v: per sequence the
+    raw q | k | v channels of its last three tokens (zeros before its first token).  Returns
+    conv_state [N, 3, C_conv] in the inputs' dtype."""
+    T, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    n = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    dims = make_dims(n, T, h_qk, h_v, _dt(q), _dt(q), d_k, d_v)
+    if conv_state is None:
+        conv_state = torch.empty((n, 3, (2 * h_qk + h_v) * d_k), dtype=q.dtype, device=q.device)
+    rc = lib().gdn_prefill_conv_state(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                      _ptr(conv_state), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_prefill_conv_state")
+    return conv_state
+
+
+def gdn_decode_slots(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state_pool, state_pool,
+                     slot_ids, *, out_dtype=None, y=None, q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6,
+                     stream=None):
+    """One decode step on resident pools: sequence n updates conv_state_pool[slot_ids[n]] and
+    state_pool[slot_ids[n]] in place (slot_ids int32 on the device; a negative id is a padding
+    entry).  Returns y [N, h_v, 128]."""
+    N, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    if slot_ids.dtype != torch.int32 or slot_ids.numel() != N:
+        raise TypeError("slot_ids must be int32 with one entry per sequence")
+    if conv_state_pool.shape[0] != state_pool.shape[0]:
+        raise ValueError("conv_state_pool and state_pool must have the same number of slots")
+    if out_dtype is None:
+        out_dtype = q.dtype
+    dims = make_dims(N, N, h_qk, h_v, _dt(q), _dt(torch.empty(0, dtype=out_dtype)), d_k, d_v, q_scale,
+                     l2_eps, rms_eps)
+    if y is None:
+        y = torch.empty((N, h_v, d_v), dtype=out_dtype, device=q.device)
+    rc = lib().gdn_decode_slots(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(a), _ptr(b),
+                                _ptr(A_log), _ptr(dt_bias), _ptr(conv_w), _ptr(norm_w), _ptr(conv_state_pool),
+                                _ptr(state_pool), ctypes.c_int32(state_pool.shape[0]), _ptr(slot_ids), _ptr(y),
+                                _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_slots")
     return y

@@ -49,6 +49,7 @@ typedef struct CUstream_st* gdn_stream_t; /* identical to cudaStream_t */
 #define GDN_ERR_WORKSPACE (-5)      /* workspace missing or smaller than required */
 #define GDN_ERR_CUDA (-6)           /* a CUDA launch or runtime call failed */
 #define GDN_ERR_DEVICE_TIMEOUT (-7) /* a bounded device-side wait ran out (device status) */
+#define GDN_ERR_INDEX (-8)          /* a device-side index was out of range (device status) */
 
 /* dtype codes */
 #define GDN_DTYPE_F32 0
@@ -120,14 +121,55 @@ int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v,
                const float* conv_w, const float* norm_w, void* conv_state, float* state,
                void* y, gdn_stream_t stream);
 
+/*
+ * Prefill -> decode hand-off, part 1: the decode conv history each sequence has after a
+ * prefill over the same packed inputs.  Writes, per sequence n, the raw (pre-conv) q | k | v
+ * channels of its last three tokens: conv_state[n][r] = x_{te-3+r}, te = cu_seqlens[n+1], in
+ * gdn_decode's conv_state layout.  Rows before the sequence's first token are zeros (every
+ * prefill sequence starts with a zero conv history), so a sequence of fewer than three tokens
+ * gets leading zero rows.  The copy is bit-exact.
+ *
+ *   q, k        [T_tot][h_qk][d_k]   in_dtype
+ *   v           [T_tot][h_v][d_v]    in_dtype
+ *   cu_seqlens  [N+1] int32 device array, or NULL when N == 1
+ *   conv_state  [N][3][C_conv]       in_dtype (written)
+ * Only the dims' shape fields and in_dtype are used.  A cu_seqlens entry outside
+ * [0, T_tot] or below its predecessor makes that sequence's rows zeros and sets the device
+ * status to GDN_ERR_INDEX.
+ */
+int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, const void* v,
+                           const int32_t* cu_seqlens, void* conv_state, gdn_stream_t stream);
+
+/*
+ * Prefill -> decode hand-off, part 2: gdn_decode on resident pools, the way a serving loop
+ * keeps one state and one conv history per live request.  Same arguments and results as
+ * gdn_decode, except that sequence n reads and updates pool slot slot_ids[n]:
+ *
+ *   conv_state_pool [n_slots][3][C_conv]       in_dtype, in/out
+ *   state_pool      [n_slots][h_v][d_v][d_k]   fp32, in/out
+ *   slot_ids        [N] int32 device array
+ *
+ * A negative slot id marks a padding entry: nothing is read or written for it (its y rows
+ * are left as they were).  A slot id >= n_slots is skipped the same way and sets the device
+ * status to GDN_ERR_INDEX.  Two entries naming the same slot race on it: the caller keeps the
+ * ids of one call distinct.  Returns GDN_ERR_NULL (slot_ids NULL), GDN_ERR_SHAPE
+ * (n_slots < 1) or what gdn_decode returns.
+ */
+int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const void* v, const void* z,
+                     const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     const float* conv_w, const float* norm_w, void* conv_state_pool, float* state_pool,
+                     int32_t n_slots, const int32_t* slot_ids, void* y, gdn_stream_t stream);
+
 /* Static, NUL-terminated name of a return code ("GDN_OK", "GDN_ERR_SHAPE", ...). */
 const char* gdn_status_string(int code);
 
 /*
  * Synchronises `stream`, then returns and clears the library's device status word for
  * the current device: GDN_OK, GDN_ERR_DEVICE_TIMEOUT if a bounded device-side wait gave up
- * since the last read, or GDN_ERR_CUDA if a kernel found its launch shape inconsistent and
- * did nothing.  Returns GDN_ERR_CUDA also if the synchronisation fails.
+ * since the last read, GDN_ERR_INDEX if a slot id or a cu_seqlens entry was out of range
+ * (see gdn_decode_slots, gdn_prefill_conv_state), or GDN_ERR_CUDA if a kernel found its
+ * launch shape inconsistent and did nothing.  Returns GDN_ERR_CUDA also if the
+ * synchronisation fails.
  */
 int gdn_read_device_status(gdn_stream_t stream);
 

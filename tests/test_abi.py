@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(glib):
 def test_status_strings(glib):
     expect = {0: "GDN_OK", -1: "GDN_ERR_NULL", -2: "GDN_ERR_SHAPE", -3: "GDN_ERR_DTYPE",
               -4: "GDN_ERR_ALIGN", -5: "GDN_ERR_WORKSPACE", -6: "GDN_ERR_CUDA",
-              -7: "GDN_ERR_DEVICE_TIMEOUT"}
+              -7: "GDN_ERR_DEVICE_TIMEOUT", -8: "GDN_ERR_INDEX"}
     for c, s in expect.items():
         assert glib.gdn_status_string(c) == s
     assert glib.gdn_status_string(-99) == "GDN_ERR_UNKNOWN"
@@ -100,6 +100,36 @@ def test_decode_rejects_bad_arguments(glib):
     bad[10] = FAKE + 8
     assert call(glib.make_dims(4, 4, 16, 32, 1, 1), bad) == -4
     assert call(glib.make_dims(4, 4, 16, 32, 5, 1), good) == -3
+
+
+def test_handoff_calls_reject_bad_arguments(glib):
+    L = glib.lib()
+    V = ctypes.c_void_p
+
+    def conv(dims, q=FAKE, k=FAKE, v=FAKE, cu=FAKE, out=FAKE):
+        return L.gdn_prefill_conv_state(None if dims is None else ctypes.byref(dims),
+                                        *[V(x) if x else None for x in (q, k, v, cu, out)], None)
+
+    two = glib.make_dims(2, 100, 16, 32, 1, 1)
+    assert conv(None) == -1
+    assert conv(two, out=None) == -1
+    assert conv(two, cu=None) == -1  # two sequences need cu_seqlens
+    assert conv(two, q=None) == -1
+    assert conv(two, v=FAKE + 4) == -4
+    assert conv(glib.make_dims(2, 100, 16, 30, 1, 1)) == -2
+    assert conv(glib.make_dims(2, 100, 16, 32, 3, 1)) == -3
+
+    def slots(dims, n_slots=4, ids=FAKE, pool=FAKE):
+        ptrs = [FAKE] * 10 + [pool, FAKE]
+        return L.gdn_decode_slots(ctypes.byref(dims), *[V(x) for x in ptrs], ctypes.c_int32(n_slots),
+                                  V(ids) if ids else None, V(FAKE), None)
+
+    four = glib.make_dims(4, 4, 16, 32, 1, 1)
+    assert slots(four, ids=None) == -1
+    assert slots(four, ids=FAKE + 4) == -4
+    assert slots(four, n_slots=0) == -2
+    assert slots(glib.make_dims(4, 5, 16, 32, 1, 1)) == -2  # total_tokens != n_seqs
+    assert slots(four, pool=FAKE + 8) == -4
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

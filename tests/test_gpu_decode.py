@@ -64,3 +64,113 @@ def test_decode_norm_weights(oracle_mod):
     ref = oracle_mod.decode(inp)
     y, S, _ = run_decode(inp, torch.float32)
     check_fp32(y, ref["y"], S, ref["state"])
+
+
+# ---- prefill -> decode hand-off on resident pools ---------------------------------------
+
+def _raw_history(inp, ts, te):
+    """Rows x_{te-3..te-1} of the raw q | k | v channels, zeros before token ts (numpy)."""
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    width = q.shape[1] * q.shape[2] * 2 + v.shape[1] * v.shape[2]
+    rows = np.zeros((3, width), dtype=q.dtype)
+    for r in range(3):
+        t = te - 3 + r
+        if t >= ts:
+            rows[r] = np.concatenate([q[t].ravel(), k[t].ravel(), v[t].ravel()])
+    return rows
+
+
+def _as_np(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_conv_state_is_the_raw_history(dtype):
+    from gated_deltanet_token_b200 import gdn
+
+    lens = [0, 1, 2, 3, 70, 130]
+    inp = make_inputs("varlen8_prefill_bf16", lengths=lens, h_qk=2, h_v=4, dtype=dtype)
+    cu = inp["cu_seqlens"]
+    cs = gdn.gdn_prefill_conv_state(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]),
+                                    to_dev(cu.astype(np.int32)))
+    torch.cuda.synchronize()
+    got = _as_np(cs)
+    for n in range(len(lens)):
+        assert np.array_equal(got[n], _raw_history(inp, int(cu[n]), int(cu[n + 1])))  # bit-exact
+
+
+def test_handoff_prefill_to_decode_slots(oracle_mod):
+    """Prefill the first L_n tokens of each sequence, hand the final states and conv histories to
+    pool slots (scattered, with spare slots), decode token L_n + 1 of each sequence plus one
+    padding entry through gdn_decode_slots, and compare with the oracle's prefill over L_n + 1
+    tokens: y of the last token and the state.  Spare slots and the padding row stay as they
+    were; each used slot's conv history is the raw history shifted by the new token."""
+    from gated_deltanet_token_b200 import gdn
+
+    L = [70, 3, 1, 0, 130]
+    N = len(L)
+    full = make_inputs("varlen8_prefill_bf16", lengths=[n + 1 for n in L], h_qk=2, h_v=4, seed=3)
+    cf = full["cu_seqlens"]
+    head = dict(full)
+    for nm in ("q", "k", "v", "z", "a", "b"):
+        head[nm] = np.ascontiguousarray(np.concatenate([full[nm][cf[n]:cf[n] + L[n]] for n in range(N)]))
+    ch = np.zeros(N + 1, np.int32)
+    ch[1:] = np.cumsum(L)
+    head["cu_seqlens"] = ch
+    d = {nm: to_dev(head[nm]) for nm in ("q", "k", "v", "z", "a", "b")}
+    par = {nm: to_dev(full[nm]) for nm in ("A_log", "dt_bias", "conv_w", "norm_w")}
+    cu_d = to_dev(ch)
+    _, fs = gdn.gdn_prefill(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], par["A_log"], par["dt_bias"],
+                            par["conv_w"], par["norm_w"], to_dev(full["init_state"]), cu_d,
+                            out_dtype=torch.float32)
+    cs = gdn.gdn_prefill_conv_state(d["q"], d["k"], d["v"], cu_d)
+
+    n_slots, perm = N + 2, [4, 0, 6, 2, 1]
+    g = torch.Generator(device="cuda").manual_seed(7)
+    state_pool = torch.randn((n_slots,) + tuple(fs.shape[1:]), generator=g, device="cuda")
+    conv_pool = torch.randn((n_slots,) + tuple(cs.shape[1:]), generator=g, device="cuda").to(cs.dtype)
+    for n, sl in enumerate(perm):
+        state_pool[sl].copy_(fs[n])
+        conv_pool[sl].copy_(cs[n])
+    spare = [s for s in range(n_slots) if s not in perm]
+    spare_state, spare_conv = state_pool[spare].clone(), conv_pool[spare].clone()
+
+    last = [int(cf[n + 1]) - 1 for n in range(N)] + [int(cf[1]) - 1]  # + one padding entry
+    dec = {nm: to_dev(np.ascontiguousarray(full[nm][last])) for nm in ("q", "k", "v", "z", "a", "b")}
+    ids = to_dev(np.array(perm + [-1], np.int32))
+    y = torch.full((N + 1, 4, 128), float("nan"), device="cuda")
+    gdn.gdn_decode_slots(dec["q"], dec["k"], dec["v"], dec["z"], dec["a"], dec["b"], par["A_log"],
+                         par["dt_bias"], par["conv_w"], par["norm_w"], conv_pool, state_pool, ids,
+                         out_dtype=torch.float32, y=y)
+    torch.cuda.synchronize()
+    assert gdn.gdn_read_device_status() == 0
+
+    ref = oracle_mod.prefill(full)
+    yy = y.cpu().numpy().astype(np.float64)
+    S = state_pool.cpu().numpy().astype(np.float64)
+    check_bf16(yy[:N], ref["y"][last[:N]], S[perm], ref["final_state"])
+    assert np.isnan(yy[N]).all()  # the padding entry wrote nothing
+    assert torch.equal(state_pool[spare], spare_state) and torch.equal(conv_pool[spare], spare_conv)
+    got = _as_np(conv_pool)
+    for n, sl in enumerate(perm):  # the history now ends with the decoded token, bit-exact
+        assert np.array_equal(got[sl], _raw_history(full, int(cf[n]), int(cf[n + 1])))
+
+
+def test_decode_slot_past_the_pool_sets_the_index_status():
+    from gated_deltanet_token_b200 import gdn
+
+    inp = make_inputs("decode_N256_bf16", n_seqs=2, h_qk=2, h_v=4)
+    dd = {nm: to_dev(inp[nm]) for nm in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w",
+                                          "norm_w", "conv_state", "state")}
+    ref_state, ref_conv = dd["state"].clone(), dd["conv_state"].clone()
+    y_ref = gdn.gdn_decode(dd["q"], dd["k"], dd["v"], dd["z"], dd["a"], dd["b"], dd["A_log"], dd["dt_bias"],
+                           dd["conv_w"], dd["norm_w"], ref_conv, ref_state, out_dtype=torch.float32)
+    y = torch.full((2, 4, 128), float("nan"), device="cuda")
+    gdn.gdn_decode_slots(dd["q"], dd["k"], dd["v"], dd["z"], dd["a"], dd["b"], dd["A_log"], dd["dt_bias"],
+                         dd["conv_w"], dd["norm_w"], dd["conv_state"], dd["state"],
+                         to_dev(np.array([0, 2], np.int32)), out_dtype=torch.float32, y=y)
+    assert gdn.gdn_read_device_status() == gdn.GDN_ERR_INDEX
+    assert gdn.gdn_read_device_status() == 0  # read clears it
+    assert torch.equal(y[0], y_ref[0]) and torch.isnan(y[1]).all()
+    assert torch.equal(dd["state"][0], ref_state[0])  # entry 0 ran; slot 1 was left alone
+    assert torch.equal(dd["state"][1], torch.from_numpy(inp["state"][1]).cuda())
