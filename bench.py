@@ -427,6 +427,28 @@ def gpu_arm(args):
     torch.cuda.synchronize()
     barrier()
     dms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
+    # the same step through the pool-slot call: the 256 states as a pool, slots in reverse order
+    slot_ids = torch.arange(255, -1, -1, dtype=torch.int32, device=dev)
+
+    def dstep_slots():
+        gdn.gdn_decode_slots(dd["q"], dd["k"], dd["v"], dd["z"], dd["a"], dd["b"], dd["A_log"], dd["dt_bias"],
+                             dd["conv_w"], dd["norm_w"], dd["conv_state"], dd["state"], slot_ids,
+                             out_dtype=torch.bfloat16, y=yd)
+
+    try:
+        for _ in range(3):
+            dstep_slots()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(dsteps):
+            dstep_slots()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        slots_ms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
+    except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
+        slots_ms = f"failed: {exc}"
     clk = clocks.stop()
     state_bytes = 256 * 32 * 128 * 128 * 4 * 2
     other = 256 * (2 * 16 * 128 * 2 + 2 * 32 * 128 * 2 + 2 * 32 * 4 + 32 * 128 * 2 + 2 * 3 * 8192 * 2)
@@ -434,7 +456,8 @@ def gpu_arm(args):
               "state_GBps": state_bytes / (dms / 1e3) / 1e9,
               "total_GBps": (state_bytes + other) / (dms / 1e3) / 1e9,
               "peak_GBps": hbm, "frac_state": state_bytes / (dms / 1e3) / 1e9 / hbm,
-              "tokens_per_s": 256 / (dms / 1e3), "traffic": ncu_traffic("decode")}
+              "tokens_per_s": 256 / (dms / 1e3), "traffic": ncu_traffic("decode"),
+              "slots_ms_per_step": slots_ms}
     del dd
 
     # --- end to end through the public call with host buffers ----------------------------------
