@@ -123,7 +123,9 @@ int gdn_decode(const gdn_dims_t* d, const void* q, const void* k, const void* v,
 
 /*
  * Prefill -> decode hand-off, part 1: the decode conv history each sequence has after a
- * prefill over the same packed inputs.  Writes, per sequence n, the raw (pre-conv) q | k | v
+ * prefill over the same packed inputs.  The width-4 causal conv of step 1 ("Qwen3.8-Flash-Next"
+ * technical report, Fig. 2) needs the three raw rows before each new token; the decode step
+ * keeps them beside the fixed-size state (field guide, §02).  Writes, per sequence n, the raw (pre-conv) q | k | v
  * channels of its last three tokens: conv_state[n][r] = x_{te-3+r}, te = cu_seqlens[n+1], in
  * gdn_decode's conv_state layout.  Rows before the sequence's first token are zeros (every
  * prefill sequence starts with a zero conv history), so a sequence of fewer than three tokens
@@ -142,7 +144,8 @@ int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, co
 
 /*
  * Prefill -> decode hand-off, part 2: gdn_decode on resident pools, the way a serving loop
- * keeps one state and one conv history per live request.  Same arguments and results as
+ * keeps one state and one conv history per live request (field guide, §02: the state stays
+ * the same size however long the sequence grows, so it can live in a fixed slot).  Same arguments and results as
  * gdn_decode, except that sequence n reads and updates pool slot slot_ids[n]:
  *
  *   conv_state_pool [n_slots][3][C_conv]       in_dtype, in/out

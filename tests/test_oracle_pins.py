@@ -336,6 +336,35 @@ def test_I9_decode_continues_prefill(oracle_mod, dtype):
     assert np.array_equal(o["conv_state"][0], _f64(expect))
 
 
+@pytest.mark.parametrize("T", [2, 9])
+def test_decode_steps_continue_prefill(oracle_mod, T):
+    """K = 5 decode steps in a row, from prefill(T)'s final state and conv history (zeros
+    before the first token when T < 3), equal the last K tokens and the final state of
+    prefill(T + K): the decode step composes with itself as the recurrence does."""
+    K = 5
+    full = make_inputs("tiny_prefill_fp32", T=T + K)
+    head = dict(full)
+    for n in ("q", "k", "v", "z", "a", "b"):
+        head[n] = full[n][:T]
+    pre = oracle_mod.prefill(full)
+    state = oracle_mod.prefill(head)["final_state"].astype(np.float32)
+    width = 2 * full["q"].shape[1] * full["q"].shape[2] + full["v"].shape[1] * full["v"].shape[2]
+    hist = np.zeros((1, 3, width), np.float32)
+    for r in range(3):
+        t = T - 3 + r
+        if t >= 0:
+            hist[0, r] = np.concatenate([full["q"][t].ravel(), full["k"][t].ravel(), full["v"][t].ravel()])
+    for i in range(K):
+        dec = dict(full)
+        for n in ("q", "k", "v", "z", "a", "b"):
+            dec[n] = full[n][T + i:T + i + 1]
+        dec["state"], dec["conv_state"] = state, hist
+        o = oracle_mod.decode(dec)
+        assert np.abs(o["y"][0] - pre["y"][T + i]).max() < 1e-5
+        state, hist = o["state"].astype(np.float32), o["conv_state"].astype(np.float32)
+    assert rel(o["state"][0], pre["final_state"][0]) < 1e-5
+
+
 def test_decode_exact_state_roundtrip(oracle_mod):
     """With the state given exactly in fp32, decode equals a one-token prefill whose
     conv history is the same raw values (both in fp64)."""
