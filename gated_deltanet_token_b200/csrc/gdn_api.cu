@@ -25,7 +25,7 @@ namespace {
 
 __device__ float g_selftest_out[2];
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0: the prefill-to-decode hand-off calls
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
