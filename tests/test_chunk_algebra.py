@@ -11,7 +11,11 @@ Two regroupings of the same update are checked as well: the state update through
 W2^T = K^T diag(D) T (no U = T R), and the whole chunk as one affine map of the state,
   S^T <- (e^{gamma_L} I - W2^T diag(beta e^gamma) K) S^T + W2^T diag(beta) V,
   y   = (diag(e^gamma) Q - P diag(beta e^gamma) K) S^T + P diag(beta) V,
-which leaves one product with the state per chunk on the sequential path."""
+which leaves one product with the state per chunk on the sequential path.  A fourth form
+software-pipelines the three-round chain: the next chunk's first product splits as
+  [K;Q]_{c+1} S_{c+1}^T = e^{gamma_L} [K;Q]_{c+1} S_c^T + X_{c+1} U~_c,
+  X_{c+1} = [K;Q]_{c+1} K_c^T,  U~_c = diag(D) T R,
+so its state part can run a chunk early, off the chain."""
 import numpy as np
 import pytest
 
@@ -42,6 +46,8 @@ def _chunk_terms(q, k, v, g, beta):
 def _run(q, k, v, g, beta, S0, C, form):
     S = S0.T.copy()  # S^T: [d_k, d_v]
     ys = []
+    if form == "pipelined":
+        return _run_pipelined(q, k, v, g, beta, S0, C)
     for c0 in range(0, len(g), C):
         sl = slice(c0, c0 + C)
         qc, kc, vc, gc, bc = q[sl], k[sl], v[sl], g[sl], beta[sl]
@@ -64,7 +70,33 @@ def _run(q, k, v, g, beta, S0, C, form):
     return np.concatenate(ys), S.T
 
 
-@pytest.mark.parametrize("form", ["three_rounds", "w2", "affine"])
+def _run_pipelined(q, k, v, g, beta, S0, C):
+    """Three rounds, with [K S^T ; Q S^T] of each chunk after the first formed from the previous
+    chunk's state and its U~ only: e^{gamma_L} (early product) + X U~."""
+    S = S0.T.copy()
+    ys = []
+    carry = None  # (e^{gamma_L} [K;Q]_{c} S_{c-1}^T, X_c U~_{c-1}) for the next chunk
+    starts = list(range(0, len(g), C))
+    for ci, c0 in enumerate(starts):
+        sl = slice(c0, c0 + C)
+        qc, kc, vc, gc, bc = q[sl], k[sl], v[sl], g[sl], beta[sl]
+        gam, T, P, D = _chunk_terms(qc, kc, vc, gc, bc)
+        eg, eL = np.exp(gam), np.exp(gam[-1])
+        KQ = np.concatenate([kc, qc])
+        first = KQ @ S if carry is None else carry[0] + carry[1]
+        KS, QS = first[:len(gc)], first[len(gc):]
+        R = bc[:, None] * (vc - eg[:, None] * KS)
+        ys.append(eg[:, None] * QS + P @ R)
+        Ut = D[:, None] * (T @ R)
+        if ci + 1 < len(starts):
+            nsl = slice(starts[ci + 1], starts[ci + 1] + C)
+            KQn = np.concatenate([k[nsl], q[nsl]])
+            carry = (eL * (KQn @ S), (KQn @ kc.T) @ Ut)  # early product; X_{c+1} U~_c
+        S = eL * S + kc.T @ Ut
+    return np.concatenate(ys), S.T
+
+
+@pytest.mark.parametrize("form", ["three_rounds", "w2", "affine", "pipelined"])
 @pytest.mark.parametrize("T,C", [(1, 64), (63, 64), (64, 64), (65, 64), (200, 64), (37, 16)])
 def test_chunk_forms_equal_token_form(oracle_mod, form, T, C):
     rng = np.random.default_rng(7 + T + C)
