@@ -15,6 +15,7 @@
 #include "gdn.h"
 #include "gdn_common.cuh"
 #include "k_chunk_simt.cuh"
+#include "k_chunk_pipe.cuh"
 #include "k_chunk_tc.cuh"
 #include "k_decode.cuh"
 #include "k_stream.cuh"
@@ -46,7 +47,7 @@ bool use_tc(const gdn_dims_t* d) {
 // Workspace of the prefill, carved from the caller's buffer in this order.
 struct WsLayout {
   size_t tab, seqc0, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
-  size_t kq, tp, gb, vs;  // tensor-core path
+  size_t kq, tp, xt, gb, vs;  // tensor-core path
   int max_chunks;
   bool tc;
 };
@@ -68,6 +69,7 @@ WsLayout ws_layout_tc(const gdn_dims_t* d) {
   L.seqc0 = take((N + 1) * sizeof(int));
   L.kq = take(MC * hq * KQ_BYTES);
   L.tp = take(MC * hv * TP_BYTES);
+  L.xt = take(MC * hq * XT_BYTES);
   L.gb = take(MC * hv * GB_FLOATS * 4);
   L.vs = take(MC * hv * VS_BYTES);
   L.yraw = take(T * hv * D * 4);
@@ -255,7 +257,13 @@ int configure_device() {
       cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)PB_TC_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)PB_TC_SMEM) != cudaSuccess)
+                           (int)PB_TC_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkscan_pipe<PB_Y_RAW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)PP_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkscan_pipe<PB_Y_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)PP_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_chunkscan_pipe<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)PP_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   done_mask.fetch_or(bit);
   return GDN_OK;
@@ -375,6 +383,7 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     const int* seqc0c = need_map ? seqc0 : nullptr;
     uint8_t* kq = reinterpret_cast<uint8_t*>(ws + L.kq);
     uint8_t* tp = reinterpret_cast<uint8_t*>(ws + L.tp);
+    uint8_t* xt = reinterpret_cast<uint8_t*>(ws + L.xt);
     if (d->total_tokens > 0) {
       {
         ProfScope p("prologue_tc", s);
@@ -392,7 +401,7 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
       }
       ProfScope p("chunk_prep_tc", s);
       if (launch_dep(k_chunkprep_tc, dim3(d->h_qk, L.max_chunks), dim3(256), PA_TC_SMEM, s, 1, kd, tabc, a, b, A_log,
-                     dt_bias, (const uint8_t*)kq, tp, F(L.gb)) != cudaSuccess)
+                     dt_bias, (const uint8_t*)kq, tp, xt, F(L.gb)) != cudaSuccess)
         return GDN_ERR_CUDA;
     }
     // The output norm runs inside phase B (clusters of the four slices of a head) unless that
@@ -403,23 +412,36 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     const long waves_plain = (units * (D / TC_NV) + g_num_sms - 1) / g_num_sms;
     const bool fused = per_wave > 0 && waves_fused <= waves_plain && getenv_flag("GDN_NO_FUSED_NORM") == 0;
     const dim3 grid(d->n_seqs, d->h_v, D / TC_NV);
+    // phase B with the software-pipelined chain, unless GDN_PB_PIPE=0 asks for the three-round one
+    const bool pipe = getenv("GDN_PB_PIPE") == nullptr || getenv_flag("GDN_PB_PIPE") == 1;
     if (fused) {
       ProfScope p("chunk_scan_tc_norm", s);
       const uint16_t* zb = static_cast<const uint16_t*>(z);
-      cudaError_t e = launch_dep(kd.out_bf16 ? k_chunkscan_tc<PB_Y_BF16> : k_chunkscan_tc<PB_Y_F32>, grid, dim3(384),
-                                 PB_TC_SMEM, s, D / TC_NV, kd, (const int*)cu_seqlens, seqc0c, (const uint8_t*)kq,
-                                 (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs), init_state,
-                                 F(L.yraw), final_state, zb, norm_w, y);
+      cudaError_t e = pipe ? launch_dep(kd.out_bf16 ? k_chunkscan_pipe<PB_Y_BF16> : k_chunkscan_pipe<PB_Y_F32>, grid,
+                                        dim3(384), PP_SMEM, s, D / TC_NV, kd, (const int*)cu_seqlens, seqc0c,
+                                        (const uint8_t*)kq, (const uint8_t*)tp, (const uint8_t*)xt,
+                                        (const float*)F(L.gb), (const float*)F(L.vs), init_state, F(L.yraw),
+                                        final_state, zb, norm_w, y)
+                           : launch_dep(kd.out_bf16 ? k_chunkscan_tc<PB_Y_BF16> : k_chunkscan_tc<PB_Y_F32>, grid,
+                                        dim3(384), PB_TC_SMEM, s, D / TC_NV, kd, (const int*)cu_seqlens, seqc0c,
+                                        (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb),
+                                        (const float*)F(L.vs), init_state, F(L.yraw), final_state, zb, norm_w, y);
       if (e != cudaSuccess) return GDN_ERR_CUDA;
       return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
     }
     {
       ProfScope p("chunk_scan_tc", s);
-      if (launch_dep(k_chunkscan_tc<PB_Y_RAW>, grid, dim3(288), PB_TC_SMEM, s, 1, kd, (const int*)cu_seqlens, seqc0c,
-                     (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
-                     init_state, F(L.yraw), final_state, (const uint16_t*)nullptr, (const float*)nullptr,
-                     (void*)nullptr) != cudaSuccess)
-        return GDN_ERR_CUDA;
+      cudaError_t e = pipe ? launch_dep(k_chunkscan_pipe<PB_Y_RAW>, grid, dim3(320), PP_SMEM, s, 1, kd,
+                                        (const int*)cu_seqlens, seqc0c, (const uint8_t*)kq, (const uint8_t*)tp,
+                                        (const uint8_t*)xt, (const float*)F(L.gb), (const float*)F(L.vs), init_state,
+                                        F(L.yraw), final_state, (const uint16_t*)nullptr, (const float*)nullptr,
+                                        (void*)nullptr)
+                           : launch_dep(k_chunkscan_tc<PB_Y_RAW>, grid, dim3(288), PB_TC_SMEM, s, 1, kd,
+                                        (const int*)cu_seqlens, seqc0c, (const uint8_t*)kq, (const uint8_t*)tp,
+                                        (const float*)F(L.gb), (const float*)F(L.vs), init_state, F(L.yraw),
+                                        final_state, (const uint16_t*)nullptr, (const float*)nullptr,
+                                        (void*)nullptr);
+      if (e != cudaSuccess) return GDN_ERR_CUDA;
     }
     if (d->total_tokens > 0) {
       ProfScope p("epilogue", s);

@@ -39,6 +39,7 @@ constexpr uint32_t KQ_TILE = 128 * 128 * 2;          // one bf16 tile of [K;Q] (
 constexpr uint32_t KQ_BYTES = 2 * KQ_TILE;           // per (chunk, QK head)
 constexpr uint32_t TP_TILE = 128 * 64 * 2;           // one bf16 tile of [T;P]: 16 KB
 constexpr uint32_t TP_BYTES = 2 * TP_TILE;           // per (chunk, value head)
+constexpr uint32_t XT_BYTES = 2 * TP_TILE;           // X = [K;Q]_c K_{c-1}^T (128 x 64) hi | lo, per (chunk, QK head)
 constexpr uint32_t GB_FLOATS = 128;                  // gamma[64], beta[64] per (chunk, value head)
 constexpr uint32_t VS_SLICE = 64 * TC_NV * 4;        // v after conv + SiLU (fp32), one 32-column slice: 8 KB
 constexpr uint32_t VS_BYTES = 4 * VS_SLICE;          // per (chunk, value head)
@@ -467,7 +468,7 @@ __global__ void __launch_bounds__(256, 2)
     k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
-                   uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
+                   uint8_t* __restrict__ tp_ws, uint8_t* __restrict__ xt_ws, float* __restrict__ gb_ws) {
   tc::grid_dep_wait();  // the prologue's tiles are complete
   tc::grid_dep_launch_dependents();
   // head-fastest grid, chunks from the last: the prologue writes its tiles in chunk order, so
@@ -500,17 +501,27 @@ __global__ void __launch_bounds__(256, 2)
     tc::fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // cols 0..63: [K;Q]K^T, 128..255: P pair
+    tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // cols 0..63: [K;Q]K^T, 64..127: X, 128..255: P pair
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
+  // X = [K;Q] K_prev^T needs the K rows of the sequence's previous chunk (the chunk slots of a
+  // sequence are consecutive); its first chunk has none
+  const bool has_prev = e.t0 > e.seq_start;
   if (tid == 0) {  // the [K;Q] tile written by the prologue
     const uint32_t bar = tc::smem_u32(&mbar);
-    tc::mbar_arrive_expect_tx(bar, KQ_BYTES);
+    tc::mbar_arrive_expect_tx(bar, KQ_BYTES + (has_prev ? KQ_TILE : 0u));
     tc::bulk_g2s(tc::smem_u32(sm), kq_ws + ((size_t)chunk * hq + j) * KQ_BYTES, KQ_BYTES, bar);
+    if (has_prev) {  // its K rows (hi, lo), 1 KB per key group, into the T matrices' space
+      const uint8_t* src = kq_ws + ((size_t)(chunk - 1) * hq + j) * KQ_BYTES;
+      for (int kk = 0; kk < 16; ++kk) {
+        tc::bulk_g2s(tc::smem_u32(sm + PA_OFF_T + kk * 1024), src + kk * LBO128, 1024, bar);
+        tc::bulk_g2s(tc::smem_u32(sm + PA_OFF_T + 16384 + kk * 1024), src + KQ_TILE + kk * LBO128, 1024, bar);
+      }
+    }
   }
   uint32_t mma_phase = 0;
   bool aborted = false;
@@ -558,6 +569,16 @@ __global__ void __launch_bounds__(256, 2)
             const uint64_t o = (uint64_t)((ks * 2 * LBO128) >> 4);
             tc::umma_bf16(tbase, dd[term == 2] + o, dd[term == 1] + o, idesc, (ks | term) != 0);
           }
+        if (has_prev) {  // X = [K;Q] K_prev^T (128 x 64) into TMEM columns 64..127
+          const uint64_t dp[2] = {tc::sdesc(tc::smem_u32(sm + PA_OFF_T), 1024, 128),
+                                  tc::sdesc(tc::smem_u32(sm + PA_OFF_T + 16384), 1024, 128)};
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int term = 0; term < 3; ++term)
+              tc::umma_bf16(tbase + 64, dd[term == 2] + (uint64_t)((ks * 2 * LBO128) >> 4),
+                            dp[term == 1] + (uint64_t)((ks * 2 * 1024) >> 4), idesc, (ks | term) != 0);
+        }
         tc::umma_commit(tc::smem_u32(&mbar));
       }
       if (!s_abort && !tc::mbar_wait(tc::smem_u32(&mbar), 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
@@ -566,6 +587,23 @@ __global__ void __launch_bounds__(256, 2)
     __syncthreads();
     aborted = s_abort != 0;
     if (aborted) break;
+    if (ga == 0 && has_prev) {  // X to the workspace: warp w, rows 32 (w % 4) + lane, columns 32 (w / 4) ..
+      const int q4 = warp & 3, c0 = (warp >> 2) * 32, r = q4 * 32 + lane;
+      uint32_t x[32];
+      tc::tmem_ld32(tbase + 64 + ((uint32_t)(q4 * 32) << 16) + c0, x);
+      tc::tmem_wait_ld();
+      uint8_t* out = xt_ws + ((size_t)chunk * hq + j) * XT_BYTES;
+#pragma unroll
+      for (int s8 = 0; s8 < 32; s8 += 8) {
+        float xv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xv[c] = __uint_as_float(x[s8 + c]);
+        uint4 hi, lo;
+        tc::split8(xv, hi, lo);
+        *reinterpret_cast<uint4*>(out + kmaj128(r, c0 + s8)) = hi;
+        *reinterpret_cast<uint4*>(out + TP_TILE + kmaj128(r, c0 + s8)) = lo;
+      }
+    }
     // A (fp32) of both heads and the Mq rows of the P operand, straight from the [K;Q]K^T
     // accumulator: warp w reads TMEM lanes 32 (w % 4).. (rows 0..63 K K^T, 64..127 Q K^T),
     // columns 32 (w / 4) .. + 31.
