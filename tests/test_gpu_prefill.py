@@ -254,3 +254,20 @@ def test_back_to_back_calls_chain_the_state(oracle_mod):
         check_bf16(y.float().cpu().numpy().astype(np.float64), ref["y"], ref["final_state"], ref["final_state"])
     check_bf16(ys[-1].float().cpu().numpy().astype(np.float64), ref["y"], state.cpu().numpy().astype(np.float64),
                ref["final_state"])
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_pipelined_phase_b_matches_three_rounds(oracle_mod, monkeypatch, fused):
+    """The software-pipelined phase B (default) and the three-round one (GDN_PB_PIPE=0) agree,
+    and both meet the oracle, on varlen sequences whose lengths cross chunk boundaries."""
+    if not fused:
+        monkeypatch.setenv("GDN_NO_FUSED_NORM", "1")
+    inp = make_inputs("varlen8_prefill_bf16", lengths=[1, 64, 65, 130, 200, 0, 3], h_qk=4, h_v=8)
+    ref = _oracle(oracle_mod, inp)
+    y_p, S_p = run_prefill(inp, torch.float32)
+    monkeypatch.setenv("GDN_PB_PIPE", "0")
+    y_3, S_3 = run_prefill(inp, torch.float32)
+    check_bf16(y_p, ref["y"], S_p, ref["final_state"])
+    check_bf16(y_3, ref["y"], S_3, ref["final_state"])
+    assert np.abs(y_p - y_3).max() <= 1e-3 * max(1.0, np.abs(y_3).max())
+    assert np.linalg.norm(S_p - S_3) <= 1e-4 * np.linalg.norm(S_3)
