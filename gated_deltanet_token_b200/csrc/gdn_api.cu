@@ -18,6 +18,7 @@
 #include "k_chunk_pipe.cuh"
 #include "k_chunk_tc.cuh"
 #include "k_decode.cuh"
+#include "k_decode_multi.cuh"
 #include "k_stream.cuh"
 
 using namespace gdn;
@@ -263,7 +264,15 @@ int configure_device() {
       cudaFuncSetAttribute(k_chunkscan_pipe<PB_Y_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)PP_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_chunkscan_pipe<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)PP_SMEM) != cudaSuccess)
+                           (int)PP_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   done_mask.fetch_or(bit);
   return GDN_OK;
@@ -525,6 +534,44 @@ int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const vo
   if (n_slots < 1) return GDN_ERR_SHAPE;
   return decode_impl(d, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state_pool, state_pool, y,
                      slot_ids, n_slots, stream);
+}
+
+int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const void* k, const void* v,
+                     const void* z, const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+                     gdn_stream_t stream) {
+  if (!d) return GDN_ERR_NULL;
+  if (n_tokens < 1 || n_tokens > DECM_KMAX) return GDN_ERR_SHAPE;
+  if ((int64_t)d->n_seqs * n_tokens != (int64_t)d->total_tokens) return GDN_ERR_SHAPE;
+  gdn_dims_t d1 = *d;
+  d1.total_tokens = d->n_seqs;  // one entry per sequence, n_tokens tokens each
+  int rc = check_dims(&d1, true);
+  if (rc != GDN_OK) return rc;
+  const void* ptrs[] = {q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y};
+  for (const void* p : ptrs)
+    if (!p) return GDN_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  if (d->h_qk > 65535) return GDN_ERR_SHAPE;
+  rc = configure_device();
+  if (rc != GDN_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Dims kd = kdims(&d1);
+  const dim3 grid(d->n_seqs, d->h_qk);
+  ProfScope p("decode_multi", s);
+  if (kd.in_bf16 && kd.out_bf16)
+    k_decode_multi<true, true><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                           norm_w, conv_state, state, y);
+  else if (kd.in_bf16)
+    k_decode_multi<true, false><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                            norm_w, conv_state, state, y);
+  else if (kd.out_bf16)
+    k_decode_multi<false, true><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                            norm_w, conv_state, state, y);
+  else
+    k_decode_multi<false, false><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias,
+                                                             conv_w, norm_w, conv_state, state, y);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, const void* v,

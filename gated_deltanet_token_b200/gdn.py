@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode.argtypes = [dp] + [vp] * 13 + [vp]
         L.gdn_decode_slots.restype = ctypes.c_int
         L.gdn_decode_slots.argtypes = [dp] + [vp] * 12 + [ctypes.c_int32, vp, vp, vp]
+        L.gdn_decode_multi.restype = ctypes.c_int
+        L.gdn_decode_multi.argtypes = [dp, ctypes.c_int32] + [vp] * 13 + [vp]
         L.gdn_prefill_conv_state.restype = ctypes.c_int
         L.gdn_prefill_conv_state.argtypes = [dp] + [vp] * 5 + [vp]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -273,4 +275,25 @@ def gdn_decode_slots(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_stat
                                 _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_slots")
+    return y
+
+
+def gdn_decode_multi(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, *,
+                     out_dtype=None, y=None, q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6, stream=None):
+    """n_tokens decode steps per sequence in one call: q, k [N, n_tokens, h_qk, 128]; v, z
+    [N, n_tokens, h_v, 128]; a, b [N, n_tokens, h_v].  conv_state [N, 3, C_conv] and state
+    [N, h_v, 128, 128] are updated in place.  Returns y [N, n_tokens, h_v, 128]."""
+    N, K, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[2], v.shape[3]
+    if out_dtype is None:
+        out_dtype = q.dtype
+    dims = make_dims(N, N * K, h_qk, h_v, _dt(q), _dt(torch.empty(0, dtype=out_dtype)), d_k, d_v, q_scale,
+                     l2_eps, rms_eps)
+    if y is None:
+        y = torch.empty((N, K, h_v, d_v), dtype=out_dtype, device=q.device)
+    rc = lib().gdn_decode_multi(ctypes.byref(dims), ctypes.c_int32(K), _ptr(q), _ptr(k), _ptr(v), _ptr(z),
+                                _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(conv_w), _ptr(norm_w),
+                                _ptr(conv_state), _ptr(state), _ptr(y), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_multi")
     return y

@@ -163,6 +163,26 @@ int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const vo
                      const float* conv_w, const float* norm_w, void* conv_state_pool, float* state_pool,
                      int32_t n_slots, const int32_t* slot_ids, void* y, gdn_stream_t stream);
 
+/*
+ * Several decode tokens per sequence in one call (1 <= n_tokens <= 8), e.g. to verify drafted
+ * tokens: the same per-token rule as gdn_decode (field guide, §02, steps 1-6, then the gated
+ * RMSNorm) applied to n_tokens consecutive tokens of each sequence, reading and writing each
+ * state row once per call instead of once per token.
+ *
+ *   q, k        [N][n_tokens][h_qk][d_k]   in_dtype
+ *   v, z        [N][n_tokens][h_v][d_v]    in_dtype
+ *   a, b        [N][n_tokens][h_v]         fp32
+ *   conv_state  [N][3][C_conv]             in/out: replaced by the last three raw rows
+ *   state       [N][h_v][d_v][d_k]         fp32, in/out: the state after the last token
+ *   y           [N][n_tokens][h_v][d_v]    out_dtype (written)
+ * d->total_tokens must equal d->n_seqs * n_tokens.  Returns GDN_ERR_SHAPE for n_tokens
+ * outside 1..8, otherwise what gdn_decode returns.
+ */
+int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const void* k, const void* v,
+                     const void* z, const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+                     gdn_stream_t stream);
+
 /* Static, NUL-terminated name of a return code ("GDN_OK", "GDN_ERR_SHAPE", ...). */
 const char* gdn_status_string(int code);
 

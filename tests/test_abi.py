@@ -132,6 +132,26 @@ def test_handoff_calls_reject_bad_arguments(glib):
     assert slots(four, pool=FAKE + 8) == -4
 
 
+def test_decode_multi_rejects_bad_arguments(glib):
+    L = glib.lib()
+
+    def call(dims, K, ptrs=None):
+        p = [FAKE] * 13 if ptrs is None else ptrs
+        return L.gdn_decode_multi(None if dims is None else ctypes.byref(dims), ctypes.c_int32(K),
+                                  *[ctypes.c_void_p(x) if x else None for x in p], None)
+
+    assert call(None, 2) == -1
+    assert call(glib.make_dims(4, 8, 16, 32, 1, 1), 0) == -2
+    assert call(glib.make_dims(4, 36, 16, 32, 1, 1), 9) == -2  # more than 8 tokens
+    assert call(glib.make_dims(4, 7, 16, 32, 1, 1), 2) == -2   # total_tokens != n_seqs * n_tokens
+    bad = [FAKE] * 13
+    bad[11] = None
+    assert call(glib.make_dims(4, 8, 16, 32, 1, 1), 2, bad) == -1
+    bad = [FAKE] * 13
+    bad[0] = FAKE + 2
+    assert call(glib.make_dims(4, 8, 16, 32, 1, 1), 2, bad) == -4
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     from gated_deltanet_token_b200 import gdn
 
