@@ -449,6 +449,35 @@ def gpu_arm(args):
         slots_ms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         slots_ms = f"failed: {exc}"
+    # four decode tokens per sequence in one call (each state row read and written once)
+    multi = None
+    try:
+        K4 = 4
+        per_tok = [make_inputs(DECODE_WORKLOAD, seed=rank + 100 + i) for i in range(K4)]
+        dm = {nm: to_dev(np.ascontiguousarray(np.stack([p_[nm] for p_ in per_tok], axis=1)), dev)
+              for nm in ("q", "k", "v", "z", "a", "b")}
+        del per_tok
+        ym = torch.empty((256, K4, 32, 128), dtype=torch.bfloat16, device=dev)
+
+        def dstep_multi():
+            gdn.gdn_decode_multi(dm["q"], dm["k"], dm["v"], dm["z"], dm["a"], dm["b"], dd["A_log"], dd["dt_bias"],
+                                 dd["conv_w"], dd["norm_w"], dd["conv_state"], dd["state"],
+                                 out_dtype=torch.bfloat16, y=ym)
+
+        for _ in range(3):
+            dstep_multi()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(dsteps):
+            dstep_multi()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        mms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
+        multi = {"tokens_per_sequence": K4, "ms_per_call": mms, "tokens_per_s": 256 * K4 / (mms / 1e3)}
+    except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
+        multi = f"failed: {exc}"
     clk = clocks.stop()
     state_bytes = 256 * 32 * 128 * 128 * 4 * 2
     other = 256 * (2 * 16 * 128 * 2 + 2 * 32 * 128 * 2 + 2 * 32 * 4 + 32 * 128 * 2 + 2 * 3 * 8192 * 2)
@@ -457,7 +486,7 @@ def gpu_arm(args):
               "total_GBps": (state_bytes + other) / (dms / 1e3) / 1e9,
               "peak_GBps": hbm, "frac_state": state_bytes / (dms / 1e3) / 1e9 / hbm,
               "tokens_per_s": 256 / (dms / 1e3), "traffic": ncu_traffic("decode"),
-              "slots_ms_per_step": slots_ms}
+              "slots_ms_per_step": slots_ms, "multi_token": multi}
     del dd
 
     # --- end to end through the public call with host buffers ----------------------------------
