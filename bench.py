@@ -179,6 +179,7 @@ KERNEL_SOURCES = {
     "prologue_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "chunk_prep_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "chunk_scan_tc_norm": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
+    "decode_multi": ("k_decode_multi.cuh", "gdn_common.cuh"),
     "decode": ("k_decode.cuh", "gdn_common.cuh"),
     "chunk_phaseB_simt": ("k_chunk_simt.cuh", "gdn_common.cuh"),
 }
@@ -217,13 +218,26 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(target_s: float):
+def cpu_model() -> str:
+    """The host CPU's model name (first "model name" line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample(target_s: float, threads: int = 0):
     """Time the fp64 oracle on a prefix of the bench workload (all 32 value heads), sized
-    to take about target_s seconds.  Returns (tokens/s, tokens, seconds, threads)."""
+    to take about target_s seconds, on `threads` host threads (0: every core).  Returns
+    (tokens/s, tokens, seconds, threads)."""
     import oracle
     from gated_deltanet_token_b200.inputs import make_inputs
 
-    cores = cpu_cores()
+    cores = threads if threads > 0 else cpu_cores()
     full = make_inputs(WORKLOAD)
 
     def run(T):
@@ -243,6 +257,19 @@ def oracle_sample(target_s: float):
         dt += run(T)
         reps += 1
     return reps * T / dt, reps * T, dt, cores
+
+
+def sample_text(Ts: int, secs: float) -> str:
+    return (f"the T=4096 workload, all 32 value heads, run {Ts // 4096} times, {secs:.1f} s" if Ts >= 4096
+            else f"first {Ts} tokens of the T=4096 workload, all 32 value heads, {secs:.1f} s")
+
+
+def bench_config(world: int, n_sets: int = 3) -> dict:
+    """The `config` of the bench line; the reference arm reports the same one."""
+    return {"workload": WORKLOAD, "B": 1, "T": 4096, "h_qk": 16, "h_v": 32, "d": 128, "chunk": 64,
+            "in_dtype": "bf16", "out_dtype": "bf16", "state_dtype": "f32",
+            "l2": f"{n_sets} rotating input sets of 97 MiB (> 126 MB L2)",
+            "parallelism": f"replicas x{world}"}
 
 
 def reference_arm(args):
@@ -274,15 +301,15 @@ def reference_arm(args):
     times = [step(T) for _ in range(args.steps)]
     total = sum(times)
     value = T * args.steps / total / 1e6
-    sample = f"first {T} of 4096 tokens, all 32 value heads, per step"
+    sample = (f"the whole T=4096 workload, all 32 value heads, per step" if T >= 4096
+              else f"first {T} of the 4096 tokens, all 32 value heads, per step")
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "B": 1, "T": 4096, "h_qk": 16, "h_v": 32,
-                                        "d": 128, "sample_tokens": T},
+        "data": "synthetic", "config": bench_config(world),
         "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
@@ -449,6 +476,35 @@ def gpu_arm(args):
         slots_ms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         slots_ms = f"failed: {exc}"
+    # four decode tokens per sequence in one call (each state row read and written once)
+    multi = None
+    try:
+        K4 = 4
+        per_tok = [make_inputs(DECODE_WORKLOAD, seed=rank + 100 + i) for i in range(K4)]
+        dm = {nm: to_dev(np.ascontiguousarray(np.stack([p_[nm] for p_ in per_tok], axis=1)), dev)
+              for nm in ("q", "k", "v", "z", "a", "b")}
+        del per_tok
+        ym = torch.empty((256, K4, 32, 128), dtype=torch.bfloat16, device=dev)
+
+        def dstep_multi():
+            gdn.gdn_decode_multi(dm["q"], dm["k"], dm["v"], dm["z"], dm["a"], dm["b"], dd["A_log"], dd["dt_bias"],
+                                 dd["conv_w"], dd["norm_w"], dd["conv_state"], dd["state"],
+                                 out_dtype=torch.bfloat16, y=ym)
+
+        for _ in range(3):
+            dstep_multi()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(dsteps):
+            dstep_multi()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        mms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
+        multi = {"tokens_per_sequence": K4, "ms_per_call": mms, "tokens_per_s": 256 * K4 / (mms / 1e3)}
+    except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
+        multi = f"failed: {exc}"
     clk = clocks.stop()
     state_bytes = 256 * 32 * 128 * 128 * 4 * 2
     other = 256 * (2 * 16 * 128 * 2 + 2 * 32 * 128 * 2 + 2 * 32 * 4 + 32 * 128 * 2 + 2 * 3 * 8192 * 2)
@@ -457,7 +513,7 @@ def gpu_arm(args):
               "total_GBps": (state_bytes + other) / (dms / 1e3) / 1e9,
               "peak_GBps": hbm, "frac_state": state_bytes / (dms / 1e3) / 1e9 / hbm,
               "tokens_per_s": 256 / (dms / 1e3), "traffic": ncu_traffic("decode"),
-              "slots_ms_per_step": slots_ms}
+              "slots_ms_per_step": slots_ms, "multi_token": multi}
     del dd
 
     # --- end to end through the public call with host buffers ----------------------------------
@@ -521,10 +577,10 @@ def gpu_arm(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, Ts, secs, cores = oracle_sample(12.0)
+        tps1, Ts1, secs1, _ = oracle_sample(8.0, threads=1)
         cpu = {"value": tps / 1e6, "unit": "Mtok/s", "cores": cores, "kind": "oracle",
-               "sample": (f"the T=4096 workload, all 32 value heads, run {Ts // 4096} times, {secs:.1f} s"
-                          if Ts >= 4096 else f"first {Ts} tokens of the T=4096 workload, all 32 value heads, "
-                          f"{secs:.1f} s")}
+               "sample": sample_text(Ts, secs), "cpu_model": cpu_model(),
+               "threads_1": {"value": tps1 / 1e6, "unit": "Mtok/s", "threads": 1, "sample": sample_text(Ts1, secs1)}}
 
     if world > 1:
         dist.destroy_process_group()
@@ -534,10 +590,7 @@ def gpu_arm(args):
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16x3/f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": 1, "T": T, "h_qk": 16, "h_v": 32, "d": 128, "chunk": 64,
-                   "in_dtype": "bf16", "out_dtype": "bf16", "state_dtype": "f32",
-                   "l2": f"{n_sets} rotating input sets of 97 MiB (> 126 MB L2)",
-                   "parallelism": f"replicas x{world}"},
+        "config": bench_config(world, n_sets),
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "pipeline": "3 streams, 2 slots", "matches_device": e2e_match},

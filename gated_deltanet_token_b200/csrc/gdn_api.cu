@@ -17,6 +17,7 @@
 #include "k_chunk_simt.cuh"
 #include "k_chunk_tc.cuh"
 #include "k_decode.cuh"
+#include "k_decode_multi.cuh"
 #include "k_stream.cuh"
 
 using namespace gdn;
@@ -29,18 +30,30 @@ constexpr int kVersion = 200;  // 0.2.0: the prefill-to-decode hand-off calls
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// The bf16-input prefill runs its chunk contractions on tcgen05 (bf16 hi/lo products); the
-// fp32-input prefill keeps true fp32 FFMA.  GDN_FORCE_SIMT=1 in the environment sends bf16
-// inputs down the fp32 path too, and GDN_NO_FUSED_NORM=1 keeps the output norm of the bf16
-// path in its own kernel (both for comparisons).
-int getenv_flag(const char* name) {
+// Path options (gdn_set_options).  The bf16-input prefill runs its chunk contractions on
+// tcgen05 (bf16 hi/lo products); the fp32-input prefill keeps true fp32 FFMA.  The options
+// select the slower alternatives for comparisons: bf16 inputs down the fp32 path, the output
+// norm of the bf16 path in its own kernel, and plain stream order between the prefill kernels.
+// Their initial value is read from the environment once per process (GDN_FORCE_SIMT=1,
+// GDN_NO_FUSED_NORM=1, GDN_NO_PDL=1); later calls only read the word.
+int env_flag(const char* name, const char* on) {
   const char* f = getenv(name);
-  return f && f[0] == '1' ? 1 : 0;
+  return f && strcmp(f, on) == 0 ? 1 : 0;
 }
+uint32_t options_from_env() {
+  return (env_flag("GDN_FORCE_SIMT", "1") ? GDN_OPT_FORCE_FP32_PATH : 0u) |
+         (env_flag("GDN_NO_FUSED_NORM", "1") ? GDN_OPT_SEPARATE_NORM : 0u) |
+         (env_flag("GDN_NO_PDL", "1") ? GDN_OPT_NO_PDL : 0u);
+}
+std::atomic<uint32_t>& options_word() {
+  static std::atomic<uint32_t> w{options_from_env()};
+  return w;
+}
+bool opt(uint32_t bit) { return (options_word().load(std::memory_order_relaxed) & bit) != 0; }
 
 bool use_tc(const gdn_dims_t* d) {
   if (d->in_dtype != GDN_DTYPE_BF16) return false;
-  return getenv_flag("GDN_FORCE_SIMT") == 0;
+  return !opt(GDN_OPT_FORCE_FP32_PATH);
 }
 
 // Workspace of the prefill, carved from the caller's buffer in this order.
@@ -134,8 +147,8 @@ struct ProfScope {
 
 // Launches a tensor-core prefill kernel with programmatic dependent launch: its CTAs may
 // become resident while the previous kernel on the stream drains, and wait in
-// griddepcontrol.wait (their first statement) until it has completed.  GDN_NO_PDL=1 gives plain
-// stream order.  cluster_z > 1 adds a (1, 1, cluster_z) cluster shape.
+// griddepcontrol.wait (their first statement) until it has completed, unless the options ask for plain
+// stream order (option GDN_OPT_NO_PDL).  cluster_z > 1 adds a (1, 1, cluster_z) cluster shape.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_z,
                        Args&&... args) {
@@ -146,7 +159,7 @@ cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   unsigned na = 0;
-  if (getenv_flag("GDN_NO_PDL") == 0) {
+  if (!opt(GDN_OPT_NO_PDL)) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
@@ -255,7 +268,15 @@ int configure_device() {
       cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)PB_TC_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)PB_TC_SMEM) != cudaSuccess)
+                           (int)PB_TC_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_decode_multi<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)DECM_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   done_mask.fetch_or(bit);
   return GDN_OK;
@@ -316,6 +337,10 @@ void launch_epilogue(const Dims& kd, const float* yraw, const void* z, const flo
 extern "C" {
 
 int gdn_version(void) { return kVersion; }
+
+uint32_t gdn_set_options(uint32_t flags) { return options_word().exchange(flags & GDN_OPT_ALL); }
+
+uint32_t gdn_get_options(void) { return options_word().load(); }
 
 const char* gdn_status_string(int code) {
   switch (code) {
@@ -401,7 +426,7 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     const int per_wave = scan_clusters_per_wave();
     const long waves_fused = per_wave > 0 ? (units + per_wave - 1) / per_wave : 0;
     const long waves_plain = (units * (D / TC_NV) + g_num_sms - 1) / g_num_sms;
-    const bool fused = per_wave > 0 && waves_fused <= waves_plain && getenv_flag("GDN_NO_FUSED_NORM") == 0;
+    const bool fused = per_wave > 0 && waves_fused <= waves_plain && !opt(GDN_OPT_SEPARATE_NORM);
     const dim3 grid(d->n_seqs, d->h_v, D / TC_NV);
     if (fused) {
       ProfScope p("chunk_scan_tc_norm", s);
@@ -505,6 +530,44 @@ int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const vo
                      slot_ids, n_slots, stream);
 }
 
+int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const void* k, const void* v,
+                     const void* z, const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+                     gdn_stream_t stream) {
+  if (!d) return GDN_ERR_NULL;
+  if (n_tokens < 1 || n_tokens > DECM_KMAX) return GDN_ERR_SHAPE;
+  if ((int64_t)d->n_seqs * n_tokens != (int64_t)d->total_tokens) return GDN_ERR_SHAPE;
+  gdn_dims_t d1 = *d;
+  d1.total_tokens = d->n_seqs;  // one entry per sequence, n_tokens tokens each
+  int rc = check_dims(&d1, true);
+  if (rc != GDN_OK) return rc;
+  const void* ptrs[] = {q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y};
+  for (const void* p : ptrs)
+    if (!p) return GDN_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  if (d->h_qk > 65535) return GDN_ERR_SHAPE;
+  rc = configure_device();
+  if (rc != GDN_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Dims kd = kdims(&d1);
+  const dim3 grid(d->n_seqs, d->h_qk);
+  ProfScope p("decode_multi", s);
+  if (kd.in_bf16 && kd.out_bf16)
+    k_decode_multi<true, true><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                           norm_w, conv_state, state, y);
+  else if (kd.in_bf16)
+    k_decode_multi<true, false><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                            norm_w, conv_state, state, y);
+  else if (kd.out_bf16)
+    k_decode_multi<false, true><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                            norm_w, conv_state, state, y);
+  else
+    k_decode_multi<false, false><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias,
+                                                             conv_w, norm_w, conv_state, state, y);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, const void* v,
                            const int32_t* cu_seqlens, void* conv_state, gdn_stream_t stream) {
   const int rc = check_dims(d, false);
@@ -602,6 +665,17 @@ int gdn_selftest_tc(int case_id, float* out2) {
     return GDN_ERR_CUDA;
   if (cudaMemcpyFromSymbol(out2, g_selftest_out, sizeof zero) != cudaSuccess) return GDN_ERR_CUDA;
   return GDN_OK;
+}
+
+int gdn_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) return GDN_ERR_SHAPE;
+  const unsigned long long v = ns;
+  return cudaMemcpyToSymbol(g_gdn_wait_ns, &v, sizeof v) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_selftest_wait_timeout(gdn_stream_t stream) {
+  k_selftest_wait_timeout<<<1, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 int gdn_read_device_status(gdn_stream_t stream) {

@@ -201,6 +201,36 @@ __global__ void __launch_bounds__(128) k_selftest_umma(float* out) {
 }
 
 // ======================================================================================
+// Diagnostic of the bounded waits (gdn_selftest_wait_timeout): one CTA holds tensor memory and
+// waits on an mbarrier that nothing completes -- no copy and no MMA is ever issued -- with the
+// same bounded wait the prefill kernels use.  The wait runs out, the timeout is recorded in the
+// device status word and the CTA frees its tensor memory and returns.
+// ======================================================================================
+__global__ void __launch_bounds__(128) k_selftest_wait_timeout() {
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tslot;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(tc::smem_u32(&mbar), 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tc::smem_u32(&tslot), 32);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = tslot;
+  // warp-uniform, as the prefill kernels take it ahead of their warp-collective TMEM loads
+  const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&mbar), 0));
+  if (!ok && threadIdx.x == 0) atomicExch(&g_gdn_status, -7);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, 32);
+}
+
+// ======================================================================================
 // Prologue of the tensor-core path.  Persistent: each CTA walks work items (head group,
 // half chunk) with a stride of the grid size.  A group is up to 8 heads of one stream -- q,
 // k or value heads -- whose slices of a token row are contiguous (2 KB).  The next item's
@@ -860,10 +890,28 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   auto named_bar_sync = [](int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
   };
-  // the chunk barrier: every warp but the norm warps
-  auto loop_sync = [&]() {
-    if (FUSED) named_bar_sync(2, 320);
-    else __syncthreads();
+  // the chunk barrier over every warp but the norm warps, returning the OR of `v` over them
+  auto loop_sync_or = [&](bool v) -> bool {
+    if (!FUSED) return __syncthreads_or(v) != 0;
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 2, 320, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+  };
+  // A bounded wait that records a timeout.  Once any thread has recorded one, later waits of
+  // the CTA return at once (the barriers they wait on may never complete) and no new MMA or
+  // copy is issued, so the CTA reaches its next chunk barrier, and leaves, within one limit.
+  auto aborted_now = [&]() { return *static_cast<volatile int*>(&s_abort) != 0; };
+  auto wait_ok = [&](uint64_t& bar, uint32_t parity) -> bool {
+    if (aborted_now()) return false;
+    if (tc::mbar_wait(tc::smem_u32(&bar), parity)) return true;
+    s_abort = 1;
+    atomicExch(&g_gdn_status, -7);
+    return false;
   };
   // (producer warp, lane 0) copies of chunk c into stage st
   auto issue_load = [&](int c, int st) {
@@ -901,7 +949,11 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   // accumulators (2 nv columns each: [a_hi b_hi + a_lo b_hi | a_hi b_lo])
   const uint32_t T_A = tbase, T_CD = tbase + 2 * NV, T_E = tbase + 4 * NV;
   const uint32_t t_a = T_A + lane_off + cb, t_cd = T_CD + lane_off + cb, t_e = T_E + lane_off + cb;
-  if (producer && lane == 0 && nchunks > 0) issue_load(0, 0);
+  int last_load = -1;  // (producer lane) the last chunk whose stage copies were issued
+  if (producer && lane == 0 && nchunks > 0) {
+    issue_load(0, 0);
+    last_load = 0;
+  }
   constexpr uint32_t idesc_kn2 = tc::idesc_bf16(128, 2 * NV, 0, 1);  // A K-major, B MN-major, N = 2 nv
   constexpr uint32_t idesc_kn = tc::idesc_bf16(128, NV, 0, 1);
   constexpr uint32_t idesc_mn2 = tc::idesc_bf16(128, 2 * NV, 1, 1);  // A and B MN-major
@@ -931,7 +983,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       uint64_t now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t_start == 0) t_start = now;
-      else if (now - t_start > 2000000000ull) return false;
+      else if (now - t_start > g_gdn_wait_ns) return false;
     }
     float tot = 0.0f;  // the same words in the same order in every slice: identical norms
 #pragma unroll
@@ -941,7 +993,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       const float inv = rsqrtf(tot * (1.0f / D) + d.rms_eps);
       const float4* nw4 = reinterpret_cast<const float4*>(norm_w + i0);
       const size_t base = ((size_t)y_tok * hv + h) * D + i0;
-      const uint4* zp = reinterpret_cast<const uint4*>(z + base);  // prefetched into L2 at round 2
+      const uint4* zp = reinterpret_cast<const uint4*>(z + base);
 #pragma unroll
       for (int g8 = 0; g8 < NV / 8; ++g8) {  // 8 columns at a time
         const uint4 zq = __ldg(zp + g8);
@@ -978,11 +1030,11 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       const int t0 = ts + c * CH, L = min(CH, te - t0);
       const float* gsm = reinterpret_cast<const float*>(stage[st] + PBStage::GB);
       // warp-uniform, so that the warp-collective TMEM loads run on every lane or none
-      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st]));
+      bool ok = __all_sync(0xffffffffu, wait_ok(mbar_ld[st], ph_ld[st]));
       ph_ld[st] ^= 1;
       const float eg = (ok && t < L) ? __expf(gsm[t]) : 0.0f;
       float qs[NV];  // e^{gamma_t} (Q S^T)[t][:], all 32 columns of the slice, 16 at a time
-      ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma));
+      ok = __all_sync(0xffffffffu, ok && wait_ok(mbar_mma[0], ph_mma));
       tc::tc_fence_after();
       if (ok) {
 #pragma unroll
@@ -995,7 +1047,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
           for (int i = 0; i < 16; ++i) qs[16 * h16 + i] = eg * (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
         }
       }
-      ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma));
+      ok = __all_sync(0xffffffffu, ok && wait_ok(mbar_mma[1], ph_mma));
       ph_mma ^= 1;
       tc::tc_fence_after();
       if (ok) {  // Y = e^gamma Q S^T + (M o QK^T) U, and this slice's sum of squares to the peers
@@ -1026,8 +1078,9 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       }
       tc::tc_fence_before();
       tc::mbar_arrive(tc::smem_u32(&norm_done));  // this chunk's TMEM rows and stage are read
-      if (!ok || !finish(c)) { s_abort = 1; atomicExch(&g_gdn_status, -7); break; }
-      if (s_abort) break;
+      // warp-uniform decisions: every lane of a norm warp leaves at the same chunk
+      if (!__all_sync(0xffffffffu, ok && finish(c))) { s_abort = 1; atomicExch(&g_gdn_status, -7); break; }
+      if (__any_sync(0xffffffffu, aborted_now())) break;
     }
   }
   for (int c = 0; c < nchunks && !aborted && !normw; ++c) {
@@ -1037,7 +1090,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     uint8_t* r_hi = sg + PBStage::VS;
     uint8_t* r_lo = r_hi + PB_R_TILE;
     const uint32_t kq0 = tc::smem_u32(sg + PBStage::KQ), tp0 = tc::smem_u32(sg + PBStage::TP);
-    if (worker && !tc::mbar_wait(tc::smem_u32(&mbar_ld[st]), ph_ld[st])) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    if (worker) (void)wait_ok(mbar_ld[st], ph_ld[st]);
     ph_ld[st] ^= 1;
     const float* gsm = reinterpret_cast<const float*>(sg + PBStage::GB);
     const float gL = gsm[L - 1];
@@ -1054,14 +1107,12 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     const float eg = t < L ? __expf(gsm[t]) : 0.0f;
     // the norm warps are done with the previous chunk's TMEM rows and stage before this
     // chunk's first round overwrites the one and the producer reloads the other
-    if (FUSED && tid == 0 && c > 0 && !tc::mbar_wait(tc::smem_u32(&norm_done), (uint32_t)(c - 1) & 1u)) {
-      s_abort = 1;
-      atomicExch(&g_gdn_status, -7);
-    }
-    loop_sync();
-    if (s_abort) { aborted = true; break; }
+    if (FUSED && tid == 0 && c > 0) (void)wait_ok(norm_done, (uint32_t)(c - 1) & 1u);
+    // the chunk barrier, reducing the abort flag: a timeout recorded by any thread before it
+    // arrived ends the loop for every thread at the same chunk
+    if (loop_sync_or(aborted_now())) { aborted = true; break; }
     // ---- round 1: [K S^T ; Q S^T] = [K;Q] (128 x 128) x S^T (K = 128, N = nv) -------------
-    if (tid == 0) {
+    if (tid == 0 && !aborted_now()) {
       tc::tc_fence_after();
       const uint64_t da[2] = {tc::sdesc(kq0, LBO128, 128), tc::sdesc(kq0 + KQ_TILE, LBO128, 128)};
 #pragma unroll
@@ -1072,8 +1123,11 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       }
       tc::umma_commit(tc::smem_u32(&mbar_mma[0]));
     }
-    if (producer && lane == 0 && c + 1 < nchunks) issue_load(c + 1, st ^ 1);  // stage last read by chunk c-1
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[0]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    if (producer && lane == 0 && c + 1 < nchunks && !aborted_now()) {  // stage last read by chunk c-1
+      issue_load(c + 1, st ^ 1);
+      last_load = c + 1;
+    }
+    (void)wait_ok(mbar_mma[0], ph_mma);
     tc::tc_fence_after();
     float qs[NH];  // y rows (separate-epilogue mode): e^{gamma_t} (Q S^T)[t][:]
     if (rwarp || (!FUSED && worker)) {
@@ -1105,7 +1159,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     tc::tc_fence_before();
     if (rwarp) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 2: [U ; (M o QK^T) U] = [T;P] (128 x 64) x R (K = 64, N = nv) ----------------
-    if (tid == 0) {
+    if (tid == 0 && !aborted_now()) {
       tc::tc_fence_after();
       const uint64_t da[2] = {tc::sdesc(tp0, LBO128, 128), tc::sdesc(tp0 + TP_TILE, LBO128, 128)};
       const uint64_t db = tc::sdesc(tc::smem_u32(r_hi), 128, 8 * 128);
@@ -1117,7 +1171,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       }
       tc::umma_commit(tc::smem_u32(&mbar_mma[1]));
     }
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[1]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    (void)wait_ok(mbar_mma[1], ph_mma);
     tc::tc_fence_after();
     if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
@@ -1153,7 +1207,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     tc::tc_fence_before();
     if (rwarp) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 3: K^T U-tilde: A = MN-major view of the K rows (M = 128 key comps, K = 64 tokens)
-    if (tid == 0) {
+    if (tid == 0 && !aborted_now()) {
       tc::tc_fence_after();
       const uint64_t da[2] = {tc::sdesc(kq0, 128, LBO128), tc::sdesc(kq0 + KQ_TILE, 128, LBO128)};
       const uint64_t db = tc::sdesc(tc::smem_u32(r_hi), 128, 8 * 128);
@@ -1165,7 +1219,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       }
       tc::umma_commit(tc::smem_u32(&mbar_mma[2]));
     }
-    if (!tc::mbar_wait(tc::smem_u32(&mbar_mma[2]), ph_mma)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+    (void)wait_ok(mbar_mma[2], ph_mma);
     ph_mma ^= 1;
     tc::tc_fence_after();
     if (worker) {
@@ -1185,6 +1239,12 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
 #pragma unroll
     for (int i = 0; i < NH; ++i) final_state[sbase + (size_t)(cb + i) * D + row] = S[i];
   }
+  // after a timeout, let the stage copies still in flight land (bounded) before the shared
+  // memory they write is released: the last issued one completes its barrier's phase
+  // (last_load >> 1) & 1, and every earlier one completed before it was waited on or before
+  // the next copy into its stage was issued
+  if (aborted_now() && producer && lane == 0 && last_load >= 0)
+    (void)tc::mbar_wait(tc::smem_u32(&mbar_ld[last_load & 1]), (uint32_t)(last_load >> 1) & 1u);
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tbase, 256);

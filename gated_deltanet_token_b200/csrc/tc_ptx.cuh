@@ -17,7 +17,17 @@
 #include <stdint.h>
 
 namespace gdn {
+
+// Limit of every bounded wait below, in ns of %globaltimer (set by gdn_set_wait_limit_ns).
+__device__ unsigned long long g_gdn_wait_ns = 2000000000ull;
+
 namespace tc {
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -59,16 +69,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: gives up after ~2 s of the global timer and returns false.
+// Bounded wait: gives up after g_gdn_wait_ns of the global timer (2 s by default) and
+// returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  const uint64_t t0 = globaltimer();
+  const uint64_t lim = *static_cast<volatile unsigned long long*>(&g_gdn_wait_ns);
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    if (t - t0 > 2000000000ull) return false;
+    if (globaltimer() - t0 > lim) return false;
   }
 }
 
@@ -115,6 +124,10 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // `bar`.  `tmap` is the address of a __grid_constant__ CUtensorMap kernel parameter; (x, y, z)
 // is the box origin in elements (x * element size must be a multiple of 16 bytes; the other
 // coordinates may be negative or past the end: those elements read as zeros).
+// L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned global address
+__device__ __forceinline__ void prefetch_l2(const void* gptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "

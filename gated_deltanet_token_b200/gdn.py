@@ -15,8 +15,13 @@ import torch
 
 GDN_OK = 0
 GDN_ERR_INDEX = -8
+GDN_ERR_DEVICE_TIMEOUT = -7
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
+# path options (gdn_set_options): slower alternatives with the same results, for comparisons
+GDN_OPT_FORCE_FP32_PATH = 1
+GDN_OPT_SEPARATE_NORM = 2
+GDN_OPT_NO_PDL = 4
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 _lib = None
 
@@ -66,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode.argtypes = [dp] + [vp] * 13 + [vp]
         L.gdn_decode_slots.restype = ctypes.c_int
         L.gdn_decode_slots.argtypes = [dp] + [vp] * 12 + [ctypes.c_int32, vp, vp, vp]
+        L.gdn_decode_multi.restype = ctypes.c_int
+        L.gdn_decode_multi.argtypes = [dp, ctypes.c_int32] + [vp] * 13 + [vp]
         L.gdn_prefill_conv_state.restype = ctypes.c_int
         L.gdn_prefill_conv_state.argtypes = [dp] + [vp] * 5 + [vp]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -80,6 +87,14 @@ def lib() -> ctypes.CDLL:
         L.gdn_selftest_tc.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_float)]
         L.gdn_version.restype = ctypes.c_int
         L.gdn_version.argtypes = []
+        L.gdn_set_options.restype = ctypes.c_uint32
+        L.gdn_set_options.argtypes = [ctypes.c_uint32]
+        L.gdn_get_options.restype = ctypes.c_uint32
+        L.gdn_get_options.argtypes = []
+        L.gdn_set_wait_limit_ns.restype = ctypes.c_int
+        L.gdn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.gdn_selftest_wait_timeout.restype = ctypes.c_int
+        L.gdn_selftest_wait_timeout.argtypes = [vp]
         _lib = L
     return _lib
 
@@ -123,6 +138,28 @@ def gdn_version() -> int:
 
 def gdn_read_device_status(stream=None) -> int:
     return lib().gdn_read_device_status(_stream(stream))
+
+
+def gdn_set_options(flags: int) -> int:
+    """Replace the process-wide path options; returns the previous word."""
+    return int(lib().gdn_set_options(int(flags)))
+
+
+def gdn_get_options() -> int:
+    return int(lib().gdn_get_options())
+
+
+def gdn_set_wait_limit_ns(ns: int) -> None:
+    rc = lib().gdn_set_wait_limit_ns(int(ns))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_set_wait_limit_ns")
+
+
+def gdn_selftest_wait_timeout(stream=None) -> None:
+    """Launch the bounded-wait diagnostic (read its result with gdn_read_device_status)."""
+    rc = lib().gdn_selftest_wait_timeout(_stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_selftest_wait_timeout")
 
 
 def gdn_selftest_tc(case_id: int) -> tuple[float, float]:
@@ -273,4 +310,25 @@ def gdn_decode_slots(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_stat
                                 _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_slots")
+    return y
+
+
+def gdn_decode_multi(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, *,
+                     out_dtype=None, y=None, q_scale=1.0, l2_eps=1e-6, rms_eps=1e-6, stream=None):
+    """n_tokens decode steps per sequence in one call: q, k [N, n_tokens, h_qk, 128]; v, z
+    [N, n_tokens, h_v, 128]; a, b [N, n_tokens, h_v].  conv_state [N, 3, C_conv] and state
+    [N, h_v, 128, 128] are updated in place.  Returns y [N, n_tokens, h_v, 128]."""
+    N, K, h_qk, d_k = q.shape
+    h_v, d_v = v.shape[2], v.shape[3]
+    if out_dtype is None:
+        out_dtype = q.dtype
+    dims = make_dims(N, N * K, h_qk, h_v, _dt(q), _dt(torch.empty(0, dtype=out_dtype)), d_k, d_v, q_scale,
+                     l2_eps, rms_eps)
+    if y is None:
+        y = torch.empty((N, K, h_v, d_v), dtype=out_dtype, device=q.device)
+    rc = lib().gdn_decode_multi(ctypes.byref(dims), ctypes.c_int32(K), _ptr(q), _ptr(k), _ptr(v), _ptr(z),
+                                _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(conv_w), _ptr(norm_w),
+                                _ptr(conv_state), _ptr(state), _ptr(y), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_multi")
     return y

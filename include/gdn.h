@@ -163,6 +163,26 @@ int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const vo
                      const float* conv_w, const float* norm_w, void* conv_state_pool, float* state_pool,
                      int32_t n_slots, const int32_t* slot_ids, void* y, gdn_stream_t stream);
 
+/*
+ * Several decode tokens per sequence in one call (1 <= n_tokens <= 8), e.g. to verify drafted
+ * tokens: the same per-token rule as gdn_decode (field guide, §02, steps 1-6, then the gated
+ * RMSNorm) applied to n_tokens consecutive tokens of each sequence, reading and writing each
+ * state row once per call instead of once per token.
+ *
+ *   q, k        [N][n_tokens][h_qk][d_k]   in_dtype
+ *   v, z        [N][n_tokens][h_v][d_v]    in_dtype
+ *   a, b        [N][n_tokens][h_v]         fp32
+ *   conv_state  [N][3][C_conv]             in/out: replaced by the last three raw rows
+ *   state       [N][h_v][d_v][d_k]         fp32, in/out: the state after the last token
+ *   y           [N][n_tokens][h_v][d_v]    out_dtype (written)
+ * d->total_tokens must equal d->n_seqs * n_tokens.  Returns GDN_ERR_SHAPE for n_tokens
+ * outside 1..8, otherwise what gdn_decode returns.
+ */
+int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const void* k, const void* v,
+                     const void* z, const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
+                     gdn_stream_t stream);
+
 /* Static, NUL-terminated name of a return code ("GDN_OK", "GDN_ERR_SHAPE", ...). */
 const char* gdn_status_string(int code);
 
@@ -217,7 +237,9 @@ int gdn_profile_read(gdn_kernel_time_t* out, int max_entries);
  *     exceeds GDN_NOALLOC_SCRATCH_BYTES (at the pages' model shape, 16 QK / 32 value
  *     heads, one sequence: up to 960 packed tokens with bf16 inputs, 741 with fp32).
  *   - The first call on a device looks up that device's address of the scratch array
- *     (with that device current); make that first call before any stream capture.
+ *     (with that device current); make that first call before any stream capture.  The
+ *     address is cached for the life of the process: it assumes the device's primary
+ *     context is never torn down (no cudaDeviceReset between calls).
  *   - Every call on a device shares the one array, which keeps the previous call's
  *     contents; the prefill writes every scratch byte before reading it, so nothing needs
  *     clearing.  Calls whose work overlaps on the GPU (two streams, or two host threads)
@@ -240,6 +262,47 @@ int gdn_prefill_noalloc(const gdn_dims_t* d, const void* q, const void* k, const
  * allocates nothing.  Returns GDN_OK, GDN_ERR_NULL, GDN_ERR_SHAPE (bad case) or GDN_ERR_CUDA.
  */
 int gdn_selftest_tc(int case_id, float* out2);
+
+/*
+ * Path options, process-wide (all devices, all threads).  The default, 0, is the fast path
+ * of every call; each bit selects a slower alternative that computes the same result, for
+ * comparisons and diagnostics:
+ *   GDN_OPT_FORCE_FP32_PATH   bf16-input prefills take the fp32 FFMA path
+ *   GDN_OPT_SEPARATE_NORM     the bf16 path's output norm runs in its own kernel
+ *   GDN_OPT_NO_PDL            plain stream order between the prefill's kernels
+ * The initial value is read once per process from the environment (GDN_FORCE_SIMT=1,
+ * GDN_NO_FUSED_NORM=1, GDN_NO_PDL=1).  gdn_set_options replaces the word and
+ * returns the previous one (unknown bits are dropped); it takes effect for calls made after
+ * it.  Changing it while another host thread issues calls is allowed, but which value such a
+ * call sees is unspecified.
+ */
+#define GDN_OPT_FORCE_FP32_PATH 1u
+#define GDN_OPT_SEPARATE_NORM 2u
+#define GDN_OPT_NO_PDL 4u
+#define GDN_OPT_ALL 7u
+uint32_t gdn_set_options(uint32_t flags);
+uint32_t gdn_get_options(void);
+
+/*
+ * Limit of every bounded device-side wait of the tensor-core kernels (an mbarrier that the
+ * bulk copies or the tensor cores complete, a peer CTA's exchange word), in nanoseconds of the
+ * GPU's global timer, on the current device.  Default 2e9 (2 s).  A wait that runs out records
+ * GDN_ERR_DEVICE_TIMEOUT in the device status word (gdn_read_device_status) and the kernel
+ * leaves early: its outputs are then unspecified.  Synchronous (a copy to device memory on the
+ * legacy default stream; call it with no library work in flight).  Returns GDN_OK,
+ * GDN_ERR_SHAPE for 0, or GDN_ERR_CUDA.
+ */
+int gdn_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Diagnostic of the bounded waits: one CTA allocates tensor memory, initialises an mbarrier
+ * that nothing will ever complete, and waits on it with the limit set by
+ * gdn_set_wait_limit_ns, as the prefill kernels wait on theirs.  The wait runs out, the kernel
+ * records GDN_ERR_DEVICE_TIMEOUT in the device status word, frees its tensor memory and
+ * returns; no copy is in flight at any time.  Asynchronous on `stream`; read the result with
+ * gdn_read_device_status(stream).  Returns GDN_OK or GDN_ERR_CUDA (launch failure).
+ */
+int gdn_selftest_wait_timeout(gdn_stream_t stream);
 
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gdn_version(void);

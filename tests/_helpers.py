@@ -3,8 +3,23 @@ run the oracle, and compute the parity metrics (max-abs error on y against RMS(y
 relative Frobenius error of the states)."""
 from __future__ import annotations
 
+import contextlib
+
 import numpy as np
 import torch
+
+
+@contextlib.contextmanager
+def path_options(flags):
+    """Run the body with the library's path options set to `flags` (gdn_set_options), then
+    restore the previous word."""
+    from gated_deltanet_token_b200 import gdn
+
+    prev = gdn.gdn_set_options(flags)
+    try:
+        yield
+    finally:
+        gdn.gdn_set_options(prev)
 
 
 def to_dev(x, device="cuda"):

@@ -132,6 +132,26 @@ def test_handoff_calls_reject_bad_arguments(glib):
     assert slots(four, pool=FAKE + 8) == -4
 
 
+def test_decode_multi_rejects_bad_arguments(glib):
+    L = glib.lib()
+
+    def call(dims, K, ptrs=None):
+        p = [FAKE] * 13 if ptrs is None else ptrs
+        return L.gdn_decode_multi(None if dims is None else ctypes.byref(dims), ctypes.c_int32(K),
+                                  *[ctypes.c_void_p(x) if x else None for x in p], None)
+
+    assert call(None, 2) == -1
+    assert call(glib.make_dims(4, 8, 16, 32, 1, 1), 0) == -2
+    assert call(glib.make_dims(4, 36, 16, 32, 1, 1), 9) == -2  # more than 8 tokens
+    assert call(glib.make_dims(4, 7, 16, 32, 1, 1), 2) == -2   # total_tokens != n_seqs * n_tokens
+    bad = [FAKE] * 13
+    bad[11] = None
+    assert call(glib.make_dims(4, 8, 16, 32, 1, 1), 2, bad) == -1
+    bad = [FAKE] * 13
+    bad[0] = FAKE + 2
+    assert call(glib.make_dims(4, 8, 16, 32, 1, 1), 2, bad) == -4
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     from gated_deltanet_token_b200 import gdn
 
@@ -139,3 +159,17 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(gdn, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="libgdn.so not found"):
         gdn.lib()
+
+
+def test_path_options_round_trip(glib):
+    """The path-option word (host only): set returns the previous word, unknown bits are
+    dropped, and the previous value is restored."""
+    prev = glib.gdn_set_options(0)
+    try:
+        assert glib.gdn_get_options() == 0
+        assert glib.gdn_set_options(0xFF) == 0
+        assert glib.gdn_get_options() == (glib.GDN_OPT_FORCE_FP32_PATH | glib.GDN_OPT_SEPARATE_NORM |
+                                          glib.GDN_OPT_NO_PDL)
+    finally:
+        glib.gdn_set_options(prev)
+    assert glib.gdn_get_options() == prev

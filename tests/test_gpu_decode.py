@@ -174,3 +174,77 @@ def test_decode_slot_past_the_pool_sets_the_index_status():
     assert torch.equal(y[0], y_ref[0]) and torch.isnan(y[1]).all()
     assert torch.equal(dd["state"][0], ref_state[0])  # entry 0 ran; slot 1 was left alone
     assert torch.equal(dd["state"][1], torch.from_numpy(inp["state"][1]).cuda())
+
+
+# ---- several decode tokens per sequence in one call ---------------------------------------
+
+def bf16_from_f64(x):
+    """Bits of fp64 values that are exact bf16 numbers (raw history rows), as uint16."""
+    return (np.ascontiguousarray(x, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _multi_inputs(K, N=3, dtype="bf16", seed=11):
+    """K consecutive decode tokens per sequence: the per-token fields of K seeded one-token
+    workloads stacked on axis 1; state, conv history and parameters from the first."""
+    steps = [make_inputs("decode_N256_bf16", seed=seed + i, n_seqs=N, h_qk=2, h_v=4, dtype=dtype) for i in range(K)]
+    out = dict(steps[0])
+    for nm in ("q", "k", "v", "z", "a", "b"):
+        out[nm] = np.ascontiguousarray(np.stack([s_[nm] for s_ in steps], axis=1))
+    return out
+
+
+def _run_multi(inp, out_dtype=torch.float32):
+    from gated_deltanet_token_b200 import gdn
+
+    d = {nm: to_dev(inp[nm]) for nm in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w", "norm_w",
+                                        "conv_state", "state")}
+    y = gdn.gdn_decode_multi(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                             d["conv_w"], d["norm_w"], d["conv_state"], d["state"], out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    return y, d["state"], d["conv_state"]
+
+
+def test_decode_multi_one_token_equals_decode():
+    from gated_deltanet_token_b200 import gdn
+
+    inp = _multi_inputs(1)
+    y_m, S_m, cs_m = _run_multi(inp)
+    one = dict(inp)
+    for nm in ("q", "k", "v", "z", "a", "b"):
+        one[nm] = np.ascontiguousarray(inp[nm][:, 0])
+    d = {nm: to_dev(one[nm]) for nm in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w", "norm_w",
+                                        "conv_state", "state")}
+    y_1 = gdn.gdn_decode(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["conv_w"],
+                         d["norm_w"], d["conv_state"], d["state"], out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(y_m[:, 0], y_1) and torch.equal(S_m, d["state"]) and torch.equal(cs_m, d["conv_state"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("K", [2, 5, 8])
+def test_decode_multi_equals_successive_steps(oracle_mod, K, dtype):
+    inp = _multi_inputs(K, dtype=dtype)
+    y, S, cs = _run_multi(inp)
+    state = inp["state"].astype(np.float32)
+    hist = inp["conv_state"]
+    ys = []
+    for t in range(K):  # the oracle, one token at a time, carrying the state and the history
+        step = dict(inp)
+        for nm in ("q", "k", "v", "z", "a", "b"):
+            step[nm] = np.ascontiguousarray(inp[nm][:, t])
+        step["state"], step["conv_state"] = state, hist
+        o = oracle_mod.decode(step)
+        ys.append(o["y"])
+        state = o["state"].astype(np.float32)
+        hist = (bf16_from_f64(o["conv_state"]) if dtype == "bf16" else o["conv_state"].astype(np.float32))
+    y_ref = np.stack(ys, axis=1)
+    yy = y.cpu().numpy().astype(np.float64)
+    SS = S.cpu().numpy().astype(np.float64)
+    if dtype == "bf16":
+        check_bf16(yy, y_ref, SS, o["state"])
+    else:
+        check_fp32(yy, y_ref, SS, o["state"])
+    got = cs.view(torch.int16).cpu().numpy().view(np.uint16) if cs.dtype == torch.bfloat16 else cs.cpu().numpy()
+    exp = bf16_from_f64(o["conv_state"]) if dtype == "bf16" else o["conv_state"].astype(np.float32)
+    assert np.array_equal(got, exp)  # the raw history, bit-exact
+

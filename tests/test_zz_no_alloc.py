@@ -7,9 +7,12 @@ collected last on purpose, so a run that stops at the first failure has run ever
 else first; it also passes when run alone in a fresh process.
 
 The call goes through the C ABI with raw device pointers and is compared with the
-ordinary gdn_prefill (caller workspace) within the bf16-run tolerance of the parity
-tests, on two calls in a row with different inputs (the scratch keeps the previous
-call's contents, so a stale byte would show up in the second call).
+ordinary gdn_prefill (caller workspace), on two calls in a row with different inputs (the
+scratch keeps the previous call's contents, so a stale byte would show up in the second
+call).  Both run the same kernels on the same inputs with the same workspace layout, so
+their outputs must be identical bit for bit; the parity tolerance would let a slightly
+perturbed result through.  Both input dtypes are covered: bf16 inputs use the tensor-core
+workspace layout, fp32 inputs the fp32 path's.
 """
 import ctypes
 
@@ -19,7 +22,7 @@ import torch
 
 from gated_deltanet_token_b200 import gdn
 from gated_deltanet_token_b200.inputs import make_inputs
-from tests._helpers import check_bf16, run_prefill, to_dev
+from tests._helpers import run_prefill, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -31,7 +34,8 @@ def _noalloc(inp):
     T, h_qk, _ = t["q"].shape
     h_v = t["v"].shape[1]
     n = cu.numel() - 1
-    dims = gdn.make_dims(n, T, h_qk, h_v, gdn.GDN_DTYPE_BF16, gdn.GDN_DTYPE_F32)
+    in_dt = gdn.GDN_DTYPE_BF16 if t["q"].dtype == torch.bfloat16 else gdn.GDN_DTYPE_F32
+    dims = gdn.make_dims(n, T, h_qk, h_v, in_dt, gdn.GDN_DTYPE_F32)
     assert gdn.gdn_prefill_workspace_size(dims) <= 64 << 20
     y = torch.full((T, h_v, 128), float("nan"), dtype=torch.float32, device="cuda")
     fs = torch.full((n, h_v, 128, 128), float("nan"), dtype=torch.float32, device="cuda")
@@ -44,13 +48,14 @@ def _noalloc(inp):
     return y.cpu().numpy().astype(np.float64), fs.cpu().numpy().astype(np.float64)
 
 
-def test_noalloc_matches_workspace_prefill_on_two_calls():
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_noalloc_matches_workspace_prefill_on_two_calls(dtype):
     for seed, lens in ((0, [300, 0, 129, 64]), (1, [65, 5, 250])):
-        inp = make_inputs("varlen8_prefill_bf16", seed=seed, lengths=lens)
+        inp = make_inputs("varlen8_prefill_bf16", seed=seed, lengths=lens, dtype=dtype)
         y_ref, S_ref = run_prefill(inp, torch.float32)
         y, S = _noalloc(inp)
         assert np.isfinite(y).all() and np.isfinite(S).all()
-        check_bf16(y, y_ref, S, S_ref)
+        assert np.array_equal(y, y_ref) and np.array_equal(S, S_ref)
 
 
 def test_noalloc_rejects_dims_beyond_its_scratch():
