@@ -108,7 +108,7 @@ WsLayout ws_layout(const gdn_dims_t* d) {
   L.vc = take(T * hv * D * 4);
   L.g = take(T * hv * 4);
   L.beta = take(T * hv * 4);
-  L.gam = take(T * hv * 4);
+  L.gam = take(T * hv * 8);  // gamma in fp64
   L.W = take(T * hv * D * 4);
   L.Up = take(T * hv * D * 4);
   L.mqk = take(T * hv * CH * 4);
@@ -464,12 +464,13 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     }
     ProfScope p("chunk_phaseA_simt", s);
     k_phaseA_simt<<<dim3(L.max_chunks, d->h_v), 256, PA_SMEM, s>>>(
-        kd, tab, F(L.qn), F(L.kn), F(L.vc), F(L.g), F(L.beta), F(L.gam), F(L.W), F(L.Up), F(L.mqk));
+        kd, tab, F(L.qn), F(L.kn), F(L.vc), F(L.g), F(L.beta), reinterpret_cast<double*>(ws + L.gam), F(L.W),
+        F(L.Up), F(L.mqk));
   }
   {
     ProfScope p("chunk_phaseB_simt", s);
     k_phaseB_simt<<<dim3(d->n_seqs, d->h_v, D / PB_VS), 256, PB_SMEM, s>>>(
-        kd, cu_seqlens, F(L.qn), F(L.kn), F(L.gam), F(L.W), F(L.Up), F(L.mqk), init_state, F(L.yraw),
+        kd, cu_seqlens, F(L.qn), F(L.kn), reinterpret_cast<const double*>(ws + L.gam), F(L.W), F(L.Up), F(L.mqk), init_state, F(L.yraw),
         final_state);
   }
   if (d->total_tokens > 0) {

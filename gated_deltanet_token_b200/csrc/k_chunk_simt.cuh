@@ -24,14 +24,14 @@ namespace gdn {
 
 constexpr int PA_LD = 132;  // padded row pitch (floats) of 64 x 128 tiles
 constexpr int PA_ALD = 68;  // padded row pitch of the 64 x 64 A tile
-constexpr size_t PA_SMEM = (size_t)(2 * 64 * PA_LD + 64 * PA_ALD + 3 * 64) * sizeof(float);
+constexpr size_t PA_SMEM = (size_t)(2 * 64 * PA_LD + 64 * PA_ALD + 4 * 64) * sizeof(float);
 
 // Phase A: grid (chunk, value head), 256 threads.
 __global__ void __launch_bounds__(256, 2)
     k_phaseA_simt(Dims d, const ChunkEntry* __restrict__ tab, const float* __restrict__ qn,
                   const float* __restrict__ kn, const float* __restrict__ vc,
                   const float* __restrict__ g, const float* __restrict__ beta,
-                  float* __restrict__ gam_out, float* __restrict__ W_out,
+                  double* __restrict__ gam_out, float* __restrict__ W_out,
                   float* __restrict__ Up_out, float* __restrict__ mqk_out) {
   const ChunkEntry e = tab[blockIdx.x];
   if (e.len == 0) return;
@@ -41,9 +41,9 @@ __global__ void __launch_bounds__(256, 2)
   float* Ks = reinterpret_cast<float*>(smem_f4);
   float* Qs = Ks + 64 * PA_LD;
   float* As = Qs + 64 * PA_LD;
-  float* gs = As + 64 * PA_ALD;  // gamma
-  float* bs = gs + 64;           // beta
-  float* be = bs + 64;           // beta * e^gamma
+  double* gs = reinterpret_cast<double*>(As + 64 * PA_ALD);  // gamma (fp64: see below)
+  float* bs = reinterpret_cast<float*>(gs + 64);               // beta
+  float* be = bs + 64;                                         // beta * e^gamma
 
   for (int idx = tid; idx < 64 * 32; idx += 256) {
     const int t = idx >> 5, c4 = (idx & 31) * 4;
@@ -56,13 +56,17 @@ __global__ void __launch_bounds__(256, 2)
     *reinterpret_cast<float4*>(Ks + t * PA_LD + c4) = kv;
     *reinterpret_cast<float4*>(Qs + t * PA_LD + c4) = qv;
   }
-  if (warp == 0) {  // inclusive prefix sum of g over the chunk, two tokens per lane
-    float s0 = lane < L ? g[(size_t)(e.t0 + lane) * hv + h] : 0.0f;
-    float s1 = lane + 32 < L ? g[(size_t)(e.t0 + lane + 32) * hv + h] : 0.0f;
+  // Inclusive prefix sum of g over the chunk, two tokens per lane, in fp64: every decay
+  // factor e^{gamma_t - gamma_s} is formed from a difference of two prefixes, which in fp32
+  // would carry an absolute error of ulp(|gamma|) -- about 2e-4 once a few strong decays (g of
+  // several hundred) have accumulated in the chunk.
+  if (warp == 0) {
+    double s0 = lane < L ? g[(size_t)(e.t0 + lane) * hv + h] : 0.0f;
+    double s1 = lane + 32 < L ? g[(size_t)(e.t0 + lane + 32) * hv + h] : 0.0f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const float y0 = __shfl_up_sync(0xffffffffu, s0, o);
-      const float y1 = __shfl_up_sync(0xffffffffu, s1, o);
+      const double y0 = __shfl_up_sync(0xffffffffu, s0, o);
+      const double y1 = __shfl_up_sync(0xffffffffu, s1, o);
       if (lane >= o) { s0 += y0; s1 += y1; }
     }
     s1 += __shfl_sync(0xffffffffu, s0, 31);
@@ -70,7 +74,7 @@ __global__ void __launch_bounds__(256, 2)
     const float b1 = lane + 32 < L ? beta[(size_t)(e.t0 + lane + 32) * hv + h] : 0.0f;
     gs[lane] = s0; gs[lane + 32] = s1;
     bs[lane] = b0; bs[lane + 32] = b1;
-    be[lane] = b0 * expf(s0); be[lane + 32] = b1 * expf(s1);
+    be[lane] = b0 * expf((float)s0); be[lane + 32] = b1 * expf((float)s1);
     if (lane < L) gam_out[(size_t)(e.t0 + lane) * hv + h] = s0;
     if (lane + 32 < L) gam_out[(size_t)(e.t0 + lane + 32) * hv + h] = s1;
   }
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int t = tb + 16 * r, s = sb + 16 * c;
-        const float dec = s <= t ? expf(gs[t] - gs[s]) : 0.0f;  // mask before exp
+        const float dec = s <= t ? expf((float)(gs[t] - gs[s])) : 0.0f;  // mask before exp
         As[t * PA_ALD + s] = s < t ? bs[t] * dec * kk[r][c] : 0.0f;
         if (t < L) mqk_out[((size_t)(e.t0 + t) * hv + h) * CH + s] = (s <= t) ? dec * qk[r][c] : 0.0f;
       }
@@ -140,12 +144,12 @@ constexpr int PB_LD = 132;  // row pitch of 128-wide tiles
 constexpr int PB_ULD = 36;  // row pitch of the U tile
 constexpr int PB_MLD = 68;  // row pitch of the M o QK^T tile
 constexpr size_t PB_SMEM =
-    (size_t)(PB_VS * PB_LD + 3 * 64 * PB_LD + 64 * PB_ULD + 64 * PB_MLD + 64) * sizeof(float);
+    (size_t)(PB_VS * PB_LD + 3 * 64 * PB_LD + 64 * PB_ULD + 64 * PB_MLD + 2 * 64) * sizeof(float);
 
 // Phase B: grid (sequence, value head, state slice), 256 threads.
 __global__ void __launch_bounds__(256, 1)
     k_phaseB_simt(Dims d, const int* __restrict__ cu, const float* __restrict__ qn,
-                  const float* __restrict__ kn, const float* __restrict__ gam,
+                  const float* __restrict__ kn, const double* __restrict__ gam,
                   const float* __restrict__ Wg, const float* __restrict__ Upg,
                   const float* __restrict__ mqk, const float* init_state,
                   float* __restrict__ y_raw, float* final_state) {
@@ -160,7 +164,7 @@ __global__ void __launch_bounds__(256, 1)
   float* Ks = Qs + 64 * PB_LD;                     // [64][PB_LD]  diag(e^{gamma_L - gamma}) K
   float* Us = Ks + 64 * PB_LD;                     // [64][PB_ULD] U' then U (slice columns)
   float* Ms = Us + 64 * PB_ULD;                    // [64][PB_MLD] M o QK^T
-  float* gs = Ms + 64 * PB_MLD;                    // [64] gamma
+  double* gs = reinterpret_cast<double*>(Ms + 64 * PB_MLD);  // [64] gamma (fp64)
 
   const size_t sbase = (((size_t)n * hv + h) * D + i0) * D;
   for (int idx = tid; idx < PB_VS * 32; idx += 256) {
@@ -173,9 +177,9 @@ __global__ void __launch_bounds__(256, 1)
   for (int t0 = ts; t0 < te; t0 += CH) {
     const int L = min(CH, te - t0);
     __syncthreads();  // the previous chunk is finished with every tile
-    if (tid < 64) gs[tid] = tid < L ? gam[(size_t)(t0 + tid) * hv + h] : 0.0f;
+    if (tid < 64) gs[tid] = tid < L ? gam[(size_t)(t0 + tid) * hv + h] : 0.0;
     __syncthreads();
-    const float gL = gs[L - 1];
+    const double gL = gs[L - 1];
     for (int idx = tid; idx < 64 * 32; idx += 256) {
       const int t = idx >> 5, c4 = (idx & 31) * 4;
       float4 wv = make_float4(0, 0, 0, 0), qv = wv, kv = wv;
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(256, 1)
         wv = *reinterpret_cast<const float4*>(Wg + ((size_t)(t0 + t) * hv + h) * D + c4);
         qv = *reinterpret_cast<const float4*>(qn + tk);
         kv = *reinterpret_cast<const float4*>(kn + tk);
-        const float f = expf(gL - gs[t]);
+        const float f = expf((float)(gL - gs[t]));
         kv.x *= f; kv.y *= f; kv.z *= f; kv.w *= f;
       }
       *reinterpret_cast<float4*>(Ws + t * PB_LD + c4) = wv;
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int t = tb + 16 * r;
-        const float eg = t < L ? expf(gs[t]) : 0.0f;
+        const float eg = t < L ? expf((float)gs[t]) : 0.0f;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           u[r][c] = Us[t * PB_ULD + ib + 16 * c] - wa[r][c];
@@ -271,7 +275,7 @@ __global__ void __launch_bounds__(256, 1)
     // rb + 8 r and columns 4 jb .. 4 jb + 3.
     {
       const int rb = tid >> 5, jb = (tid & 31) * 4;
-      const float eL = expf(gL);
+      const float eL = expf((float)gL);
       float4 acc[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {

@@ -5,8 +5,8 @@
 // "Qwen3.8-Flash-Next" model notes in column-vector form), regrouped so that every
 // contraction is an M = 128 tcgen05 MMA:
 //
-//   R   = diag(beta) (V - diag(e^gamma) K S^T)              [U = T R, T = (I + A)^-1]
-//   [U ; M o QK^T U] = [T ; P] R,   P = (M o QK^T) T        (one MMA, 128 x nv x 64)
+//   R   = V - diag(e^gamma) K S^T                           [U = T diag(beta) R, T = (I + A)^-1]
+//   [U ; M o QK^T U] = [T ; P] diag(beta) R,  P = (M o QK^T) T   (one MMA, 128 x nv x 64)
 //   Y   = diag(e^gamma) Q S^T + (M o QK^T) U
 //   S^T <- e^{gamma_L} S^T + K^T diag(e^{gamma_L - gamma}) U
 //   [K S^T ; Q S^T] = [K ; Q] S^T                            (one MMA, 128 x nv x 128)
@@ -39,7 +39,7 @@ constexpr uint32_t KQ_TILE = 128 * 128 * 2;          // one bf16 tile of [K;Q] (
 constexpr uint32_t KQ_BYTES = 2 * KQ_TILE;           // per (chunk, QK head)
 constexpr uint32_t TP_TILE = 128 * 64 * 2;           // one bf16 tile of [T;P]: 16 KB
 constexpr uint32_t TP_BYTES = 2 * TP_TILE;           // per (chunk, value head)
-constexpr uint32_t GB_FLOATS = 128;                  // gamma[64], beta[64] per (chunk, value head)
+constexpr uint32_t GB_FLOATS = 128;                  // gamma[64], gamma_L - gamma[64] per (chunk, value head)
 constexpr uint32_t VS_SLICE = 64 * TC_NV * 4;        // v after conv + SiLU (fp32), one 32-column slice: 8 KB
 constexpr uint32_t VS_BYTES = 4 * VS_SLICE;          // per (chunk, value head)
 constexpr uint32_t LBO128 = 2048;                    // K-direction core stride of 128-row tiles
@@ -485,7 +485,7 @@ constexpr uint32_t PA_OFF_PB = 32768;
 constexpr uint32_t PA_OFF_A = 32768;
 constexpr uint32_t PA_OFF_T = PA_OFF_A + 2 * PA_MAT;
 constexpr uint32_t PA_OFF_G = PA_OFF_T + 2 * PA_MAT;
-constexpr uint32_t PA_OFF_W = PA_OFF_G + 4 * 64 * 4;  // [16 half-warps][16 rows] float4 scratch
+constexpr uint32_t PA_OFF_W = PA_OFF_G + 2 * 64 * 8 + 2 * 64 * 4;  // [16 half-warps][16 rows] float4 scratch
 constexpr size_t PA_TC_SMEM = PA_OFF_W + 16 * 16 * 16;
 static_assert(PA_OFF_T >= KQ_BYTES, "T and the gates lie past the [K;Q] tile");
 static_assert(PA_TC_SMEM <= 113 * 1024, "two phase-A CTAs per SM");
@@ -517,8 +517,8 @@ __global__ void __launch_bounds__(256, 2)
   uint8_t* pb_lo = pb_hi + 16384;
   float* Am = reinterpret_cast<float*>(sm + PA_OFF_A);  // [2][64][PA_P]
   float* Tm = reinterpret_cast<float*>(sm + PA_OFF_T);  // [2][64][PA_P]
-  float* gs = reinterpret_cast<float*>(sm + PA_OFF_G);  // [2][64] gamma
-  float* bs = gs + 128;                                 // [2][64] beta
+  double* gs = reinterpret_cast<double*>(sm + PA_OFF_G);               // [2][64] gamma (fp64)
+  float* bs = reinterpret_cast<float*>(sm + PA_OFF_G + 2 * 64 * 8);   // [2][64] beta
   float4* wsc = reinterpret_cast<float4*>(sm + PA_OFF_W) + (tid >> 4) * 16;  // this half-warp's rows
   __shared__ uint64_t mbar;
   __shared__ uint32_t tslot;
@@ -548,7 +548,11 @@ __global__ void __launch_bounds__(256, 2)
     const int gpair[2] = {ga, ga + 1 < G ? ga + 1 : ga};
     if (warp < 2) {  // gates and gamma of the pair: warp 0 head a, warp 1 head b
       const int h = j * G + gpair[warp];
-      float g0 = 0.0f, g1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
+      // gamma is a prefix sum in fp64: a decay factor e^{gamma_t - gamma_s} is formed from the
+      // difference of two prefixes, which in fp32 would lose ulp(|gamma|) -- about 2e-4 once a
+      // few strong decays (g of several hundred) have accumulated in the chunk
+      double g0 = 0.0, g1 = 0.0;
+      float b0 = 0.0f, b1 = 0.0f;
       if (lane < L) {
         const size_t o = (size_t)(e.t0 + lane) * hv + h;
         g0 = decay_gate_f(a[o], A_log[h], dt_bias[h]);
@@ -561,17 +565,18 @@ __global__ void __launch_bounds__(256, 2)
       }
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const float y0 = __shfl_up_sync(0xffffffffu, g0, o);
-        const float y1 = __shfl_up_sync(0xffffffffu, g1, o);
+        const double y0 = __shfl_up_sync(0xffffffffu, g0, o);
+        const double y1 = __shfl_up_sync(0xffffffffu, g1, o);
         if (lane >= o) { g0 += y0; g1 += y1; }
       }
       g1 += __shfl_sync(0xffffffffu, g0, 31);
+      const double gL = __shfl_sync(0xffffffffu, g1, 31);  // gamma at the chunk's end (padding adds 0)
       gs[warp * 64 + lane] = g0; gs[warp * 64 + lane + 32] = g1;
       bs[warp * 64 + lane] = b0; bs[warp * 64 + lane + 32] = b1;
-      if (warp == 0 || gpair[1] != gpair[0]) {
+      if (warp == 0 || gpair[1] != gpair[0]) {  // phase B's gates: gamma_t and gamma_L - gamma_t
         float* gbw = gb_ws + ((size_t)chunk * hv + h) * GB_FLOATS;
-        gbw[lane] = g0; gbw[lane + 32] = g1;
-        gbw[64 + lane] = b0; gbw[96 + lane] = b1;
+        gbw[lane] = (float)g0; gbw[lane + 32] = (float)g1;
+        gbw[64 + lane] = (float)(gL - g0); gbw[96 + lane] = (float)(gL - g1);
       }
     }
     if (ga == 0) {  // [K;Q] K^T once the tile is in (the gates above overlapped the copy)
@@ -607,8 +612,8 @@ __global__ void __launch_bounds__(256, 2)
       tc::tmem_wait_ld();
 #pragma unroll 1
       for (int hp = 0; hp < 2; ++hp) {
-        const float* g_ = gs + hp * 64;
-        const float gt = g_[t];
+        const double* g_ = gs + hp * 64;
+        const double gt = g_[t];
         if (q4 < 2) {  // A[t][s] = beta_t e^{gamma_t - gamma_s} (k_t . k_s), s < t
           const float bt = bs[hp * 64 + t];
           float* Ah = Am + hp * (64 * PA_P);
@@ -619,7 +624,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int s_ = cbk + c4 * 4 + u;
-              op[u] = s_ < t ? bt * __expf(gt - g_[s_]) * __uint_as_float(r[c4 * 4 + u]) : 0.0f;
+              op[u] = s_ < t ? bt * __expf((float)(gt - g_[s_])) * __uint_as_float(r[c4 * 4 + u]) : 0.0f;
             }
             *reinterpret_cast<float4*>(Ah + t * PA_P + cbk + c4 * 4) = o;
           }
@@ -630,7 +635,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               const int s_ = cbk + c8 * 8 + u;
-              mv[u] = s_ <= t ? __expf(gt - g_[s_]) * __uint_as_float(r[c8 * 8 + u]) : 0.0f;
+              mv[u] = s_ <= t ? __expf((float)(gt - g_[s_])) * __uint_as_float(r[c8 * 8 + u]) : 0.0f;
             }
             uint4 hi, lo;
             tc::split8(mv, hi, lo);
@@ -706,15 +711,17 @@ __global__ void __launch_bounds__(256, 2)
       }
       __syncthreads();
     }
-    // T of both heads as columns hp * 64 .. of the MN-major B operand of P (over the dead A
-    // matrices), and the T rows of each head's [T;P] output tile (K-major, straight to the
-    // workspace); blocks above the diagonal are zeros.
+    // T diag(beta) of both heads as columns hp * 64 .. of the MN-major B operand of P (over the
+    // dead A matrices), and the T diag(beta) rows of each head's [T;P] output tile (K-major,
+    // straight to the workspace); blocks above the diagonal are zeros.  With beta folded in
+    // here, phase B forms R = V - diag(e^gamma) K S^T and [T;P] diag(beta) R gives U and
+    // (M o QK^T) U.
     for (int it = tid; it < 2 * 64 * 8; it += 256) {
       const int hp = it >> 9, r = it & 63, s0 = ((it >> 6) & 7) * 8;
       float tv[8];
       if ((s0 >> 4) <= (r >> 4)) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) tv[c] = Tm[hp * (64 * PA_P) + r * PA_P + s0 + c];
+        for (int c = 0; c < 8; ++c) tv[c] = Tm[hp * (64 * PA_P) + r * PA_P + s0 + c] * bs[hp * 64 + s0 + c];
       } else {
 #pragma unroll
         for (int c = 0; c < 8; ++c) tv[c] = 0.0f;
@@ -1137,11 +1144,10 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       tc::tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
-      if (quarter < 2) {  // R[t][i] = beta_t (v[t][i] - e^{gamma_t} (K S^T)[t][i])
-        const float bt = t < L ? gsm[64 + t] : 0.0f;
+      if (quarter < 2) {  // R[t][i] = v[t][i] - e^{gamma_t} (K S^T)[t][i]  (beta is in the [T;P] tile)
         float rr[NH];
 #pragma unroll
-        for (int i = 0; i < NH; ++i) rr[i] = t < L ? bt * fmaf(-eg, __uint_as_float(r[i]), vr[i]) : 0.0f;
+        for (int i = 0; i < NH; ++i) rr[i] = t < L ? fmaf(-eg, __uint_as_float(r[i]), vr[i]) : 0.0f;
 #pragma unroll
         for (int q8 = 0; q8 < 2; ++q8) {
           uint4 hi, lo;
@@ -1181,7 +1187,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
 #pragma unroll
       for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
       if (quarter < 2) {  // U-tilde[t][i] = e^{gamma_L - gamma_t} U[t][i]
-        const float f = t < L ? __expf(gL - gsm[t]) : 0.0f;
+        const float f = t < L ? __expf(gsm[64 + t]) : 0.0f;
         float uu[NH];
 #pragma unroll
         for (int i = 0; i < NH; ++i) uu[i] = f * __uint_as_float(r[i]);

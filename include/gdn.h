@@ -235,7 +235,7 @@ int gdn_profile_read(gdn_kernel_time_t* out, int max_entries);
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  *   - Returns GDN_ERR_WORKSPACE, launching nothing, when gdn_prefill_workspace_size(d)
  *     exceeds GDN_NOALLOC_SCRATCH_BYTES (at the pages' model shape, 16 QK / 32 value
- *     heads, one sequence: up to 960 packed tokens with bf16 inputs, 741 with fp32).
+ *     heads, one sequence: up to 960 packed tokens with bf16 inputs, 740 with fp32).
  *   - The first call on a device looks up that device's address of the scratch array
  *     (with that device current); make that first call before any stream capture.  The
  *     address is cached for the life of the process: it assumes the device's primary
