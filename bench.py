@@ -176,7 +176,6 @@ class ClockSampler:
 # The source files each measured kernel is compiled from (its own header and what it includes).
 # Launch configurations live in gdn_api.cu; a change there is re-captured with the kernel's.
 KERNEL_SOURCES = {
-    "prologue_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "chunk_prep_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "chunk_scan_tc_norm": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "decode_multi": ("k_decode_multi.cuh", "gdn_common.cuh"),

@@ -227,15 +227,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
   return f;
 }
 
-// Tensor map of a bf16 stream [T][nheads][128] for the prologue's box of 128 channels x
-// PRO_HG heads x PRO_ROWS tokens (elements outside the tensor read as zeros).
-int make_stream_map(CUtensorMap* m, const void* x, int T, int nheads) {
+// Tensor map of a bf16 stream [T][nheads][128] whose box is 128 channels x box_heads heads x
+// box_rows tokens (elements outside the tensor read as zeros).
+int make_stream_map(CUtensorMap* m, const void* x, int T, int nheads, int box_heads, int box_rows) {
   memset(m, 0, sizeof(*m));
   PFN_cuTensorMapEncodeTiled_v12000 f = encode_tiled();
   if (!f) return GDN_ERR_CUDA;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)nheads, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)nheads * D * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)PRO_HG, (cuuint32_t)PRO_ROWS};
+  const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -258,8 +258,6 @@ int configure_device() {
   if (cudaFuncSetAttribute(k_phaseA_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM) !=
           cudaSuccess ||
       cudaFuncSetAttribute(k_phaseB_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PB_SMEM) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(k_prologue_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PRO_SMEM) !=
           cudaSuccess ||
       cudaFuncSetAttribute(k_chunkprep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_TC_SMEM) !=
           cudaSuccess ||
@@ -401,23 +399,15 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     uint8_t* kq = reinterpret_cast<uint8_t*>(ws + L.kq);
     uint8_t* tp = reinterpret_cast<uint8_t*>(ws + L.tp);
     if (d->total_tokens > 0) {
-      {
-        ProfScope p("prologue_tc", s);
-        const int ngroups = 2 * ((d->h_qk + PRO_HG - 1) / PRO_HG) + (d->h_v + PRO_HG - 1) / PRO_HG;
-        const int nitems = ngroups * 2 * L.max_chunks;
-        const int grid = nitems < g_num_sms ? nitems : g_num_sms;
-        CUtensorMap tm_q, tm_k, tm_v;
-        if (make_stream_map(&tm_q, q, d->total_tokens, d->h_qk) != GDN_OK ||
-            make_stream_map(&tm_k, k, d->total_tokens, d->h_qk) != GDN_OK ||
-            make_stream_map(&tm_v, v, d->total_tokens, d->h_v) != GDN_OK)
-          return GDN_ERR_CUDA;
-        if (launch_dep(k_prologue_tc, dim3(grid), dim3(PRO_THREADS), PRO_SMEM, s, 1, kd, tabc, nitems, tm_q, tm_k,
-                       tm_v, conv_w, kq, F(L.vs)) != cudaSuccess)
-          return GDN_ERR_CUDA;
-      }
       ProfScope p("chunk_prep_tc", s);
-      if (launch_dep(k_chunkprep_tc, dim3(d->h_qk, L.max_chunks), dim3(256), PA_TC_SMEM, s, 1, kd, tabc, a, b, A_log,
-                     dt_bias, (const uint8_t*)kq, tp, F(L.gb)) != cudaSuccess)
+      // raw rows of a chunk with its conv history: one head of q or k, a pair of value heads
+      CUtensorMap tm_q, tm_k, tm_v;
+      if (make_stream_map(&tm_q, q, d->total_tokens, d->h_qk, 1, PF_ROWS) != GDN_OK ||
+          make_stream_map(&tm_k, k, d->total_tokens, d->h_qk, 1, PF_ROWS) != GDN_OK ||
+          make_stream_map(&tm_v, v, d->total_tokens, d->h_v, 2, PF_ROWS) != GDN_OK)
+        return GDN_ERR_CUDA;
+      if (launch_dep(k_chunkprep_tc, dim3(d->h_qk, L.max_chunks), dim3(256), PA_TC_SMEM, s, 1, kd, tabc, tm_q, tm_k,
+                     tm_v, conv_w, a, b, A_log, dt_bias, kq, F(L.vs), tp, F(L.gb)) != cudaSuccess)
         return GDN_ERR_CUDA;
     }
     // The output norm runs inside phase B (clusters of the four slices of a head) unless that
@@ -540,6 +530,11 @@ int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const
   if ((int64_t)d->n_seqs * n_tokens != (int64_t)d->total_tokens) return GDN_ERR_SHAPE;
   gdn_dims_t d1 = *d;
   d1.total_tokens = d->n_seqs;  // one entry per sequence, n_tokens tokens each
+  // One token per sequence is a plain decode step (same layouts): the single-token kernel,
+  // which keeps eight rows of 32 lanes in flight per warp, is the faster one for it.
+  if (n_tokens == 1)
+    return decode_impl(&d1, q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y, nullptr, 0,
+                       stream);
   int rc = check_dims(&d1, true);
   if (rc != GDN_OK) return rc;
   const void* ptrs[] = {q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_state, state, y};
@@ -553,19 +548,20 @@ int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const Dims kd = kdims(&d1);
   const dim3 grid(d->n_seqs, d->h_qk);
+  const size_t smem = decm_smem_bytes(n_tokens, d->h_v / d->h_qk);
   ProfScope p("decode_multi", s);
   if (kd.in_bf16 && kd.out_bf16)
-    k_decode_multi<true, true><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
-                                                           norm_w, conv_state, state, y);
+    k_decode_multi<true, true><<<grid, 256, smem, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                      norm_w, conv_state, state, y);
   else if (kd.in_bf16)
-    k_decode_multi<true, false><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
-                                                            norm_w, conv_state, state, y);
+    k_decode_multi<true, false><<<grid, 256, smem, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                       norm_w, conv_state, state, y);
   else if (kd.out_bf16)
-    k_decode_multi<false, true><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
-                                                            norm_w, conv_state, state, y);
+    k_decode_multi<false, true><<<grid, 256, smem, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                       norm_w, conv_state, state, y);
   else
-    k_decode_multi<false, false><<<grid, 256, DECM_SMEM, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias,
-                                                             conv_w, norm_w, conv_state, state, y);
+    k_decode_multi<false, false><<<grid, 256, smem, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
+                                                        norm_w, conv_state, state, y);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

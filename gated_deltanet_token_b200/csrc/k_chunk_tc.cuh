@@ -16,12 +16,12 @@
 // element, which the scale-invariant output norm amplifies on tokens with a small y_raw;
 // the split keeps the products at ~2^-17 relative error.
 //
-// Prologue (k_prologue_tc, persistent over (head group, half chunk) items): conv + SiLU of
-// q, k, v, L2 norm of q and k; writes the [K;Q] hi/lo operand tile of each (chunk, QK head)
-// and v as fp32 slices.
-// Phase A (k_chunkprep_tc, parallel over chunks x QK heads): [K;Q] K^T on tcgen05; for both
-// value heads of a pair at once: gates, gamma, A, M o QK^T, T = (I + A)^-1 (blocked 16 x 16
-// forward substitution), P = (M o QK^T) T, and the [T;P] hi/lo tiles.
+// Phase A (k_chunkprep_tc, parallel over chunks x QK heads), prologue included: the chunk's
+// raw q, k, v rows by tensor copy; conv + SiLU of q, k, v and the L2 norm of q and k; the
+// [K;Q] hi/lo operand tile of each (chunk, QK head) and v as fp32 slices for phase B;
+// [K;Q] K^T on tcgen05; for both value heads of a pair at once: gates, gamma, A, M o QK^T,
+// T = (I + A)^-1 (blocked 16 x 16 forward substitution), P = (M o QK^T) T, and the [T;P]
+// hi/lo tiles with beta folded into their columns.
 // Phase B (k_chunkscan_tc, sequential over one sequence's chunks, parallel over value
 // heads and 32-row slices of the state): the three MMA rounds above per chunk, with the
 // next chunk's tiles bulk-copied into a second stage while the current one computes, and
@@ -231,246 +231,6 @@ __global__ void __launch_bounds__(128) k_selftest_wait_timeout() {
 }
 
 // ======================================================================================
-// Prologue of the tensor-core path.  Persistent: each CTA walks work items (head group,
-// half chunk) with a stride of the grid size.  A group is up to 8 heads of one stream -- q,
-// k or value heads -- whose slices of a token row are contiguous (2 KB).  The next item's
-// 32 + 3 token rows and conv taps are bulk-copied into the other of two shared-memory stages
-// while the current item is computed, so loads overlap compute: one 3-D tensor copy of the box
-// (128 channels x 8 heads x 35 tokens; heads past the stream's count and tokens outside the
-// tensor read as zeros, tokens of a neighbouring sequence are skipped by the conv) and one
-// bulk copy of the taps.  Warp 0 issues them and leaves the item's description in shared
-// memory for the others.
-// 16 warps: warp w works on head w % 8 of the group and on tokens 16 (w / 8) .. + 15 of the
-// half chunk.
-//   q / k head j: rows 64..127 / 0..63 of the [K;Q] hi/lo tile of QK head j
-//   value head h: v after conv and SiLU as four contiguous 32-column fp32 slices [4][64][32]
-// Width-4 causal conv and SiLU ("Qwen3.8-Flash-Next" technical report, Fig. 2; field
-// guide §02), L2 norm of q and k (Fig. 2).  q/k lanes: token r = lane % 4, 8-channel groups
-// lane / 4 and lane / 4 + 8; the eight lanes of a token reduce the L2 norm with three
-// shuffles and consecutive lanes store consecutive 16-byte chunks.  Every row of a used
-// chunk slot is written (rows past the chunk's length as zeros): phase B multiplies those K
-// rows by zero weights, so stale workspace bits must not survive.
-// ======================================================================================
-constexpr int PRO_HG = 8;                  // heads per work item
-constexpr int PRO_TOK = 32;                // tokens per work item (half a chunk)
-constexpr int PRO_ROWS = PRO_TOK + 3;      // with the conv history
-constexpr int PRO_TSPLIT = 2;              // warps per head of an item (token ranges of 16)
-constexpr int PRO_THREADS = PRO_HG * PRO_TSPLIT * 32;
-constexpr uint32_t PRO_ROWS_BYTES = PRO_ROWS * PRO_HG * D * 2;
-constexpr uint32_t PRO_W_BYTES = PRO_HG * D * 16;
-constexpr uint32_t PRO_STAGE = PRO_ROWS_BYTES + PRO_W_BYTES;
-constexpr size_t PRO_SMEM = 2 * (size_t)PRO_STAGE;
-static_assert(PRO_ROWS <= 256 && PRO_HG <= 256, "tensor-copy box limits");
-
-struct ProItem {
-  ChunkEntry e;
-  int chunk, tb0, stream, h0, nh, nheads;
-  int ch0;  // first conv channel of the group
-};
-
-// Chunk slot of work item `it`.
-__device__ __forceinline__ int pro_chunk(int it, int ngroups) { return (it / ngroups) >> 1; }
-
-// Work item `it`, given its chunk-table entry e = tab[pro_chunk(it, ngroups)].
-__device__ __forceinline__ ProItem pro_item(const Dims& d, const ChunkEntry& e, int it, int ngroups) {
-  ProItem w;
-  const int grp = it % ngroups, hc = it / ngroups;
-  w.chunk = hc >> 1;
-  w.tb0 = (hc & 1) * PRO_TOK;
-  w.e = e;
-  const int hq = d.h_qk, nqg = (hq + PRO_HG - 1) / PRO_HG;
-  w.stream = grp < nqg ? 0 : grp < 2 * nqg ? 1 : 2;
-  w.nheads = w.stream == 2 ? d.h_v : hq;
-  w.h0 = (w.stream == 2 ? grp - 2 * nqg : grp - w.stream * nqg) * PRO_HG;
-  w.nh = min(PRO_HG, w.nheads - w.h0);
-  w.ch0 = w.stream == 0 ? w.h0 * D : w.stream == 1 ? (hq + w.h0) * D : 2 * hq * D + w.h0 * D;
-  return w;
-}
-
-__global__ void __launch_bounds__(PRO_THREADS, 1) k_prologue_tc(Dims d, const ChunkEntry* __restrict__ tab, int nitems,
-                                                        const __grid_constant__ CUtensorMap tm_q,
-                                                        const __grid_constant__ CUtensorMap tm_k,
-                                                        const __grid_constant__ CUtensorMap tm_v,
-                                                        const float* __restrict__ conv_w,
-                                                        uint8_t* __restrict__ kq_ws, float* __restrict__ vs_ws) {
-  tc::grid_dep_wait();  // all earlier work on the stream (the inputs, the last call's use of the workspace) is done
-  tc::grid_dep_launch_dependents();
-  const int hq = d.h_qk, hv = d.h_v;
-  const int ngroups = 2 * ((hq + PRO_HG - 1) / PRO_HG) + (hv + PRO_HG - 1) / PRO_HG;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hw = warp & (PRO_HG - 1), tsplit = warp >> 3;
-  extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t mbar[2];
-  __shared__ ProItem s_item[2];
-  __shared__ int s_abort;
-  if ((tc::smem_u32(sm) & 127u) != 0) {  // tensor copies need 128-byte aligned destinations
-    if (tid == 0) atomicExch(&g_gdn_status, -6);
-    return;
-  }
-  if (tid == 0) {
-    s_abort = 0;
-    tc::mbar_init(tc::smem_u32(&mbar[0]), 1);
-    tc::mbar_init(tc::smem_u32(&mbar[1]), 1);
-    tc::fence_mbar_init();
-  }
-  __syncthreads();
-  // (warp 0, lane 0) describe item `it` (chunk-table entry e) in s_item[st] and issue its
-  // copies into stage `st`.  Unused chunk slots copy nothing.
-  auto issue = [&](int it, const ChunkEntry& e, int st) -> bool {  // true if copies were issued
-    const ProItem w = pro_item(d, e, it, ngroups);
-    s_item[st] = w;
-    if (w.e.len == 0) return false;
-    const uint32_t bar = tc::smem_u32(&mbar[st]);
-    const uint32_t base = tc::smem_u32(sm + (size_t)st * PRO_STAGE);
-    tc::mbar_arrive_expect_tx(bar, PRO_ROWS_BYTES + (uint32_t)w.nh * D * 16);
-    tc::bulk_g2s(base + PRO_ROWS_BYTES, conv_w + (size_t)w.ch0 * 4, (uint32_t)w.nh * D * 16, bar);
-    const CUtensorMap* tm = w.stream == 0 ? &tm_q : w.stream == 1 ? &tm_k : &tm_v;
-    tc::tma_load_3d(base, tm, 0, w.h0, w.e.t0 + w.tb0 - 3, bar);  // rows t - 3 .. of the half chunk
-    return true;
-  };
-  bool pending[2] = {false, false};  // (thread 0) copies in flight per stage
-  // warp 0 reads the table entry of the item after the one it issues next, one item ahead, so
-  // that the load's latency hides behind the current item's work
-  const int g = gridDim.x;
-  ChunkEntry e_next{};
-  if (tid == 0 && (int)blockIdx.x < nitems) {
-    pending[0] = issue(blockIdx.x, chunk_entry(tab, d.total_tokens, pro_chunk(blockIdx.x, ngroups)), 0);
-    if ((int)blockIdx.x + g < nitems) e_next = chunk_entry(tab, d.total_tokens, pro_chunk(blockIdx.x + g, ngroups));
-  }
-  __syncthreads();
-  uint32_t parity[2] = {0, 0};
-  int n = 0;
-  for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
-    const int st = n & 1;
-    const ProItem w = s_item[st];
-    if (tid == 0 && it + g < nitems) {
-      pending[st ^ 1] = issue(it + g, e_next, st ^ 1);
-      if (it + 2 * g < nitems) e_next = chunk_entry(tab, d.total_tokens, pro_chunk(it + 2 * g, ngroups));
-    }
-    if (w.e.len == 0) {
-      __syncthreads();
-      continue;
-    }
-    if (!tc::mbar_wait(tc::smem_u32(&mbar[st]), parity[st])) s_abort = 1;
-    parity[st] ^= 1;
-    if (tid == 0) pending[st] = false;
-    __syncthreads();  // the abort decision is uniform
-    if (s_abort) break;
-    const uint8_t* base = sm + (size_t)st * PRO_STAGE;
-    const float4* wsm = reinterpret_cast<const float4*>(base + PRO_ROWS_BYTES) + hw * D;
-    const uint16_t* hrow = reinterpret_cast<const uint16_t*>(base) + (size_t)hw * D;  // this head in a row
-    const int L = w.e.len, tb0 = w.tb0, nh = w.nh, head = w.h0 + hw;
-    auto row_ok = [&](int r) {  // smem row r holds a token inside the sequence and the chunk
-      const int tcr = tb0 - 3 + r;
-      return tcr < L && (long)w.e.t0 + tcr >= w.e.seq_start;
-    };
-    if (hw < nh) {
-      if (w.stream < 2) {
-        // lane: token r = lane % 4 of a 4-token block, channel groups g0 = lane / 4 and g0 + 8
-        const int r = lane & 3, g0 = lane >> 2;
-        uint8_t* tile = kq_ws + ((size_t)w.chunk * hq + head) * KQ_BYTES;
-        const float scale = w.stream == 0 ? d.q_scale : 1.0f;
-#pragma unroll 1
-        for (int blk = tsplit * (PRO_TOK / PRO_TSPLIT); blk < (tsplit + 1) * (PRO_TOK / PRO_TSPLIT); blk += 4) {
-          const int t = tb0 + blk + r;  // chunk-relative token
-          float acc[2][8];
-          bool okt[4];
-#pragma unroll
-          for (int tap = 0; tap < 4; ++tap) okt[tap] = row_ok(blk + r + tap);  // row of token t - 3 + tap
-#pragma unroll
-          for (int gi = 0; gi < 2; ++gi) {
-            const int cg = (g0 + 8 * gi) * 8;
-            uint32_t xw[4][4];  // the four tap rows' 8 channels (bf16 pairs); zero outside the sequence
-#pragma unroll
-            for (int tap = 0; tap < 4; ++tap) {
-              const uint4 x = okt[tap] ? *reinterpret_cast<const uint4*>(hrow + (size_t)(blk + r + tap) * PRO_HG * D + cg)
-                                       : make_uint4(0, 0, 0, 0);
-              xw[tap][0] = x.x; xw[tap][1] = x.y; xw[tap][2] = x.z; xw[tap][3] = x.w;
-            }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float4 w4 = wsm[cg + c];  // channel cg + c, taps 0..3
-              float a_ = 0.0f;
-#pragma unroll
-              for (int tap = 0; tap < 4; ++tap)
-                a_ = fmaf(comp(w4, tap), bf2f(c & 1 ? xw[tap][c >> 1] >> 16 : xw[tap][c >> 1] & 0xffffu), a_);
-              acc[gi][c] = a_;
-            }
-          }
-          float ss0 = 0.0f, ss1 = 0.0f;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            acc[0][c] = silu_fast(acc[0][c]);
-            acc[1][c] = silu_fast(acc[1][c]);
-            ss0 = fmaf(acc[0][c], acc[0][c], ss0);
-            ss1 = fmaf(acc[1][c], acc[1][c], ss1);
-          }
-          float sst = ss0 + ss1;
-          sst += __shfl_xor_sync(0xffffffffu, sst, 4);
-          sst += __shfl_xor_sync(0xffffffffu, sst, 8);
-          sst += __shfl_xor_sync(0xffffffffu, sst, 16);
-          const float inv = t < L ? scale * rsqrtf(sst + d.l2_eps) : 0.0f;
-          const int row = (w.stream == 0 ? 64 : 0) + t;
-#pragma unroll
-          for (int gi = 0; gi < 2; ++gi) {
-            float x8[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) x8[c] = acc[gi][c] * inv;
-            uint4 hi, lo;
-            tc::split8(x8, hi, lo);
-            const uint32_t off = kmaj128(row, (g0 + 8 * gi) * 8);
-            *reinterpret_cast<uint4*>(tile + off) = hi;
-            *reinterpret_cast<uint4*>(tile + KQ_TILE + off) = lo;
-          }
-        }
-      } else {
-        const int c0 = lane * 4;
-        float wv[4][4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float4 t4 = wsm[c0 + c];
-          wv[c][0] = t4.x; wv[c][1] = t4.y; wv[c][2] = t4.z; wv[c][3] = t4.w;
-        }
-        float* out = vs_ws + ((size_t)w.chunk * hv + head) * (VS_BYTES / 4) + (size_t)(c0 / TC_NV) * (VS_SLICE / 4) +
-                     (c0 % TC_NV);
-#pragma unroll 1
-        for (int blk = tsplit * (PRO_TOK / PRO_TSPLIT); blk < (tsplit + 1) * (PRO_TOK / PRO_TSPLIT); blk += 8) {
-          uint2 x[11];  // raw bf16 of 4 channels, rows t - 3 .. t + 7
-#pragma unroll
-          for (int p = 0; p < 11; ++p) {
-            const int rr = blk + p;
-            x[p] = row_ok(rr) ? *reinterpret_cast<const uint2*>(hrow + (size_t)rr * PRO_HG * D + c0) : make_uint2(0, 0);
-          }
-          auto xv = [&](int p, int c) {
-            const uint32_t wd = c < 2 ? x[p].x : x[p].y;
-            return bf2f(c & 1 ? wd >> 16 : wd & 0xffffu);
-          };
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int t = tb0 + blk + i;
-            float r4[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float acc = fmaf(wv[c][3], xv(i + 3, c),
-                                     fmaf(wv[c][2], xv(i + 2, c), fmaf(wv[c][1], xv(i + 1, c), wv[c][0] * xv(i, c))));
-              r4[c] = t < L ? silu_fast(acc) : 0.0f;
-            }
-            *reinterpret_cast<float4*>(out + t * TC_NV) = make_float4(r4[0], r4[1], r4[2], r4[3]);
-          }
-        }
-      }
-    }
-    tc::fence_proxy_async();
-    __syncthreads();  // this stage is free for the item after next
-  }
-  if (s_abort && tid == 0) {  // record, and let copies still in flight land (bounded) before leaving
-    atomicExch(&g_gdn_status, -7);
-    for (int q2 = 0; q2 < 2; ++q2)
-      if (pending[q2]) (void)tc::mbar_wait(tc::smem_u32(&mbar[q2]), parity[q2]);
-  }
-}
-
-// ======================================================================================
 // Phase A
 // ======================================================================================
 constexpr int PA_P = 68;  // pitch (floats) of the fp32 64 x 64 matrices of phase A
@@ -490,19 +250,40 @@ constexpr size_t PA_TC_SMEM = PA_OFF_W + 16 * 16 * 16;
 static_assert(PA_OFF_T >= KQ_BYTES, "T and the gates lie past the [K;Q] tile");
 static_assert(PA_TC_SMEM <= 113 * 1024, "two phase-A CTAs per SM");
 
-// One CTA per (QK head j, chunk); value heads of QK head j in pairs (a, b), both heads of a
-// pair at once: A, M o QK^T, T = (I + A)^-1 and P = (M o QK^T) T.  Field guide §02 defines
-// the per-token steps these chunk quantities regroup.
+// Raw rows of one chunk with its conv history (tokens t0 - 3 .. t0 + 63), as the tensor
+// copies land them: [row][heads][128] bf16.  q and k of the QK head (one head each) and, later,
+// a value-head pair (two heads) share the space of the T matrices, which the solve fills only
+// after the raw rows have been consumed; the conv taps of two heads use the solve's scratch.
+constexpr int PF_ROWS = CH + 3;
+constexpr uint32_t PF_HEAD_BYTES = PF_ROWS * D * 2;  // one head's raw rows: 17,152 B
+constexpr uint32_t PF_OFF_QRAW = PA_OFF_T;
+constexpr uint32_t PF_OFF_KRAW = PA_OFF_T + PF_HEAD_BYTES;
+constexpr uint32_t PF_OFF_VRAW = PA_OFF_T;
+constexpr uint32_t PF_OFF_TAPS = PA_OFF_W;
+static_assert(PA_OFF_T + 2 * PF_HEAD_BYTES <= PA_OFF_G, "raw rows fit in the T matrices' space");
+static_assert(PA_OFF_W + 2 * D * 16 <= PA_TC_SMEM, "conv taps of two heads fit in the solve scratch");
+static_assert(PF_OFF_QRAW % 128 == 0 && PF_OFF_KRAW % 128 == 0 && PF_OFF_TAPS % 16 == 0,
+              "tensor-copy destinations are 128-byte aligned");
+static_assert(PF_ROWS <= 256, "tensor-copy box limit");
+
+// One CTA per (QK head j, chunk), prologue included: the chunk's raw q and k rows (with three
+// rows of conv history) arrive by tensor copy; the width-4 causal conv, SiLU and L2 norm
+// ("Qwen3.8-Flash-Next" technical report, Fig. 2; field guide §02) build the [K;Q] hi/lo
+// operand tile in shared memory, which is stored once for phase B.  Then, for the value heads
+// of QK head j in pairs (a, b), both heads of a pair at once: conv + SiLU of v (fp32 slices for
+// phase B), the gates, A, M o QK^T, T = (I + A)^-1 and P = (M o QK^T) T.  Field guide §02
+// defines the per-token steps these chunk quantities regroup.
 __global__ void __launch_bounds__(256, 2)
-    k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const float* __restrict__ a,
+    k_chunkprep_tc(Dims d, const ChunkEntry* __restrict__ tab, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const float* __restrict__ conv_w, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
-                   const float* __restrict__ dt_bias, const uint8_t* __restrict__ kq_ws,
+                   const float* __restrict__ dt_bias, uint8_t* __restrict__ kq_ws, float* __restrict__ vs_ws,
                    uint8_t* __restrict__ tp_ws, float* __restrict__ gb_ws) {
-  tc::grid_dep_wait();  // the prologue's tiles are complete
+  tc::grid_dep_wait();  // all earlier work on the stream (the inputs, the last call's use of the workspace) is done
   tc::grid_dep_launch_dependents();
-  // head-fastest grid, chunks from the last: the prologue writes its tiles in chunk order, so
-  // the ones it wrote last are still in L2 when they are read here first, and the early
-  // chunks' [T;P] tiles (written here last) are in L2 when phase B starts on them
+  // head-fastest grid, chunks from the last: the early chunks' tiles, written last, are still in
+  // L2 when phase B starts on them
   const int chunk = gridDim.y - 1 - blockIdx.y;
   const ChunkEntry e = chunk_entry(tab, d.total_tokens, chunk);
   if (e.len == 0) return;
@@ -520,13 +301,20 @@ __global__ void __launch_bounds__(256, 2)
   double* gs = reinterpret_cast<double*>(sm + PA_OFF_G);               // [2][64] gamma (fp64)
   float* bs = reinterpret_cast<float*>(sm + PA_OFF_G + 2 * 64 * 8);   // [2][64] beta
   float4* wsc = reinterpret_cast<float4*>(sm + PA_OFF_W) + (tid >> 4) * 16;  // this half-warp's rows
-  __shared__ uint64_t mbar;
+  const float4* taps = reinterpret_cast<const float4*>(sm + PF_OFF_TAPS);   // [2][128] conv taps
+  __shared__ uint64_t mbar;     // MMA completions
+  __shared__ uint64_t mbar_ld;  // tensor / bulk copies of raw rows and taps
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
 
+  if ((tc::smem_u32(sm) & 127u) != 0) {  // tensor copies need 128-byte aligned destinations
+    if (tid == 0) atomicExch(&g_gdn_status, -6);
+    return;
+  }
   if (tid == 0) {
     s_abort = 0;
     tc::mbar_init(tc::smem_u32(&mbar), 1);
+    tc::mbar_init(tc::smem_u32(&mbar_ld), 1);
     tc::fence_mbar_init();
   }
   if (warp == 0) {
@@ -537,12 +325,32 @@ __global__ void __launch_bounds__(256, 2)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = tslot;
-  if (tid == 0) {  // the [K;Q] tile written by the prologue
-    const uint32_t bar = tc::smem_u32(&mbar);
-    tc::mbar_arrive_expect_tx(bar, KQ_BYTES);
-    tc::bulk_g2s(tc::smem_u32(sm), kq_ws + ((size_t)chunk * hq + j) * KQ_BYTES, KQ_BYTES, bar);
-  }
-  uint32_t mma_phase = 0;
+  // (thread 0) raw rows of two heads of one stream and their conv taps into the raw space
+  int ld_issued = 0, ld_waited = 0;  // armings of mbar_ld (thread 0) and waits on it (every thread)
+  auto issue_raw = [&](const CUtensorMap* tm0, int head0, const CUtensorMap* tm1, int head1, int ch0, int ch1,
+                       uint32_t box_bytes) {
+    const uint32_t bar = tc::smem_u32(&mbar_ld);
+    ++ld_issued;
+    tc::mbar_arrive_expect_tx(bar, box_bytes + (ch1 >= 0 ? 2u : 1u) * D * 16);
+    tc::tma_load_3d(tc::smem_u32(sm + PF_OFF_QRAW), tm0, 0, head0, e.t0 - 3, bar);
+    if (tm1) tc::tma_load_3d(tc::smem_u32(sm + PF_OFF_KRAW), tm1, 0, head1, e.t0 - 3, bar);
+    tc::bulk_g2s(tc::smem_u32(sm + PF_OFF_TAPS), conv_w + (size_t)ch0 * 4, D * 16, bar);
+    if (ch1 >= 0) tc::bulk_g2s(tc::smem_u32(sm + PF_OFF_TAPS) + D * 16, conv_w + (size_t)ch1 * 4, D * 16, bar);
+  };
+  // the value-head pair starting at head index g0 of QK head j (the second head's taps only if
+  // it exists: its box rows past the tensor read as zeros)
+  auto issue_v = [&](int g0) {
+    const int h0 = j * G + g0;
+    issue_raw(&tm_v, h0, nullptr, 0, 2 * hq * D + h0 * D, g0 + 1 < G ? 2 * hq * D + (h0 + 1) * D : -1,
+              2 * PF_HEAD_BYTES);
+  };
+  if (tid == 0) issue_raw(&tm_q, j, &tm_k, j, j * D, (hq + j) * D, 2 * PF_HEAD_BYTES);
+  uint32_t ld_phase = 0, mma_phase = 0;
+  // raw row rr holds token t0 - 3 + rr: usable if inside the chunk and the sequence
+  auto row_ok = [&](int rr) {
+    const int tcr = rr - 3;
+    return tcr < L && e.t0 + tcr >= e.seq_start;
+  };
   bool aborted = false;
   for (int ga = 0; ga < G; ga += 2) {
     const int gpair[2] = {ga, ga + 1 < G ? ga + 1 : ga};
@@ -579,11 +387,84 @@ __global__ void __launch_bounds__(256, 2)
         gbw[64 + lane] = (float)(gL - g0); gbw[96 + lane] = (float)(gL - g1);
       }
     }
-    if (ga == 0) {  // [K;Q] K^T once the tile is in (the gates above overlapped the copy)
-      if (!tc::mbar_wait(tc::smem_u32(&mbar), 0)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
-      __syncthreads();
+    if (ga == 0) {
+      // ---- prologue: conv + SiLU + L2 norm of k (warps 0..3) and q (warps 4..7) into the
+      // [K;Q] tile; lane: token r = lane % 4 of a four-token block, channel groups g0 = lane / 4
+      // and g0 + 8; the eight lanes of a token reduce its norm with three shuffles
+      const bool okl = tc::mbar_wait(tc::smem_u32(&mbar_ld), ld_phase);
+      ld_phase ^= 1;
+      ++ld_waited;
+      if (!okl) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+      if (okl) {
+        const int isq = warp >> 2;
+        const uint16_t* raw = reinterpret_cast<const uint16_t*>(sm + (isq ? PF_OFF_QRAW : PF_OFF_KRAW));
+        const float4* wsm = taps + (isq ? 0 : D);
+        const int r = lane & 3, g0 = lane >> 2;
+        const float scale = isq ? d.q_scale : 1.0f;
+#pragma unroll 1
+        for (int blk = (warp & 3) * 16; blk < (warp & 3) * 16 + 16; blk += 4) {
+          const int t = blk + r;  // chunk-relative token; its taps read raw rows t .. t + 3
+          float acc[2][8];
+          bool okt[4];
+#pragma unroll
+          for (int tap = 0; tap < 4; ++tap) okt[tap] = row_ok(t + tap);
+#pragma unroll
+          for (int gi = 0; gi < 2; ++gi) {
+            const int cg = (g0 + 8 * gi) * 8;
+            uint32_t xw[4][4];
+#pragma unroll
+            for (int tap = 0; tap < 4; ++tap) {
+              const uint4 x = okt[tap] ? *reinterpret_cast<const uint4*>(raw + (size_t)(t + tap) * D + cg)
+                                       : make_uint4(0, 0, 0, 0);
+              xw[tap][0] = x.x; xw[tap][1] = x.y; xw[tap][2] = x.z; xw[tap][3] = x.w;
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 w4 = wsm[cg + c];  // channel cg + c, taps 0..3
+              float a_ = 0.0f;
+#pragma unroll
+              for (int tap = 0; tap < 4; ++tap)
+                a_ = fmaf(comp(w4, tap), bf2f(c & 1 ? xw[tap][c >> 1] >> 16 : xw[tap][c >> 1] & 0xffffu), a_);
+              acc[gi][c] = a_;
+            }
+          }
+          float ss0 = 0.0f, ss1 = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            acc[0][c] = silu_fast(acc[0][c]);
+            acc[1][c] = silu_fast(acc[1][c]);
+            ss0 = fmaf(acc[0][c], acc[0][c], ss0);
+            ss1 = fmaf(acc[1][c], acc[1][c], ss1);
+          }
+          float sst = ss0 + ss1;
+          sst += __shfl_xor_sync(0xffffffffu, sst, 4);
+          sst += __shfl_xor_sync(0xffffffffu, sst, 8);
+          sst += __shfl_xor_sync(0xffffffffu, sst, 16);
+          const float inv = t < L ? scale * rsqrtf(sst + d.l2_eps) : 0.0f;
+          const int row = (isq ? 64 : 0) + t;
+#pragma unroll
+          for (int gi = 0; gi < 2; ++gi) {
+            float x8[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) x8[c] = acc[gi][c] * inv;
+            uint4 hi, lo;
+            tc::split8(x8, hi, lo);
+            const uint32_t off = kmaj128(row, (g0 + 8 * gi) * 8);
+            *reinterpret_cast<uint4*>(kq_hi + off) = hi;
+            *reinterpret_cast<uint4*>(kq_lo + off) = lo;
+          }
+        }
+      }
+      tc::fence_proxy_async();  // the tile's generic stores, for the MMA and the bulk store
+      tc::tc_fence_before();
+      __syncthreads();          // the tile is complete and the raw q / k rows are consumed
       tc::tc_fence_after();
       if (tid == 0 && !s_abort) {
+        // the tile for phase B, then the first value pair's raw rows into the freed raw space
+        tc::bulk_s2g(kq_ws + ((size_t)chunk * hq + j) * KQ_BYTES, tc::smem_u32(sm), KQ_BYTES);
+        tc::bulk_commit();
+        issue_v(0);
+        // [K;Q] K^T (the gates above overlapped the raw copies)
         constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
         const uint64_t dd[2] = {tc::sdesc(tc::smem_u32(kq_hi), LBO128, 128), tc::sdesc(tc::smem_u32(kq_lo), LBO128, 128)};
 #pragma unroll
@@ -595,8 +476,11 @@ __global__ void __launch_bounds__(256, 2)
           }
         tc::umma_commit(tc::smem_u32(&mbar));
       }
-      if (!s_abort && !tc::mbar_wait(tc::smem_u32(&mbar), 1)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+      if (!s_abort && !tc::mbar_wait(tc::smem_u32(&mbar), mma_phase)) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+      mma_phase ^= 1;
       tc::tc_fence_after();
+      // the A matrices below overwrite the tile's lo half: the bulk store must have read it
+      if (tid == 0) tc::bulk_wait_read_all();
     }
     __syncthreads();
     aborted = s_abort != 0;
@@ -646,6 +530,54 @@ __global__ void __launch_bounds__(256, 2)
       }
     }
     __syncthreads();
+    // ---- v of the pair: conv + SiLU as four contiguous 32-column fp32 slices per head for
+    // phase B.  Warp w: head w / 4 of the pair, tokens 16 (w % 4) .. + 15 in two blocks of
+    // eight (raw rows blk .. blk + 10); lane: channels 4 lane .. 4 lane + 3.  Rows past the
+    // chunk's length are written as zeros.
+    {
+      const bool okv = tc::mbar_wait(tc::smem_u32(&mbar_ld), ld_phase);
+      ld_phase ^= 1;
+      ++ld_waited;
+      if (!okv) { s_abort = 1; atomicExch(&g_gdn_status, -7); }
+      const int hp = warp >> 2;
+      if (okv && (hp == 0 || gpair[1] != gpair[0])) {
+        const int h = j * G + gpair[hp], c0 = lane * 4;
+        const uint16_t* hrow = reinterpret_cast<const uint16_t*>(sm + PF_OFF_VRAW) + hp * D;  // row stride 2 D
+        float wv[4][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 t4 = taps[hp * D + c0 + c];
+          wv[c][0] = t4.x; wv[c][1] = t4.y; wv[c][2] = t4.z; wv[c][3] = t4.w;
+        }
+        float* out = vs_ws + ((size_t)chunk * hv + h) * (VS_BYTES / 4) + (size_t)(c0 / TC_NV) * (VS_SLICE / 4) +
+                     (c0 % TC_NV);
+#pragma unroll 1
+        for (int blk = (warp & 3) * 16; blk < (warp & 3) * 16 + 16; blk += 8) {
+          uint2 x[11];  // raw bf16 of the 4 channels, rows blk .. blk + 10 (tokens blk - 3 .. blk + 7)
+#pragma unroll
+          for (int p = 0; p < 11; ++p)
+            x[p] = row_ok(blk + p) ? *reinterpret_cast<const uint2*>(hrow + (size_t)(blk + p) * 2 * D + c0)
+                                   : make_uint2(0, 0);
+          auto xv = [&](int p, int c) {
+            const uint32_t wd = c < 2 ? x[p].x : x[p].y;
+            return bf2f(c & 1 ? wd >> 16 : wd & 0xffffu);
+          };
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int t = blk + i;
+            float r4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float acc = fmaf(wv[c][3], xv(i + 3, c),
+                                     fmaf(wv[c][2], xv(i + 2, c), fmaf(wv[c][1], xv(i + 1, c), wv[c][0] * xv(i, c))));
+              r4[c] = t < L ? silu_fast(acc) : 0.0f;
+            }
+            *reinterpret_cast<float4*>(out + t * TC_NV) = make_float4(r4[0], r4[1], r4[2], r4[3]);
+          }
+        }
+      }
+    }
+    __syncthreads();  // the raw v rows and taps are consumed before the solve writes over them
     // T = (I + A)^-1 by 16 x 16 blocks: diagonal blocks by forward substitution (thread =
     // head, block, column; rows of A read as float4) ...
     if (tid < 128) {
@@ -785,6 +717,14 @@ __global__ void __launch_bounds__(256, 2)
     }
     tc::tc_fence_before();
     __syncthreads();
+    // the next pair's raw v rows: the T matrices and the solve scratch are free again
+    if (tid == 0 && ga + 2 < G && !s_abort) issue_v(ga + 2);
+  }
+  if (tid == 0) {
+    tc::bulk_wait_all();  // the [K;Q] tile's bulk store has completed
+    // after a timeout, let raw copies still in flight land (bounded): every arming of mbar_ld
+    // but possibly the last was waited on, and the last completes the phase of parity ld_phase
+    if (s_abort && ld_issued > ld_waited) (void)tc::mbar_wait(tc::smem_u32(&mbar_ld), ld_phase);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -909,11 +849,13 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
         : "memory");
     return r != 0;
   };
-  // A bounded wait that records a timeout.  Once any thread has recorded one, later waits of
-  // the CTA return at once (the barriers they wait on may never complete) and no new MMA or
-  // copy is issued, so the CTA reaches its next chunk barrier, and leaves, within one limit.
+  // A bounded wait that records a timeout.  Once any thread has recorded one, a later wait of
+  // the CTA that does not complete at its first try returns at once (its barrier may never
+  // complete), and the MMA thread issues no round after a failed wait, so the CTA reaches its
+  // next chunk barrier, and leaves, within one limit.  The flag is read only off the fast path.
   auto aborted_now = [&]() { return *static_cast<volatile int*>(&s_abort) != 0; };
   auto wait_ok = [&](uint64_t& bar, uint32_t parity) -> bool {
+    if (tc::mbar_try_wait(tc::smem_u32(&bar), parity)) return true;
     if (aborted_now()) return false;
     if (tc::mbar_wait(tc::smem_u32(&bar), parity)) return true;
     s_abort = 1;
@@ -1119,7 +1061,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     // arrived ends the loop for every thread at the same chunk
     if (loop_sync_or(aborted_now())) { aborted = true; break; }
     // ---- round 1: [K S^T ; Q S^T] = [K;Q] (128 x 128) x S^T (K = 128, N = nv) -------------
-    if (tid == 0 && !aborted_now()) {
+    if (tid == 0) {
       tc::tc_fence_after();
       const uint64_t da[2] = {tc::sdesc(kq0, LBO128, 128), tc::sdesc(kq0 + KQ_TILE, LBO128, 128)};
 #pragma unroll
@@ -1134,7 +1076,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       issue_load(c + 1, st ^ 1);
       last_load = c + 1;
     }
-    (void)wait_ok(mbar_mma[0], ph_mma);
+    const bool ok1 = wait_ok(mbar_mma[0], ph_mma);
     tc::tc_fence_after();
     float qs[NH];  // y rows (separate-epilogue mode): e^{gamma_t} (Q S^T)[t][:]
     if (rwarp || (!FUSED && worker)) {
@@ -1165,7 +1107,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     tc::tc_fence_before();
     if (rwarp) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 2: [U ; (M o QK^T) U] = [T;P] (128 x 64) x R (K = 64, N = nv) ----------------
-    if (tid == 0 && !aborted_now()) {
+    if (tid == 0 && ok1) {
       tc::tc_fence_after();
       const uint64_t da[2] = {tc::sdesc(tp0, LBO128, 128), tc::sdesc(tp0 + TP_TILE, LBO128, 128)};
       const uint64_t db = tc::sdesc(tc::smem_u32(r_hi), 128, 8 * 128);
@@ -1177,7 +1119,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       }
       tc::umma_commit(tc::smem_u32(&mbar_mma[1]));
     }
-    (void)wait_ok(mbar_mma[1], ph_mma);
+    const bool ok2 = wait_ok(mbar_mma[1], ph_mma);
     tc::tc_fence_after();
     if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
@@ -1213,7 +1155,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     tc::tc_fence_before();
     if (rwarp) named_bar_sync(1, 128);  // the R / U-tilde writers and the MMA thread
     // ---- round 3: K^T U-tilde: A = MN-major view of the K rows (M = 128 key comps, K = 64 tokens)
-    if (tid == 0 && !aborted_now()) {
+    if (tid == 0 && ok2) {
       tc::tc_fence_after();
       const uint64_t da[2] = {tc::sdesc(kq0, 128, LBO128), tc::sdesc(kq0 + KQ_TILE, 128, LBO128)};
       const uint64_t db = tc::sdesc(tc::smem_u32(r_hi), 128, 8 * 128);

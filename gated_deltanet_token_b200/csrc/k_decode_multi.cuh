@@ -5,15 +5,29 @@
 // tokens, so each 512-byte row is read once and written once per call instead of once per
 // token.  Conv: the K new raw rows follow the three history rows; the history keeps the last
 // three raw rows.  One CTA per (sequence n, QK head j) as in k_decode.
+//
+// Row layout: eight lanes share a state row, each holding four groups of four columns
+// (columns 32 c + 4 (lane % 8) .. + 3, c = 0..3, so that every 16-byte load of the eight lanes
+// covers 128 contiguous bytes of the row).  A warp works on four rows at once, and the two dot
+// products of a token (S'k and S'q) reduce over eight lanes in three shuffle levels -- for four
+// rows together.  Two such four-row slabs are in flight per warp (8 rows, 4 KB of state).
 #pragma once
 #include "gdn_common.cuh"
 
 namespace gdn {
 
 constexpr int DECM_KMAX = 8;
-constexpr int DECM_ROWS = 4;  // state rows in flight per warp (x K tokens of dot products)
+constexpr int DECM_LPR = 8;             // lanes per state row
+constexpr int DECM_CPL = D / DECM_LPR;  // columns per lane: 16
+constexpr int DECM_SLABS = 2;           // four-row slabs in flight per warp
 
-// smem: q, k [KMAX][D]; v, y [KMAX][GMAX=8][D]; gates [KMAX][8] x 2; kq [KMAX]
+// Dynamic shared memory of one CTA (floats): q, k [K][D]; v, y [K][G][D]; alpha, beta [K][G];
+// k . q [K].
+__host__ __device__ constexpr size_t decm_smem_bytes(int K, int G) {
+  return (size_t)(2 * K * D + 2 * K * G * D + 2 * K * G + K) * sizeof(float);
+}
+constexpr size_t DECM_SMEM = decm_smem_bytes(DECM_KMAX, 8);
+
 template <bool BF16, bool OUT_BF16>
 __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void* __restrict__ q,
                                                       const void* __restrict__ k, const void* __restrict__ v,
@@ -28,18 +42,18 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
   const int hq = d.h_qk, hv = d.h_v, G = hv / hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t cconv = (size_t)(2 * hq + hv) * D;
-  extern __shared__ __align__(16) float dm[];
-  float* qs = dm;                                 // [KMAX][D]
-  float* ks = qs + DECM_KMAX * D;                 // [KMAX][D]
-  float* vs = ks + DECM_KMAX * D;                 // [KMAX][8][D]
-  float* ys = vs + DECM_KMAX * 8 * D;             // [KMAX][8][D]
-  float* al = ys + DECM_KMAX * 8 * D;             // [KMAX][8]
-  float* be = al + DECM_KMAX * 8;                 // [KMAX][8]
-  float* kqv = be + DECM_KMAX * 8;                // [KMAX]
   if (K < 1 || K > DECM_KMAX || G > 8) {
     if (tid == 0) atomicExch(&g_gdn_status, -6);
     return;
   }
+  extern __shared__ __align__(16) float dm[];
+  float* qs = dm;                 // [K][D]
+  float* ks = qs + K * D;         // [K][D]
+  float* vs = ks + K * D;         // [K][G][D]
+  float* ys = vs + K * G * D;     // [K][G][D]
+  float* al = ys + K * G * D;     // [K][G]  e^{g}
+  float* be = al + K * G;         // [K][G]  beta
+  float* kqv = be + K * G;        // [K]     k_t . q_t
 
   // conv + SiLU for the K tokens over this CTA's channels; the history becomes the last
   // three raw rows of (history, new rows), copied exactly
@@ -69,7 +83,7 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
       src = static_cast<const E*>(v) + ((size_t)n * K * hv + hh) * D + cc;
       stride = (size_t)hv * D;
       dst = vs + g * D + cc;
-      dstride = 8 * D;
+      dstride = G * D;
     }
     const float4 w = *reinterpret_cast<const float4*>(conv_w + ch * 4);
     E win[3] = {cs[ch], cs[cconv + ch], cs[2 * cconv + ch]};  // x_{-3}, x_{-2}, x_{-1}
@@ -91,8 +105,8 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
   for (int i = tid; i < K * G; i += blockDim.x) {
     const int t = i / G, g = i % G, hh = j * G + g;
     const size_t o = ((size_t)n * K + t) * hv + hh;
-    al[t * 8 + g] = expf(decay_gate_f(a[o], A_log[hh], dt_bias[hh]));
-    be[t * 8 + g] = sigmoid_f(b[o]);
+    al[i] = expf(decay_gate_f(a[o], A_log[hh], dt_bias[hh]));
+    be[i] = sigmoid_f(b[o]);
   }
   __syncthreads();
   for (int i = warp; i < 2 * K; i += 8) {  // L2 norms: q_t (times q_scale) and k_t
@@ -113,40 +127,67 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
   }
   __syncthreads();
 
-  // state rows: an equal contiguous share per warp, DECM_ROWS in flight, K tokens each
+  // State rows: an equal contiguous share of the CTA's G * 128 rows per warp (a multiple of 16),
+  // DECM_SLABS four-row slabs at a time.  Lane: row sub = lane / 8 of a slab, columns
+  // 32 c4 + cl .. + 3 for c4 = 0..3.  Per token, for each row i of value head g:
+  //   S' = alpha S;  r_k = S' k;  e = beta (v_i - r_k);  S'' = S' + e k^T;  y_i = S'' q
+  // with y_i = alpha (S q) + e (k . q).
+  const int sub = lane >> 3, cl = (lane & 7) * 4;
   const int rows_per_warp = G * D / 8;
   const size_t state0 = ((size_t)n * hv + (size_t)j * G) * D * D;
-  for (int r0 = warp * rows_per_warp; r0 < (warp + 1) * rows_per_warp; r0 += DECM_ROWS) {
-    float4 s[DECM_ROWS];
+  for (int r0 = warp * rows_per_warp; r0 < (warp + 1) * rows_per_warp; r0 += 4 * DECM_SLABS) {
+    float4 s[DECM_SLABS][DECM_CPL / 4];
 #pragma unroll
-    for (int u = 0; u < DECM_ROWS; ++u)
-      s[u] = __ldcs(reinterpret_cast<const float4*>(state + state0 + (size_t)(r0 + u) * D + lane * 4));
+    for (int sl = 0; sl < DECM_SLABS; ++sl) {
+      const float4* src = reinterpret_cast<const float4*>(state + state0 + (size_t)(r0 + 4 * sl + sub) * D + cl);
+#pragma unroll
+      for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) s[sl][c4] = __ldcs(src + 8 * c4);
+    }
     for (int t = 0; t < K; ++t) {
-      const float4 kr = *reinterpret_cast<const float4*>(ks + t * D + lane * 4);
-      const float4 qr = *reinterpret_cast<const float4*>(qs + t * D + lane * 4);
+      float4 kr[DECM_CPL / 4], qr[DECM_CPL / 4];
+#pragma unroll
+      for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) {
+        kr[c4] = *reinterpret_cast<const float4*>(ks + t * D + 32 * c4 + cl);
+        qr[c4] = *reinterpret_cast<const float4*>(qs + t * D + 32 * c4 + cl);
+      }
       const float kq = kqv[t];
 #pragma unroll
-      for (int u = 0; u < DECM_ROWS; ++u) {
-        const int row = r0 + u, g = row / D, i = row % D;
-        const float rk = warp_sum(dot4(s[u], kr));
-        const float rq = warp_sum(dot4(s[u], qr));
-        const float a_ = al[t * 8 + g];
-        const float e = be[t * 8 + g] * (vs[(t * 8 + g) * D + i] - a_ * rk);
-        s[u].x = fmaf(a_, s[u].x, e * kr.x);
-        s[u].y = fmaf(a_, s[u].y, e * kr.y);
-        s[u].z = fmaf(a_, s[u].z, e * kr.z);
-        s[u].w = fmaf(a_, s[u].w, e * kr.w);
-        if (lane == 0) ys[(t * 8 + g) * D + i] = fmaf(a_, rq, e * kq);
+      for (int sl = 0; sl < DECM_SLABS; ++sl) {
+        float rk = 0.0f, rq = 0.0f;
+#pragma unroll
+        for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) {
+          rk += dot4(s[sl][c4], kr[c4]);
+          rq += dot4(s[sl][c4], qr[c4]);
+        }
+#pragma unroll
+        for (int o = 1; o < DECM_LPR; o <<= 1) {  // the eight lanes of the row
+          rk += __shfl_xor_sync(0xffffffffu, rk, o);
+          rq += __shfl_xor_sync(0xffffffffu, rq, o);
+        }
+        const int row = r0 + 4 * sl + sub, g = row / D, i = row % D;
+        const float a_ = al[t * G + g];
+        const float e = be[t * G + g] * (vs[(t * G + g) * D + i] - a_ * rk);
+#pragma unroll
+        for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) {
+          s[sl][c4].x = fmaf(a_, s[sl][c4].x, e * kr[c4].x);
+          s[sl][c4].y = fmaf(a_, s[sl][c4].y, e * kr[c4].y);
+          s[sl][c4].z = fmaf(a_, s[sl][c4].z, e * kr[c4].z);
+          s[sl][c4].w = fmaf(a_, s[sl][c4].w, e * kr[c4].w);
+        }
+        if ((lane & (DECM_LPR - 1)) == 0) ys[(t * G + g) * D + i] = fmaf(a_, rq, e * kq);
       }
     }
 #pragma unroll
-    for (int u = 0; u < DECM_ROWS; ++u)
-      __stcs(reinterpret_cast<float4*>(state + state0 + (size_t)(r0 + u) * D + lane * 4), s[u]);
+    for (int sl = 0; sl < DECM_SLABS; ++sl) {
+      float4* dst = reinterpret_cast<float4*>(state + state0 + (size_t)(r0 + 4 * sl + sub) * D + cl);
+#pragma unroll
+      for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) __stcs(dst + 8 * c4, s[sl][c4]);
+    }
   }
   __syncthreads();
   for (int i = warp; i < K * G; i += 8) {  // gated RMSNorm of each (token, value head)
     const int t = i / G, g = i % G;
-    const float4 yv = *reinterpret_cast<const float4*>(ys + (t * 8 + g) * D + lane * 4);
+    const float4 yv = *reinterpret_cast<const float4*>(ys + (t * G + g) * D + lane * 4);
     const float ss = warp_sum(yv.x * yv.x + yv.y * yv.y + yv.z * yv.z + yv.w * yv.w);
     const float inv = 1.0f / sqrtf(ss * (1.0f / D) + d.rms_eps);
     const size_t off = (((size_t)n * K + t) * hv + (size_t)j * G + g) * D + lane * 4;
@@ -160,7 +201,5 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
     store4<OUT_BF16>(y, off, o);
   }
 }
-
-constexpr size_t DECM_SMEM = (size_t)(2 * DECM_KMAX * D + 2 * DECM_KMAX * 8 * D + 2 * DECM_KMAX * 8 + DECM_KMAX) * 4;
 
 }  // namespace gdn

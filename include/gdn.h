@@ -176,7 +176,8 @@ int gdn_decode_slots(const gdn_dims_t* d, const void* q, const void* k, const vo
  *   state       [N][h_v][d_v][d_k]         fp32, in/out: the state after the last token
  *   y           [N][n_tokens][h_v][d_v]    out_dtype (written)
  * d->total_tokens must equal d->n_seqs * n_tokens.  Returns GDN_ERR_SHAPE for n_tokens
- * outside 1..8, otherwise what gdn_decode returns.
+ * outside 1..8, otherwise what gdn_decode returns.  n_tokens = 1 is exactly a gdn_decode
+ * call (same kernel, identical results).
  */
 int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const void* k, const void* v,
                      const void* z, const float* a, const float* b, const float* A_log, const float* dt_bias,

@@ -27,7 +27,7 @@ def test_traffic_record_follows_its_kernel_sources(tmp_path, monkeypatch):
     with open(csrc / "k_decode.cuh", "a") as f:
         f.write("\n// edited\n")
     assert bench.ncu_traffic("decode") is None
-    for k in ("prologue_tc", "chunk_prep_tc", "chunk_scan_tc_norm", "chunk_phaseB_simt"):
+    for k in ("chunk_prep_tc", "chunk_scan_tc_norm", "chunk_phaseB_simt", "decode_multi"):
         assert bench.ncu_traffic(k) == rec[k]["dram_bytes_per_launch"]
     # a change to a header every kernel includes stales them all
     with open(csrc / "gdn_common.cuh", "a") as f:

@@ -183,10 +183,11 @@ def bf16_from_f64(x):
     return (np.ascontiguousarray(x, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
 
 
-def _multi_inputs(K, N=3, dtype="bf16", seed=11):
+def _multi_inputs(K, N=3, dtype="bf16", seed=11, h_qk=2, h_v=4):
     """K consecutive decode tokens per sequence: the per-token fields of K seeded one-token
     workloads stacked on axis 1; state, conv history and parameters from the first."""
-    steps = [make_inputs("decode_N256_bf16", seed=seed + i, n_seqs=N, h_qk=2, h_v=4, dtype=dtype) for i in range(K)]
+    steps = [make_inputs("decode_N256_bf16", seed=seed + i, n_seqs=N, h_qk=h_qk, h_v=h_v, dtype=dtype)
+             for i in range(K)]
     out = dict(steps[0])
     for nm in ("q", "k", "v", "z", "a", "b"):
         out[nm] = np.ascontiguousarray(np.stack([s_[nm] for s_ in steps], axis=1))
@@ -221,9 +222,19 @@ def test_decode_multi_one_token_equals_decode():
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("K", [2, 5, 8])
+@pytest.mark.parametrize("K", [2, 3, 4, 5, 8])
 def test_decode_multi_equals_successive_steps(oracle_mod, K, dtype):
-    inp = _multi_inputs(K, dtype=dtype)
+    _check_multi(oracle_mod, _multi_inputs(K, dtype=dtype), K, dtype)
+
+
+@pytest.mark.parametrize("h_qk,h_v", [(2, 2), (2, 8), (1, 8), (16, 32)])
+def test_decode_multi_head_ratios(oracle_mod, h_qk, h_v):
+    """Every value-head ratio the row partition of the multi-token kernel handles (1, 4, 8 and
+    the model's 2), four tokens per sequence."""
+    _check_multi(oracle_mod, _multi_inputs(4, N=2, h_qk=h_qk, h_v=h_v), 4, "bf16")
+
+
+def _check_multi(oracle_mod, inp, K, dtype):
     y, S, cs = _run_multi(inp)
     state = inp["state"].astype(np.float32)
     hist = inp["conv_state"]
