@@ -58,6 +58,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     p.add_argument("--decode-steps", type=int, default=None)
+    p.add_argument("--profile", choices=["prefill", "decode", "decode_multi"], default=None,
+                   help="only run W + K calls of one workload (for ncu captures; prints no bench line)")
     p.add_argument("--configs", action="store_true",
                    help="time every workload (GPU and the oracle on a bounded sample) instead of the bench step")
     return p.parse_args(argv)
@@ -704,8 +706,50 @@ def configs_table(args):
     return 0
 
 
+def profile_case(args):
+    """`--profile`: W + K calls of one workload and nothing else, with a small device footprint
+    (one input set: the prefill holds ~0.5 GB, the decode the 512 MiB of resident state), for
+    ncu captures of a single kernel."""
+    import numpy as np
+    import torch
+
+    from gated_deltanet_token_b200 import gdn
+    from gated_deltanet_token_b200.inputs import make_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n = args.warmup + args.steps
+    if args.profile == "prefill":
+        inp = make_inputs(WORKLOAD)
+        d = {k: to_dev(inp[k], dev) for k in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w", "norm_w")}
+        y = torch.empty((inp["spec"]["T"], 32, 128), dtype=torch.bfloat16, device=dev)
+        for _ in range(n):
+            gdn.gdn_prefill(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["conv_w"],
+                            d["norm_w"], None, None, out_dtype=torch.bfloat16, y=y)
+    else:
+        K = 4 if args.profile == "decode_multi" else 1
+        per_tok = [make_inputs(DECODE_WORKLOAD, seed=100 + i) for i in range(K)]
+        d = {k: to_dev(per_tok[0][k], dev) for k in ("A_log", "dt_bias", "conv_w", "norm_w", "conv_state", "state")}
+        for k in ("q", "k", "v", "z", "a", "b"):
+            d[k] = to_dev(np.ascontiguousarray(np.stack([p_[k] for p_ in per_tok], axis=1)) if K > 1
+                          else per_tok[0][k], dev)
+        del per_tok
+        for _ in range(n):
+            if K > 1:
+                gdn.gdn_decode_multi(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                                     d["conv_w"], d["norm_w"], d["conv_state"], d["state"], out_dtype=torch.bfloat16)
+            else:
+                gdn.gdn_decode(d["q"], d["k"], d["v"], d["z"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["conv_w"],
+                               d["norm_w"], d["conv_state"], d["state"], out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    print(f"profile {args.profile}: {n} calls", flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.profile:
+        return profile_case(args)
     if args.impl == "reference":
         return reference_arm(args)
     if args.configs:

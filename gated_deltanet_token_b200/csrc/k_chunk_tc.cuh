@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(256, 2)
   uint8_t* pb_lo = pb_hi + 16384;
   float* Am = reinterpret_cast<float*>(sm + PA_OFF_A);  // [2][64][PA_P]
   float* Tm = reinterpret_cast<float*>(sm + PA_OFF_T);  // [2][64][PA_P]
-  double* gs = reinterpret_cast<double*>(sm + PA_OFF_G);               // [2][64] gamma (fp64)
+  float2* gs = reinterpret_cast<float2*>(sm + PA_OFF_G);               // [2][64] gamma as hi + lo
   float* bs = reinterpret_cast<float*>(sm + PA_OFF_G + 2 * 64 * 8);   // [2][64] beta
   float4* wsc = reinterpret_cast<float4*>(sm + PA_OFF_W) + (tid >> 4) * 16;  // this half-warp's rows
   const float4* taps = reinterpret_cast<const float4*>(sm + PF_OFF_TAPS);   // [2][128] conv taps
@@ -379,7 +379,12 @@ __global__ void __launch_bounds__(256, 2)
       }
       g1 += __shfl_sync(0xffffffffu, g0, 31);
       const double gL = __shfl_sync(0xffffffffu, g1, 31);  // gamma at the chunk's end (padding adds 0)
-      gs[warp * 64 + lane] = g0; gs[warp * 64 + lane + 32] = g1;
+      // gamma as an unevaluated float pair hi + lo (|lo| <= ulp(hi) / 2): a difference of two
+      // prefixes, (hi_t - hi_s) + (lo_t - lo_s), then has a relative error of a few fp32 ulp of
+      // the difference itself, whatever the size of gamma, and needs no fp64 arithmetic per element
+      const float h0f = (float)g0, h1f = (float)g1;
+      gs[warp * 64 + lane] = make_float2(h0f, (float)(g0 - (double)h0f));
+      gs[warp * 64 + lane + 32] = make_float2(h1f, (float)(g1 - (double)h1f));
       bs[warp * 64 + lane] = b0; bs[warp * 64 + lane + 32] = b1;
       if (warp == 0 || gpair[1] != gpair[0]) {  // phase B's gates: gamma_t and gamma_L - gamma_t
         float* gbw = gb_ws + ((size_t)chunk * hv + h) * GB_FLOATS;
@@ -496,19 +501,25 @@ __global__ void __launch_bounds__(256, 2)
       tc::tmem_wait_ld();
 #pragma unroll 1
       for (int hp = 0; hp < 2; ++hp) {
-        const double* g_ = gs + hp * 64;
-        const double gt = g_[t];
+        const float2* g_ = gs + hp * 64;
+        const float2 gt = g_[t];
+        // the block of columns cbk .. cbk + 31 lies wholly above the diagonal for rows 0..31
+        // (warp-uniform): zeros, with no exponentials
+        const bool upper = cbk > (q4 & 1) * 32;
         if (q4 < 2) {  // A[t][s] = beta_t e^{gamma_t - gamma_s} (k_t . k_s), s < t
           const float bt = bs[hp * 64 + t];
           float* Ah = Am + hp * (64 * PA_P);
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
-            float4 o;
+            float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             float* op = &o.x;
+            if (!upper) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int s_ = cbk + c4 * 4 + u;
-              op[u] = s_ < t ? bt * __expf((float)(gt - g_[s_])) * __uint_as_float(r[c4 * 4 + u]) : 0.0f;
+              for (int u = 0; u < 4; ++u) {
+                const int s_ = cbk + c4 * 4 + u;
+                op[u] = s_ < t ? bt * __expf((gt.x - g_[s_].x) + (gt.y - g_[s_].y)) * __uint_as_float(r[c4 * 4 + u])
+                               : 0.0f;
+              }
             }
             *reinterpret_cast<float4*>(Ah + t * PA_P + cbk + c4 * 4) = o;
           }
@@ -519,7 +530,9 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               const int s_ = cbk + c8 * 8 + u;
-              mv[u] = s_ <= t ? __expf((float)(gt - g_[s_])) * __uint_as_float(r[c8 * 8 + u]) : 0.0f;
+              mv[u] = (!upper && s_ <= t)
+                          ? __expf((gt.x - g_[s_].x) + (gt.y - g_[s_].y)) * __uint_as_float(r[c8 * 8 + u])
+                          : 0.0f;
             }
             uint4 hi, lo;
             tc::split8(mv, hi, lo);
@@ -768,9 +781,10 @@ enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 // token's sum into the three other CTAs of the cluster as one 32-bit word whose two low bits
 // carry a chunk tag (the value is the flag: no fence or barrier between CTAs), then waits for
 // the peers' words and normalises its y row.  The norm warps stay out of the workers' chunk
-// barriers: they arrive on an mbarrier once they are done with a chunk's TMEM rows and stage,
-// and thread 0 waits for that before the next chunk's first MMA round, so the exchange never
-// holds up the state chain.  Every slice sums the same four tag-stripped words in rank order,
+// barriers: they arrive on per-parity mbarriers once they have read a chunk's gates and once
+// they are done with its TMEM rows; the accumulators of rounds 1 and 2 are double-buffered by
+// chunk parity, so thread 0 waits for the rows of chunk c - 2 only, and the producer reloads a
+// stage only after the norm warps read its gates.  The exchange never holds up the state chain.  Every slice sums the same four tag-stripped words in rank order,
 // so all four use the same norm.  Warp 9 idles.
 template <int YM>
 __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
@@ -800,12 +814,17 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   uint8_t* s_lo = sm + PB_S_TILE;
   uint8_t* stage[2] = {sm + 2 * PB_S_TILE, sm + 2 * PB_S_TILE + PBStage::BYTES};
   __shared__ uint64_t mbar_ld[2];
-  __shared__ uint64_t mbar_mma[3];  // one per MMA round: each completes once per chunk
+  // MMA completions: rounds 1 and 2 by chunk parity (their accumulators are double-buffered,
+  // so the norm warps may read chunk c's rows while chunk c + 1 runs), round 3 once per chunk
+  __shared__ uint64_t mbar_r1[2], mbar_r2[2], mbar_r3;
   __shared__ uint32_t tslot;
   __shared__ int s_abort;
-  __shared__ uint64_t norm_done;  // fused norm: the norm warps are done with a chunk (64 arrivals)
+  // fused norm, by chunk parity (64 arrivals each): the norm warps have read a chunk's gates
+  // (the stage may be reloaded) and its TMEM rows (the accumulators may be reused)
+  __shared__ uint64_t gates_read[2], norm_done[2];
   // fused norm: tagged sums of squares from the three other slices, [chunk parity][peer][token]
   __shared__ uint32_t red[FUSED ? 2 * 3 * 64 : 1];
+  __shared__ __align__(16) float nw_s[FUSED ? NV : 4];  // fused norm: this slice's norm_w
   const int rank = FUSED ? (int)tc::cluster_ctarank() : 0;
 
   if (FUSED && tc::cluster_nctarank() != D / NV) {  // launched without its clusters: no exchange
@@ -824,12 +843,17 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     s_abort = 0;
     tc::mbar_init(tc::smem_u32(&mbar_ld[0]), 1);
     tc::mbar_init(tc::smem_u32(&mbar_ld[1]), 1);
-    for (int q3 = 0; q3 < 3; ++q3) tc::mbar_init(tc::smem_u32(&mbar_mma[q3]), 1);
-    if (FUSED) tc::mbar_init(tc::smem_u32(&norm_done), 64);
+    for (int p2 = 0; p2 < 2; ++p2) {
+      tc::mbar_init(tc::smem_u32(&mbar_r1[p2]), 1);
+      tc::mbar_init(tc::smem_u32(&mbar_r2[p2]), 1);
+      tc::mbar_init(tc::smem_u32(&gates_read[p2]), 64);
+      tc::mbar_init(tc::smem_u32(&norm_done[p2]), 64);
+    }
+    tc::mbar_init(tc::smem_u32(&mbar_r3), 1);
     tc::fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(&tslot), 256);  // D_a 0..63, D_cd 64..127, D_e 128..191
+    tc::tmem_alloc(tc::smem_u32(&tslot), 512);  // by chunk parity p: D_a 256 p + 0..63, D_cd 256 p + 64..127; D_e 128..191
     tc::tmem_relinquish();
   }
   // named barrier over a subset of the warps (id 1: the R / U-tilde writers, id 2: all but
@@ -886,8 +910,10 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     }
   };
   if (worker) write_s_tile();
-  if (FUSED)
+  if (FUSED) {
     for (int i = tid; i < 2 * 3 * 64; i += blockDim.x) red[i] = 3u;  // tag 3: no chunk yet
+    if (tid < NV / 4) reinterpret_cast<float4*>(nw_s)[tid] = __ldg(reinterpret_cast<const float4*>(norm_w + i0) + tid);
+  }
   tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
@@ -896,8 +922,10 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   const uint32_t tbase = tslot;
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
   // accumulators (2 nv columns each: [a_hi b_hi + a_lo b_hi | a_hi b_lo])
+  // accumulators; rounds 1 and 2 add 256 columns for odd chunks
   const uint32_t T_A = tbase, T_CD = tbase + 2 * NV, T_E = tbase + 4 * NV;
   const uint32_t t_a = T_A + lane_off + cb, t_cd = T_CD + lane_off + cb, t_e = T_E + lane_off + cb;
+  auto par_cols = [](int c) { return (uint32_t)(c & 1) * 256u; };
   int last_load = -1;  // (producer lane) the last chunk whose stage copies were issued
   if (producer && lane == 0 && nchunks > 0) {
     issue_load(0, 0);
@@ -909,12 +937,17 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   constexpr uint32_t idesc_mn = tc::idesc_bf16(128, NV, 1, 1);
   const uint64_t d_s[2] = {tc::sdesc(tc::smem_u32(s_hi), 128, 16 * 128), tc::sdesc(tc::smem_u32(s_lo), 128, 16 * 128)};
 
-  uint32_t ph_ld[2] = {0, 0}, ph_mma = 0;  // ph_mma: parity of this chunk's phase of each round barrier
+  uint32_t ph_ld[2] = {0, 0};
+  // phase parity of chunk c's completion on a barrier that completes once per chunk (round 3) or
+  // once every two chunks (the per-parity barriers)
+  auto ph1 = [](int c) { return (uint32_t)c & 1u; };
+  auto ph2 = [](int c) { return (uint32_t)(c >> 1) & 1u; };
   bool aborted = false;
   // fused norm, norm threads: the previous chunk's y row (in keep, token y_tok, or -1)
   float* yv = keep;
   float own = 0.0f;
   int y_tok = -1;
+  uint4 zcur[NV / 8];  // fused norm: the z row of this thread's token in the current chunk
   auto untag = [](uint32_t w) { return __uint_as_float(w & ~3u); };
   const uint32_t t_norm = tbase + ((uint32_t)(64 + 32 * (warp & 1)) << 16);  // norm warps: lanes 64.. / 96..
   // normalise and store the y row held from chunk cy (bounded wait for the peers' words)
@@ -940,14 +973,13 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
       tot += rr == rank ? own : untag(rr < rank ? w[rr < 3 ? rr : 2] : w[rr > 0 ? rr - 1 : 0]);
     if (y_tok >= 0) {
       const float inv = rsqrtf(tot * (1.0f / D) + d.rms_eps);
-      const float4* nw4 = reinterpret_cast<const float4*>(norm_w + i0);
+      const float4* nw4 = reinterpret_cast<const float4*>(nw_s);
       const size_t base = ((size_t)y_tok * hv + h) * D + i0;
-      const uint4* zp = reinterpret_cast<const uint4*>(z + base);
 #pragma unroll
       for (int g8 = 0; g8 < NV / 8; ++g8) {  // 8 columns at a time
-        const uint4 zq = __ldg(zp + g8);
+        const uint4 zq = zcur[g8];
         const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
-        const float4 wa = __ldg(nw4 + 2 * g8), wb = __ldg(nw4 + 2 * g8 + 1);
+        const float4 wa = nw4[2 * g8], wb = nw4[2 * g8 + 1];
         float o[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -977,35 +1009,41 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int st = c & 1;
       const int t0 = ts + c * CH, L = min(CH, te - t0);
+      if (t < L) {  // this token's z row, read now so that it has landed when the row is finished
+        const uint4* zp = reinterpret_cast<const uint4*>(z + ((size_t)(t0 + t) * hv + h) * D + i0);
+#pragma unroll
+        for (int g8 = 0; g8 < NV / 8; ++g8) zcur[g8] = __ldg(zp + g8);
+      }
       const float* gsm = reinterpret_cast<const float*>(stage[st] + PBStage::GB);
       // warp-uniform, so that the warp-collective TMEM loads run on every lane or none
       bool ok = __all_sync(0xffffffffu, wait_ok(mbar_ld[st], ph_ld[st]));
       ph_ld[st] ^= 1;
       const float eg = (ok && t < L) ? __expf(gsm[t]) : 0.0f;
+      tc::mbar_arrive(tc::smem_u32(&gates_read[st]));  // the stage may be reloaded for chunk c + 2
+      const uint32_t tn_c = t_norm + par_cols(c);
       float qs[NV];  // e^{gamma_t} (Q S^T)[t][:], all 32 columns of the slice, 16 at a time
-      ok = __all_sync(0xffffffffu, ok && wait_ok(mbar_mma[0], ph_mma));
+      ok = __all_sync(0xffffffffu, ok && wait_ok(mbar_r1[st], ph2(c)));
       tc::tc_fence_after();
       if (ok) {
 #pragma unroll
         for (int h16 = 0; h16 < 2; ++h16) {
           uint32_t r[16], r2[16];
-          tc::tmem_ld16(t_norm + 16 * h16, r);
-          tc::tmem_ld16(t_norm + NV + 16 * h16, r2);
+          tc::tmem_ld16(tn_c + 16 * h16, r);
+          tc::tmem_ld16(tn_c + NV + 16 * h16, r2);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) qs[16 * h16 + i] = eg * (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
         }
       }
-      ok = __all_sync(0xffffffffu, ok && wait_ok(mbar_mma[1], ph_mma));
-      ph_mma ^= 1;
+      ok = __all_sync(0xffffffffu, ok && wait_ok(mbar_r2[st], ph2(c)));
       tc::tc_fence_after();
       if (ok) {  // Y = e^gamma Q S^T + (M o QK^T) U, and this slice's sum of squares to the peers
         float p = 0.0f;
 #pragma unroll
         for (int h16 = 0; h16 < 2; ++h16) {
           uint32_t r[16], r2[16];
-          tc::tmem_ld16(t_norm + 2 * NV + 16 * h16, r);
-          tc::tmem_ld16(t_norm + 3 * NV + 16 * h16, r2);
+          tc::tmem_ld16(tn_c + 2 * NV + 16 * h16, r);
+          tc::tmem_ld16(tn_c + 3 * NV + 16 * h16, r2);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -1026,7 +1064,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
         }
       }
       tc::tc_fence_before();
-      tc::mbar_arrive(tc::smem_u32(&norm_done));  // this chunk's TMEM rows and stage are read
+      tc::mbar_arrive(tc::smem_u32(&norm_done[st]));  // this chunk's TMEM rows are read
       // warp-uniform decisions: every lane of a norm warp leaves at the same chunk
       if (!__all_sync(0xffffffffu, ok && finish(c))) { s_abort = 1; atomicExch(&g_gdn_status, -7); break; }
       if (__any_sync(0xffffffffu, aborted_now())) break;
@@ -1056,7 +1094,9 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     const float eg = t < L ? __expf(gsm[t]) : 0.0f;
     // the norm warps are done with the previous chunk's TMEM rows and stage before this
     // chunk's first round overwrites the one and the producer reloads the other
-    if (FUSED && tid == 0 && c > 0) (void)wait_ok(norm_done, (uint32_t)(c - 1) & 1u);
+    // the norm warps are done with chunk c - 2's accumulator rows, which this chunk's rounds 1
+    // and 2 overwrite
+    if (FUSED && tid == 0 && c > 1) (void)wait_ok(norm_done[st], ph2(c - 2));
     // the chunk barrier, reducing the abort flag: a timeout recorded by any thread before it
     // arrived ends the loop for every thread at the same chunk
     if (loop_sync_or(aborted_now())) { aborted = true; break; }
@@ -1067,22 +1107,24 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t ao = (uint64_t)((ks * 2 * LBO128) >> 4), bo = (uint64_t)((ks * 256) >> 4);
-        tc::umma_bf16(T_A, da[0] + ao, d_s[0] + bo, idesc_kn2, ks != 0);  // a_hi [s_hi | s_lo]
-        tc::umma_bf16(T_A, da[1] + ao, d_s[0] + bo, idesc_kn, 1);         // a_lo s_hi
+        tc::umma_bf16(T_A + par_cols(c), da[0] + ao, d_s[0] + bo, idesc_kn2, ks != 0);  // a_hi [s_hi | s_lo]
+        tc::umma_bf16(T_A + par_cols(c), da[1] + ao, d_s[0] + bo, idesc_kn, 1);         // a_lo s_hi
       }
-      tc::umma_commit(tc::smem_u32(&mbar_mma[0]));
+      tc::umma_commit(tc::smem_u32(&mbar_r1[st]));
     }
-    if (producer && lane == 0 && c + 1 < nchunks && !aborted_now()) {  // stage last read by chunk c-1
+    // the stage last read by chunk c - 1 (and, fused, its gates by the norm warps)
+    if (producer && lane == 0 && c + 1 < nchunks && !aborted_now() &&
+        (!FUSED || c == 0 || wait_ok(gates_read[st ^ 1], ph2(c - 1)))) {
       issue_load(c + 1, st ^ 1);
       last_load = c + 1;
     }
-    const bool ok1 = wait_ok(mbar_mma[0], ph_mma);
+    const bool ok1 = wait_ok(mbar_r1[st], ph2(c));
     tc::tc_fence_after();
     float qs[NH];  // y rows (separate-epilogue mode): e^{gamma_t} (Q S^T)[t][:]
     if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
-      tc::tmem_ld16(t_a, r);
-      tc::tmem_ld16(t_a + NV, r2);
+      tc::tmem_ld16(t_a + par_cols(c), r);
+      tc::tmem_ld16(t_a + par_cols(c) + NV, r2);
       tc::tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
@@ -1114,17 +1156,17 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         const uint64_t ao = (uint64_t)((ks * 2 * LBO128) >> 4), bo = (uint64_t)((ks * 256) >> 4);
-        tc::umma_bf16(T_CD, da[0] + ao, db + bo, idesc_kn2, ks != 0);
-        tc::umma_bf16(T_CD, da[1] + ao, db + bo, idesc_kn, 1);
+        tc::umma_bf16(T_CD + par_cols(c), da[0] + ao, db + bo, idesc_kn2, ks != 0);
+        tc::umma_bf16(T_CD + par_cols(c), da[1] + ao, db + bo, idesc_kn, 1);
       }
-      tc::umma_commit(tc::smem_u32(&mbar_mma[1]));
+      tc::umma_commit(tc::smem_u32(&mbar_r2[st]));
     }
-    const bool ok2 = wait_ok(mbar_mma[1], ph_mma);
+    const bool ok2 = wait_ok(mbar_r2[st], ph2(c));
     tc::tc_fence_after();
     if (rwarp || (!FUSED && worker)) {
       uint32_t r[16], r2[16];
-      tc::tmem_ld16(t_cd, r);
-      tc::tmem_ld16(t_cd + NV, r2);
+      tc::tmem_ld16(t_cd + par_cols(c), r);
+      tc::tmem_ld16(t_cd + par_cols(c) + NV, r2);
       tc::tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
@@ -1165,10 +1207,9 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
         tc::umma_bf16(T_E, da[0] + o, db + o, idesc_mn2, ks != 0);
         tc::umma_bf16(T_E, da[1] + o, db + o, idesc_mn, 1);
       }
-      tc::umma_commit(tc::smem_u32(&mbar_mma[2]));
+      tc::umma_commit(tc::smem_u32(&mbar_r3));
     }
-    (void)wait_ok(mbar_mma[2], ph_mma);
-    ph_mma ^= 1;
+    (void)wait_ok(mbar_r3, ph1(c));
     tc::tc_fence_after();
     if (worker) {
       uint32_t r[16], r2[16];
@@ -1195,7 +1236,7 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     (void)tc::mbar_wait(tc::smem_u32(&mbar_ld[last_load & 1]), (uint32_t)(last_load >> 1) & 1u);
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tbase, 256);
+  if (warp == 0) tc::tmem_dealloc(tbase, 512);
   if (FUSED) tc::cluster_sync();  // no CTA leaves while a peer may still write to it
 }
 

@@ -7,10 +7,14 @@
 // three raw rows.  One CTA per (sequence n, QK head j) as in k_decode.
 //
 // Row layout: eight lanes share a state row, each holding four groups of four columns
-// (columns 32 c + 4 (lane % 8) .. + 3, c = 0..3, so that every 16-byte load of the eight lanes
-// covers 128 contiguous bytes of the row).  A warp works on four rows at once, and the two dot
-// products of a token (S'k and S'q) reduce over eight lanes in three shuffle levels -- for four
-// rows together.  Two such four-row slabs are in flight per warp (8 rows, 4 KB of state).
+// (columns 32 c + 4 (lane % 8) .. + 3, c = 0..3).  A warp works on four rows at once, and the
+// two dot products of a token (S'k and S'q) reduce over eight lanes in three shuffle levels --
+// for four rows together.  A warp takes its rows in groups of eight (two four-row slabs):
+// each group is copied into shared memory by asynchronous 16-byte copies two groups ahead
+// (double-buffered; the first two start before the conv prologue), so the next 4 KB of state
+// is always in flight while the current group is updated in registers; the updated rows go
+// straight back to global memory.  The dot products
+// and the row update use paired fp32 FMAs.
 #pragma once
 #include "gdn_common.cuh"
 
@@ -19,12 +23,16 @@ namespace gdn {
 constexpr int DECM_KMAX = 8;
 constexpr int DECM_LPR = 8;             // lanes per state row
 constexpr int DECM_CPL = D / DECM_LPR;  // columns per lane: 16
-constexpr int DECM_SLABS = 2;           // four-row slabs in flight per warp
+constexpr int DECM_SLABS = 1;           // four-row slabs per group
 
-// Dynamic shared memory of one CTA (floats): q, k [K][D]; v, y [K][G][D]; alpha, beta [K][G];
-// k . q [K].
+constexpr int DECM_WARPS = 8;
+constexpr int DECM_GROUP = 4 * DECM_SLABS;                      // state rows per group
+constexpr int DECM_BUF_FLOATS = 2 * DECM_WARPS * DECM_GROUP * D;  // two group buffers per warp
+
+// Dynamic shared memory of one CTA (floats): the state-row buffers; q, k [K][D]; v, y [K][G][D];
+// alpha, beta [K][G]; k . q [K].
 __host__ __device__ constexpr size_t decm_smem_bytes(int K, int G) {
-  return (size_t)(2 * K * D + 2 * K * G * D + 2 * K * G + K) * sizeof(float);
+  return (size_t)(DECM_BUF_FLOATS + 2 * K * D + 2 * K * G * D + 2 * K * G + K) * sizeof(float);
 }
 constexpr size_t DECM_SMEM = decm_smem_bytes(DECM_KMAX, 8);
 
@@ -47,7 +55,8 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
     return;
   }
   extern __shared__ __align__(16) float dm[];
-  float* qs = dm;                 // [K][D]
+  float* sbuf = dm;               // [warps][2][8 rows][D] state-row buffers
+  float* qs = sbuf + DECM_BUF_FLOATS;  // [K][D]
   float* ks = qs + K * D;         // [K][D]
   float* vs = ks + K * D;         // [K][G][D]
   float* ys = vs + K * G * D;     // [K][G][D]
@@ -55,6 +64,26 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
   float* be = al + K * G;         // [K][G]  beta
   float* kqv = be + K * G;        // [K]     k_t . q_t
 
+  const int sub = lane >> 3, cl = (lane & 7) * 4;
+  const int rows_per_warp = G * D / DECM_WARPS;  // a multiple of DECM_GROUP
+  const int ngroups = rows_per_warp / DECM_GROUP;
+  const size_t wrow0 = ((size_t)n * hv + (size_t)j * G) * D + (size_t)warp * rows_per_warp;  // first row
+  float* wbuf = sbuf + warp * 2 * DECM_GROUP * D;
+  // group gi of this warp's rows into buffer gi & 1: 256 chunks of 16 bytes, 8 per lane
+  auto load_group = [&](int gi) {
+    const float* src = state + (wrow0 + (size_t)gi * DECM_GROUP) * D;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf + (gi & 1) * DECM_GROUP * D));
+#pragma unroll
+    for (int m = 0; m < DECM_GROUP * D / 4 / 32; ++m) {
+      const int idx = lane + 32 * m;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + idx * 16), "l"(src + idx * 4) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // the first two groups start streaming now, under the conv, gates and norms below
+  load_group(0);
+  if (ngroups > 1) load_group(1);
+  else asm volatile("cp.async.commit_group;" ::: "memory");
   // conv + SiLU for the K tokens over this CTA's channels; the history becomes the last
   // three raw rows of (history, new rows), copied exactly
   E* cs = static_cast<E*>(conv_state) + (size_t)n * 3 * cconv;
@@ -132,17 +161,20 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
   // 32 c4 + cl .. + 3 for c4 = 0..3.  Per token, for each row i of value head g:
   //   S' = alpha S;  r_k = S' k;  e = beta (v_i - r_k);  S'' = S' + e k^T;  y_i = S'' q
   // with y_i = alpha (S q) + e (k . q).
-  const int sub = lane >> 3, cl = (lane & 7) * 4;
-  const int rows_per_warp = G * D / 8;
-  const size_t state0 = ((size_t)n * hv + (size_t)j * G) * D * D;
-  for (int r0 = warp * rows_per_warp; r0 < (warp + 1) * rows_per_warp; r0 += 4 * DECM_SLABS) {
+  for (int gi = 0; gi < ngroups; ++gi) {
+    // committed so far: groups 0 .. gi + 1 (an empty group stands in past the last one)
+    asm volatile("cp.async.wait_group 1;" ::: "memory");  // this lane's copies of group gi landed
+    __syncwarp();                                           // ... and every lane's
+    const float* gb = wbuf + (gi & 1) * DECM_GROUP * D;
     float4 s[DECM_SLABS][DECM_CPL / 4];
 #pragma unroll
-    for (int sl = 0; sl < DECM_SLABS; ++sl) {
-      const float4* src = reinterpret_cast<const float4*>(state + state0 + (size_t)(r0 + 4 * sl + sub) * D + cl);
+    for (int sl = 0; sl < DECM_SLABS; ++sl)
 #pragma unroll
-      for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) s[sl][c4] = __ldcs(src + 8 * c4);
-    }
+      for (int c4 = 0; c4 < DECM_CPL / 4; ++c4)
+        s[sl][c4] = *reinterpret_cast<const float4*>(gb + (4 * sl + sub) * D + 32 * c4 + cl);
+    __syncwarp();  // every lane has read the buffer before group gi + 2 refills it
+    if (gi + 2 < ngroups) load_group(gi + 2);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
     for (int t = 0; t < K; ++t) {
       float4 kr[DECM_CPL / 4], qr[DECM_CPL / 4];
 #pragma unroll
@@ -153,37 +185,44 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
       const float kq = kqv[t];
 #pragma unroll
       for (int sl = 0; sl < DECM_SLABS; ++sl) {
-        float rk = 0.0f, rq = 0.0f;
+        float2 rk2 = make_float2(0.0f, 0.0f), rq2 = rk2;
 #pragma unroll
         for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) {
-          rk += dot4(s[sl][c4], kr[c4]);
-          rq += dot4(s[sl][c4], qr[c4]);
+          const float2 s0 = make_float2(s[sl][c4].x, s[sl][c4].y), s1 = make_float2(s[sl][c4].z, s[sl][c4].w);
+          rk2 = __ffma2_rn(s0, make_float2(kr[c4].x, kr[c4].y), rk2);
+          rk2 = __ffma2_rn(s1, make_float2(kr[c4].z, kr[c4].w), rk2);
+          rq2 = __ffma2_rn(s0, make_float2(qr[c4].x, qr[c4].y), rq2);
+          rq2 = __ffma2_rn(s1, make_float2(qr[c4].z, qr[c4].w), rq2);
         }
+        float rk = rk2.x + rk2.y, rq = rq2.x + rq2.y;
 #pragma unroll
         for (int o = 1; o < DECM_LPR; o <<= 1) {  // the eight lanes of the row
           rk += __shfl_xor_sync(0xffffffffu, rk, o);
           rq += __shfl_xor_sync(0xffffffffu, rq, o);
         }
-        const int row = r0 + 4 * sl + sub, g = row / D, i = row % D;
+        const int row = warp * rows_per_warp + gi * DECM_GROUP + 4 * sl + sub, g = row / D, i = row % D;
         const float a_ = al[t * G + g];
         const float e = be[t * G + g] * (vs[(t * G + g) * D + i] - a_ * rk);
+        const float2 a2 = make_float2(a_, a_), e2 = make_float2(e, e);
 #pragma unroll
         for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) {
-          s[sl][c4].x = fmaf(a_, s[sl][c4].x, e * kr[c4].x);
-          s[sl][c4].y = fmaf(a_, s[sl][c4].y, e * kr[c4].y);
-          s[sl][c4].z = fmaf(a_, s[sl][c4].z, e * kr[c4].z);
-          s[sl][c4].w = fmaf(a_, s[sl][c4].w, e * kr[c4].w);
+          const float2 lo = __ffma2_rn(a2, make_float2(s[sl][c4].x, s[sl][c4].y),
+                                       __fmul2_rn(e2, make_float2(kr[c4].x, kr[c4].y)));
+          const float2 hi = __ffma2_rn(a2, make_float2(s[sl][c4].z, s[sl][c4].w),
+                                       __fmul2_rn(e2, make_float2(kr[c4].z, kr[c4].w)));
+          s[sl][c4] = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
         if ((lane & (DECM_LPR - 1)) == 0) ys[(t * G + g) * D + i] = fmaf(a_, rq, e * kq);
       }
     }
 #pragma unroll
     for (int sl = 0; sl < DECM_SLABS; ++sl) {
-      float4* dst = reinterpret_cast<float4*>(state + state0 + (size_t)(r0 + 4 * sl + sub) * D + cl);
+      float4* dst = reinterpret_cast<float4*>(state + (wrow0 + (size_t)gi * DECM_GROUP + 4 * sl + sub) * D + cl);
 #pragma unroll
       for (int c4 = 0; c4 < DECM_CPL / 4; ++c4) __stcs(dst + 8 * c4, s[sl][c4]);
     }
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   for (int i = warp; i < K * G; i += 8) {  // gated RMSNorm of each (token, value head)
     const int t = i / G, g = i % G;

@@ -124,10 +124,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // `bar`.  `tmap` is the address of a __grid_constant__ CUtensorMap kernel parameter; (x, y, z)
 // is the box origin in elements (x * element size must be a multiple of 16 bytes; the other
 // coordinates may be negative or past the end: those elements read as zeros).
-// L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned global address
-__device__ __forceinline__ void prefetch_l2(const void* gptr, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");
-}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
