@@ -18,6 +18,7 @@
 #include "k_chunk_tc.cuh"
 #include "k_decode.cuh"
 #include "k_decode_multi.cuh"
+#include "k_proj.cuh"
 #include "k_stream.cuh"
 
 using namespace gdn;
@@ -243,6 +244,22 @@ int make_stream_map(CUtensorMap* m, const void* x, int T, int nheads, int box_he
   return r == CUDA_SUCCESS ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// Tensor map of a K-major bf16 matrix [rows][K] for the projection GEMM: boxes of 64 K x box_rows
+// rows in the 128-byte swizzled layout (rows past the matrix read as zeros).
+int make_kmajor_map(CUtensorMap* m, const void* x, long long rows, int K, int box_rows) {
+  memset(m, 0, sizeof(*m));
+  PFN_cuTensorMapEncodeTiled_v12000 f = encode_tiled();
+  if (!f) return GDN_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)PJ_BK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GDN_OK : GDN_ERR_CUDA;
+}
+
 // Opt the large-shared-memory kernels in once per device.
 int configure_device() {
   static std::atomic<uint64_t> done_mask{0};
@@ -267,6 +284,7 @@ int configure_device() {
                            (int)PB_TC_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)PB_TC_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_proj_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PJ_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_decode_multi<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)DECM_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_decode_multi<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -563,6 +581,78 @@ int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const
     k_decode_multi<false, false><<<grid, 256, smem, s>>>(kd, n_tokens, q, k, v, z, a, b, A_log, dt_bias, conv_w,
                                                         norm_w, conv_state, state, y);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// C = A B^T on tcgen05 into the output segments of `po` (M rows of A, N rows of B, K columns).
+static int proj_launch(const void* A, long long M, const void* B, int N, int K, const ProjOut& po,
+                       gdn_stream_t stream) {
+  int rc = configure_device();
+  if (rc != GDN_OK) return rc;
+  if (M == 0) return GDN_OK;
+  CUtensorMap ta, tb;
+  if (make_kmajor_map(&ta, A, M, K, PJ_BM) != GDN_OK || make_kmajor_map(&tb, B, N, K, PJ_BN) != GDN_OK)
+    return GDN_ERR_CUDA;
+  const dim3 grid((unsigned)((N + PJ_BN - 1) / PJ_BN), (unsigned)((M + PJ_BM - 1) / PJ_BM));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope p("proj_gemm", s);
+  k_proj_gemm<<<grid, 192, PJ_SMEM, s>>>((int)M, N, K, ta, tb, po);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_in_proj(const gdn_dims_t* d, int32_t hidden, const void* x, const void* w_in, void* q, void* k, void* v,
+                void* z, float* a, float* b, gdn_stream_t stream) {
+  int rc = check_dims(d, false);
+  if (rc != GDN_OK) return rc;
+  if (d->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_DTYPE;
+  if (hidden <= 0 || hidden % PJ_BK != 0 || hidden > (1 << 20)) return GDN_ERR_SHAPE;
+  const void* ptrs[] = {x, w_in, q, k, v, z, a, b};
+  for (const void* p : ptrs)
+    if (!p) return GDN_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const int nq = d->h_qk * D, nv = d->h_v * D;
+  const long long N = 2LL * nq + 2LL * nv + 2LL * d->h_v;
+  if (N > (1 << 24)) return GDN_ERR_SHAPE;
+  ProjOut po{};
+  po.nseg = 6;
+  int n = 0;
+  auto seg = [&](int i, int width, long long ld, int f32, void* out) {
+    po.seg[i].n0 = n;
+    po.seg[i].n1 = n + width;
+    po.seg[i].ld = ld;
+    po.seg[i].f32 = f32;
+    po.seg[i].out = out;
+    n += width;
+  };
+  seg(0, nq, nq, 0, q);
+  seg(1, nq, nq, 0, k);
+  seg(2, nv, nv, 0, v);
+  seg(3, nv, nv, 0, z);
+  seg(4, d->h_v, d->h_v, 1, a);
+  seg(5, d->h_v, d->h_v, 1, b);
+  return proj_launch(x, d->total_tokens, w_in, (int)N, hidden, po, stream);
+}
+
+int gdn_out_proj(const gdn_dims_t* d, int32_t hidden, const void* y, const void* w_out, void* out,
+                 gdn_stream_t stream) {
+  int rc = check_dims(d, false);
+  if (rc != GDN_OK) return rc;
+  if (d->out_dtype != GDN_DTYPE_BF16) return GDN_ERR_DTYPE;
+  if (hidden <= 0 || hidden % 32 != 0 || hidden > (1 << 20)) return GDN_ERR_SHAPE;
+  const void* ptrs[] = {y, w_out, out};
+  for (const void* p : ptrs)
+    if (!p) return GDN_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const int K = d->h_v * D;
+  ProjOut po{};
+  po.nseg = 1;
+  po.seg[0].n0 = 0;
+  po.seg[0].n1 = hidden;
+  po.seg[0].ld = hidden;
+  po.seg[0].f32 = 0;
+  po.seg[0].out = out;
+  return proj_launch(y, d->total_tokens, w_out, hidden, K, po, stream);
 }
 
 int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, const void* v,

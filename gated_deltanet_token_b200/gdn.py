@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_slots.argtypes = [dp] + [vp] * 12 + [ctypes.c_int32, vp, vp, vp]
         L.gdn_decode_multi.restype = ctypes.c_int
         L.gdn_decode_multi.argtypes = [dp, ctypes.c_int32] + [vp] * 13 + [vp]
+        L.gdn_in_proj.restype = ctypes.c_int
+        L.gdn_in_proj.argtypes = [dp, ctypes.c_int32] + [vp] * 8 + [vp]
+        L.gdn_out_proj.restype = ctypes.c_int
+        L.gdn_out_proj.argtypes = [dp, ctypes.c_int32] + [vp] * 3 + [vp]
         L.gdn_prefill_conv_state.restype = ctypes.c_int
         L.gdn_prefill_conv_state.argtypes = [dp] + [vp] * 5 + [vp]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -332,3 +336,47 @@ def gdn_decode_multi(q, k, v, z, a, b, A_log, dt_bias, conv_w, norm_w, conv_stat
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_multi")
     return y
+
+
+def gdn_in_proj(x, w_in, h_qk, h_v, *, d_k=128, d_v=128, out=None, stream=None):
+    """[q | k | v | z | a | b] = x w_in^T for x [T, hidden] bf16 and w_in [N_in, hidden] bf16.
+    Returns (q [T, h_qk, d_k], k, v [T, h_v, d_v], z, a [T, h_v] fp32, b); `out` may hold
+    preallocated tensors in that order."""
+    T, hidden = x.shape
+    if w_in.dtype != torch.bfloat16 or x.dtype != torch.bfloat16:
+        raise TypeError("x and w_in must be bf16")
+    if w_in.shape != (2 * h_qk * d_k + 2 * h_v * d_v + 2 * h_v, hidden):
+        raise ValueError("w_in must be [2 h_qk d_k + 2 h_v d_v + 2 h_v, hidden]")
+    if out is None:
+        dev = x.device
+        out = (torch.empty((T, h_qk, d_k), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, h_qk, d_k), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, h_v, d_v), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, h_v, d_v), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, h_v), dtype=torch.float32, device=dev),
+               torch.empty((T, h_v), dtype=torch.float32, device=dev))
+    dims = make_dims(1, T, h_qk, h_v, GDN_DTYPE_BF16, GDN_DTYPE_BF16, d_k, d_v)
+    rc = lib().gdn_in_proj(ctypes.byref(dims), ctypes.c_int32(hidden), _ptr(x), _ptr(w_in),
+                           *[_ptr(t) for t in out], _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_in_proj")
+    return out
+
+
+def gdn_out_proj(y, w_out, h_qk, h_v, *, d_v=128, out=None, stream=None):
+    """out = y w_out^T for y [T, h_v, d_v] (or [T, h_v d_v]) bf16 and w_out [hidden, h_v d_v] bf16;
+    returns out [T, hidden] bf16."""
+    T = y.shape[0]
+    hidden = w_out.shape[0]
+    if y.dtype != torch.bfloat16 or w_out.dtype != torch.bfloat16:
+        raise TypeError("y and w_out must be bf16")
+    if w_out.shape[1] != h_v * d_v or y.numel() != T * h_v * d_v:
+        raise ValueError("w_out must be [hidden, h_v d_v] and y [T, h_v, d_v]")
+    if out is None:
+        out = torch.empty((T, hidden), dtype=torch.bfloat16, device=y.device)
+    dims = make_dims(1, T, h_qk, h_v, GDN_DTYPE_BF16, GDN_DTYPE_BF16, 128, d_v)
+    rc = lib().gdn_out_proj(ctypes.byref(dims), ctypes.c_int32(hidden), _ptr(y), _ptr(w_out), _ptr(out),
+                            _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_out_proj")
+    return out

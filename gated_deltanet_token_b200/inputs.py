@@ -117,3 +117,17 @@ def make_inputs(name: str, seed: int = 0, **over) -> dict:
         out["state"] = _normal(rng, (n_seqs, hv, d, d), "f32", 0.02)
         out["conv_state"] = _normal(rng, (n_seqs, 3, cconv), dt)
     return out
+
+
+def make_proj_inputs(T: int, hidden: int = 2048, h_qk: int = 16, h_v: int = 32, d: int = 128,
+                     seed: int = 0) -> dict:
+    """Synthetic inputs of the projections around the mixer (the pages print no weights):
+    x ~ N(0, 1) [T, hidden], W_in ~ N(0, 1/hidden) [2 h_qk d + 2 h_v d + 2 h_v, hidden],
+    W_out ~ N(0, 1/(h_v d)) [hidden, h_v d] and a mixer output y ~ N(0, 1) [T, h_v, d], all bf16
+    (raw bits, round to nearest even), drawn in that order from one PCG64 stream."""
+    rng = np.random.default_rng(seed)
+    n_in = 2 * h_qk * d + 2 * h_v * d + 2 * h_v
+    return {"x": _normal(rng, (T, hidden), "bf16"),
+            "w_in": _normal(rng, (n_in, hidden), "bf16", float(hidden) ** -0.5),
+            "w_out": _normal(rng, (hidden, h_v * d), "bf16", float(h_v * d) ** -0.5),
+            "y": _normal(rng, (T, h_v, d), "bf16")}

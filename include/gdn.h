@@ -184,6 +184,37 @@ int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const
                      const float* conv_w, const float* norm_w, void* conv_state, float* state, void* y,
                      gdn_stream_t stream);
 
+/*
+ * Input projection of the mixer ("Qwen3.8-Flash-Next" technical report, Fig. 2: the query, key
+ * and value streams are projections of the block input, as are the gate inputs a, b and the
+ * output gate z).  One GEMM on the tensor cores, for every token t:
+ *   [q | k | v | z | a | b][t] = W_in x[t]       (fp32 accumulation over `hidden`)
+ *   x      [T][hidden]                  bf16, T = d->total_tokens
+ *   w_in   [N_in][hidden]               bf16, row-major (the nn.Linear layout), rows in the order
+ *                                       q | k | v | z | a | b: N_in = 2 h_qk d_k + 2 h_v d_v + 2 h_v
+ * Outputs, written in the layouts gdn_prefill and gdn_decode take:
+ *   q, k   [T][h_qk][d_k]               bf16 (round to nearest even)
+ *   v, z   [T][h_v][d_v]                bf16
+ *   a, b   [T][h_v]                     fp32
+ * d->in_dtype must be GDN_DTYPE_BF16 and hidden a positive multiple of 64.  The pages print no
+ * weights; tests and benchmarks use synthetic ones.  Asynchronous on `stream`; allocates nothing.
+ * Returns GDN_OK, GDN_ERR_NULL, GDN_ERR_SHAPE, GDN_ERR_DTYPE, GDN_ERR_ALIGN or GDN_ERR_CUDA.
+ */
+int gdn_in_proj(const gdn_dims_t* d, int32_t hidden, const void* x, const void* w_in, void* q, void* k,
+                void* v, void* z, float* a, float* b, gdn_stream_t stream);
+
+/*
+ * Output projection (field guide §02: the gated, RMS-normalised mixer output goes through the
+ * output projection): out[t] = W_out y[t].
+ *   y      [T][h_v d_v]                 bf16 (gdn_prefill's or gdn_decode's y)
+ *   w_out  [hidden][h_v d_v]            bf16, row-major
+ *   out    [T][hidden]                  bf16 (fp32 accumulation, round to nearest even)
+ * d->out_dtype must be GDN_DTYPE_BF16 and hidden a positive multiple of 32.  Same conventions
+ * and return codes as gdn_in_proj.
+ */
+int gdn_out_proj(const gdn_dims_t* d, int32_t hidden, const void* y, const void* w_out, void* out,
+                 gdn_stream_t stream);
+
 /* Static, NUL-terminated name of a return code ("GDN_OK", "GDN_ERR_SHAPE", ...). */
 const char* gdn_status_string(int code);
 

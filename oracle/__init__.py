@@ -2,8 +2,9 @@
 
 Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
 may import this package.  The CUDA library never calls it, and it shares no code with
-the CUDA library: the arithmetic lives in ``gdn_oracle.c`` (plain C, fp64), this module
-only marshals numpy arrays through ctypes.
+the CUDA library: the mixer's arithmetic lives in ``gdn_oracle.c`` (plain C, fp64) and this
+module marshals numpy arrays through ctypes; the two projections around the mixer are one
+fp64 matrix product each (``in_proj``, ``out_proj`` below, numpy).
 
 Element encodings: numpy ``float32`` arrays are fp32 inputs, ``uint16`` arrays are raw
 bf16 bits.  Both are widened exactly to fp64 inside the C code.
@@ -236,3 +237,37 @@ def decode(inp: dict, n_threads: int = 0, q_scale: float = 1.0, l2_eps: float = 
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
     return {"y": y, "y_raw": y_raw, "state": st, "conv_state": cso}
+
+
+# ---- the projections around the mixer ---------------------------------------------------------
+
+def _wide(x: np.ndarray) -> np.ndarray:
+    """Exact fp64 value of raw bf16 bits (uint16) or of fp32 values."""
+    if x.dtype == np.uint16:
+        return (np.ascontiguousarray(x).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.asarray(x, dtype=np.float64)
+
+
+def in_proj(x: np.ndarray, w_in: np.ndarray, h_qk: int, h_v: int, d_k: int = 128, d_v: int = 128):
+    """Input projection ("Qwen3.8-Flash-Next" technical report, Fig. 2: the query, key and value
+    streams -- and the gate inputs a, b and the output gate z -- are projections of the block
+    input): every token's feature vector is W_in x_t, in fp64.  w_in [N_in, hidden] with rows
+    q | k | v | z | a | b.  Returns dict(q [T,h_qk,d_k], k, v [T,h_v,d_v], z, a [T,h_v], b)."""
+    X, W = _wide(x), _wide(w_in)
+    F = X @ W.T
+    T = X.shape[0]
+    nq, nv = h_qk * d_k, h_v * d_v
+    cuts = np.cumsum([0, nq, nq, nv, nv, h_v, h_v])
+    if cuts[-1] != W.shape[0]:
+        raise ValueError("w_in has the wrong number of rows")
+    parts = [F[:, cuts[i]:cuts[i + 1]] for i in range(6)]
+    return {"q": parts[0].reshape(T, h_qk, d_k), "k": parts[1].reshape(T, h_qk, d_k),
+            "v": parts[2].reshape(T, h_v, d_v), "z": parts[3].reshape(T, h_v, d_v),
+            "a": parts[4], "b": parts[5]}
+
+
+def out_proj(y: np.ndarray, w_out: np.ndarray) -> np.ndarray:
+    """Output projection (field guide §02: the gated, RMS-normalised output goes through the
+    output projection): W_out y_t for every token, in fp64.  y [T, h_v, d_v] or [T, h_v d_v]."""
+    Y = _wide(y)
+    return Y.reshape(Y.shape[0], -1) @ _wide(w_out).T

@@ -389,3 +389,58 @@ def test_decode_exact_state_roundtrip(oracle_mod):
         r = oracle_mod.prefill(pre)
         assert rel(r["y"][3], o["y"][n]) < 1e-12
         assert rel(r["final_state"][0], o["state"][n]) < 1e-12
+
+
+# ---- the projections around the mixer (technical report Fig. 2; field guide §02) -----------
+
+def _bits(a):
+    return (np.asarray(a, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_projections_brute_force_tiny(oracle_mod):
+    """A triple loop over (token, feature, input) on values that are exact in bf16."""
+    oracle = oracle_mod
+    rng = np.random.default_rng(3)
+    T, hidden, h_qk, h_v, d = 3, 8, 1, 1, 2
+    n_in = 2 * h_qk * d + 2 * h_v * d + 2 * h_v
+    x = rng.integers(-4, 5, size=(T, hidden)).astype(np.float32)
+    w = rng.integers(-4, 5, size=(n_in, hidden)).astype(np.float32)
+    o = oracle.in_proj(_bits(x), _bits(w), h_qk, h_v, d, d)
+    flat = np.concatenate([o["q"].reshape(T, -1), o["k"].reshape(T, -1), o["v"].reshape(T, -1),
+                           o["z"].reshape(T, -1), o["a"], o["b"]], axis=1)
+    for t in range(T):
+        for n in range(n_in):
+            acc = 0.0
+            for i in range(hidden):
+                acc += float(x[t, i]) * float(w[n, i])
+            assert flat[t, n] == acc
+    wo = rng.integers(-4, 5, size=(5, h_v * d)).astype(np.float32)
+    y = rng.integers(-4, 5, size=(T, h_v, d)).astype(np.float32)
+    out = oracle.out_proj(_bits(y), _bits(wo))
+    for t in range(T):
+        for n in range(5):
+            assert out[t, n] == sum(float(y.reshape(T, -1)[t, i]) * float(wo[n, i]) for i in range(h_v * d))
+
+
+def test_in_proj_row_order_and_head_layout(oracle_mod):
+    """Selector weights: row n of W_in picks input feature n % hidden, scaled by its block's
+    number (q 1, k 2, v 3, z 4, a 5, b 6), so every output lands where the mixer reads it."""
+    oracle = oracle_mod
+    T, hidden, h_qk, h_v, d = 2, 16, 2, 4, 4
+    nq, nv = h_qk * d, h_v * d
+    sizes = [nq, nq, nv, nv, h_v, h_v]
+    w = np.zeros((sum(sizes), hidden), np.float32)
+    r = 0
+    for blk, sz in enumerate(sizes):
+        for i in range(sz):
+            w[r, r % hidden] = blk + 1
+            r += 1
+    x = np.arange(T * hidden, dtype=np.float32).reshape(T, hidden) + 1
+    o = oracle.in_proj(_bits(x), _bits(w), h_qk, h_v, d, d)
+    r = 0
+    for blk, name in enumerate(("q", "k", "v", "z", "a", "b")):
+        arr = o[name].reshape(T, -1)
+        for i in range(arr.shape[1]):
+            assert np.array_equal(arr[:, i], (blk + 1) * x[:, r % hidden])
+            r += 1
+    assert o["q"].shape == (T, h_qk, d) and o["v"].shape == (T, h_v, d) and o["a"].shape == (T, h_v)
