@@ -58,7 +58,7 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     p.add_argument("--decode-steps", type=int, default=None)
-    p.add_argument("--profile", choices=["prefill", "decode", "decode_multi"], default=None,
+    p.add_argument("--profile", choices=["prefill", "decode", "decode_multi", "proj"], default=None,
                    help="only run W + K calls of one workload (for ncu captures; prints no bench line)")
     p.add_argument("--configs", action="store_true",
                    help="time every workload (GPU and the oracle on a bounded sample) instead of the bench step")
@@ -181,6 +181,7 @@ KERNEL_SOURCES = {
     "chunk_prep_tc": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "chunk_scan_tc_norm": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "decode_multi": ("k_decode_multi.cuh", "gdn_common.cuh"),
+    "proj_gemm": ("k_proj.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "decode": ("k_decode.cuh", "gdn_common.cuh"),
     "chunk_phaseB_simt": ("k_chunk_simt.cuh", "gdn_common.cuh"),
 }
@@ -517,6 +518,44 @@ def gpu_arm(args):
               "slots_ms_per_step": slots_ms, "multi_token": multi}
     del dd
 
+    # --- the projections around the mixer at T = 4096 (tcgen05 GEMMs), synthetic weights --------
+    proj = None
+    try:
+        from gated_deltanet_token_b200.inputs import make_proj_inputs
+
+        pp = make_proj_inputs(T, 2048, 16, 32, seed=rank)
+        xp, wi, wo = to_dev(pp["x"], dev), to_dev(pp["w_in"], dev), to_dev(pp["w_out"], dev)
+        del pp
+        pouts = gdn.gdn_in_proj(xp, wi, 16, 32)
+        yo = torch.empty((T, 2048), dtype=torch.bfloat16, device=dev)
+
+        def time_call(fn, reps=20):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            barrier()
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            return max_over_ranks(e0.elapsed_time(e1), dev) / reps
+
+        ms_in = time_call(lambda: gdn.gdn_in_proj(xp, wi, 16, 32, out=pouts))
+        ms_out = time_call(lambda: gdn.gdn_out_proj(y, wo, 16, 32, out=yo))
+        fl_in = 2.0 * T * 2048 * wi.shape[0]
+        fl_out = 2.0 * T * 4096 * 2048
+        pk = float(peaks["bf16_tflops"])
+        proj = {"in_proj_us": ms_in * 1e3, "in_proj_tflops": fl_in / (ms_in / 1e3) / 1e12,
+                "out_proj_us": ms_out * 1e3, "out_proj_tflops": fl_out / (ms_out / 1e3) / 1e12,
+                "peak_tflops": pk, "peak_source": f"{peak_src} bf16_tflops",
+                "in_proj_frac": fl_in / (ms_in / 1e3) / 1e12 / pk, "out_proj_frac": fl_out / (ms_out / 1e3) / 1e12 / pk,
+                "shape": "x [4096, 2048] -> 12352 features; y [4096, 4096] -> 2048"}
+        del xp, wi, wo, pouts, yo
+    except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
+        proj = f"failed: {exc}"
+
     # --- end to end through the public call with host buffers ----------------------------------
     # Every step copies its own inputs in from pinned host memory and its y and final state back
     # out.  Three streams (host->device copies, the prefill, device->host copies) and two buffer
@@ -595,7 +634,7 @@ def gpu_arm(args):
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "pipeline": "3 streams, 2 slots", "matches_device": e2e_match},
-        "gpu_launches": launches, "clocks": clk, "decode": decode,
+        "gpu_launches": launches, "clocks": clk, "decode": decode, "projections": proj,
     }
     print(json.dumps(out), flush=True)
     return 0
@@ -719,7 +758,15 @@ def profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     n = args.warmup + args.steps
-    if args.profile == "prefill":
+    if args.profile == "proj":
+        from gated_deltanet_token_b200.inputs import make_proj_inputs
+
+        pp = make_proj_inputs(4096, 2048, 16, 32)
+        x, wi, wo, y = (to_dev(pp[k], dev) for k in ("x", "w_in", "w_out", "y"))
+        for _ in range(n):
+            gdn.gdn_in_proj(x, wi, 16, 32)
+            gdn.gdn_out_proj(y, wo, 16, 32)
+    elif args.profile == "prefill":
         inp = make_inputs(WORKLOAD)
         d = {k: to_dev(inp[k], dev) for k in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w", "norm_w")}
         y = torch.empty((inp["spec"]["T"], 32, 128), dtype=torch.bfloat16, device=dev)
