@@ -173,6 +173,45 @@ def recurrence(qh, kh, v, g, beta, S0, q_scale: float = 1.0, chunk: int = 0):
     return y, S
 
 
+def recurrence_backward(qh, kh, v, g, beta, S0, dy, dS_T):
+    """Reverse-mode gradients of the recurrence core of one (sequence, value head), in fp64.
+
+    The forward is field guide §02's per-token rule (column-vector S, d_v x d_k), with
+    alpha_t = e^{g_t}:  S'_t = alpha_t S_{t-1};  e_t = v_t - S'_t k_t;
+    S_t = S'_t + beta_t e_t k_t^T;  y_t = S_t q_t.  Given dy [T, d_v] (dL/dy_t) and dS_T
+    (dL/dS_T), walking the tokens from the last with D = dL/dS_t:
+      D += dy_t q_t^T;  dq_t = S_t^T dy_t;  w = D k_t;  de_t = beta_t w;  dbeta_t = e_t . w;
+      dv_t = de_t;  dk_t = beta_t D^T e_t - S'_t^T de_t;  dS'_t = D - de_t k_t^T;
+      dg_t = alpha_t <dS'_t, S_{t-1}>;  D <- alpha_t dS'_t.
+    Returns dict(dq [T, d_k], dk [T, d_k], dv [T, d_v], dg [T], dbeta [T], dS0 [d_v, d_k])."""
+    qh, kh, v, g, beta, dy = map(lambda a: np.asarray(a, np.float64), (qh, kh, v, g, beta, dy))
+    T = kh.shape[0]
+    S = [np.asarray(S0, np.float64).copy()]
+    for t in range(T):  # the forward, keeping every state
+        Sp = np.exp(g[t]) * S[-1]
+        e = v[t] - Sp @ kh[t]
+        S.append(Sp + beta[t] * np.outer(e, kh[t]))
+    D = np.asarray(dS_T, np.float64).copy()
+    out = {"dq": np.zeros_like(qh), "dk": np.zeros_like(kh), "dv": np.zeros_like(v),
+           "dg": np.zeros(T), "dbeta": np.zeros(T)}
+    for t in range(T - 1, -1, -1):
+        a = np.exp(g[t])
+        Sp = a * S[t]
+        e = v[t] - Sp @ kh[t]
+        D = D + np.outer(dy[t], qh[t])
+        out["dq"][t] = S[t + 1].T @ dy[t]
+        w = D @ kh[t]
+        de = beta[t] * w
+        out["dbeta"][t] = e @ w
+        out["dv"][t] = de
+        out["dk"][t] = beta[t] * (D.T @ e) - Sp.T @ de
+        dSp = D - np.outer(de, kh[t])
+        out["dg"][t] = a * np.sum(dSp * S[t])
+        D = a * dSp
+    out["dS0"] = D
+    return out
+
+
 # ---- whole mixer ----------------------------------------------------------------------
 
 def _dims(n_seqs, total, h_qk, h_v, d_k, d_v, enc, q_scale, l2_eps, rms_eps, chunk, threads):

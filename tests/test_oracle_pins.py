@@ -444,3 +444,53 @@ def test_in_proj_row_order_and_head_layout(oracle_mod):
             assert np.array_equal(arr[:, i], (blk + 1) * x[:, r % hidden])
             r += 1
     assert o["q"].shape == (T, h_qk, d) and o["v"].shape == (T, h_v, d) and o["a"].shape == (T, h_v)
+
+
+# ---- the backward of the recurrence core (NEXT-4) --------------------------------------------
+
+def test_recurrence_backward_matches_finite_differences(oracle_mod):
+    """Every gradient of the reverse-mode oracle against central differences of the forward
+    recurrence (the C per-token rule) of L = sum dy . y + <dS_T, S_T>, on a tiny case."""
+    rng = np.random.default_rng(7)
+    T, d = 5, 4
+    qh = rng.standard_normal((T, d)); kh = rng.standard_normal((T, d))
+    kh /= np.linalg.norm(kh, axis=1, keepdims=True)
+    v = rng.standard_normal((T, d)); g = -rng.uniform(0.05, 1.0, T); beta = rng.uniform(0.1, 0.9, T)
+    S0 = rng.standard_normal((d, d)) * 0.3
+    dy = rng.standard_normal((T, d)); dST = rng.standard_normal((d, d))
+
+    def loss(qh_, kh_, v_, g_, b_, S0_):
+        y, S = oracle_mod.recurrence(qh_, kh_, v_, g_, b_, S0_)
+        return float(np.sum(dy * y) + np.sum(dST * S))
+
+    got = oracle_mod.recurrence_backward(qh, kh, v, g, beta, S0, dy, dST)
+    args = [qh, kh, v, g, beta, S0]
+    names = ["dq", "dk", "dv", "dg", "dbeta", "dS0"]
+    h = 1e-6
+    for ai, name in enumerate(names):
+        base = args[ai]
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[ai][idx] += h
+            minus[ai][idx] -= h
+            fd[idx] = (loss(*plus) - loss(*minus)) / (2 * h)
+        np.testing.assert_allclose(got[name], fd, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_recurrence_backward_zero_write_is_pure_decay(oracle_mod):
+    """beta = 0: the state only decays, S_T = e^{sum g} S_0, y_t = e^{gamma_t} S_0 q_t; then
+    dv = 0, dS_0 = sum_t e^{gamma_t} dy_t q_t^T + e^{gamma_T} dS_T in closed form."""
+    rng = np.random.default_rng(8)
+    T, d = 6, 3
+    qh = rng.standard_normal((T, d)); kh = rng.standard_normal((T, d)); v = rng.standard_normal((T, d))
+    g = -rng.uniform(0.1, 0.5, T); beta = np.zeros(T); S0 = rng.standard_normal((d, d))
+    dy = rng.standard_normal((T, d)); dST = rng.standard_normal((d, d))
+    got = oracle_mod.recurrence_backward(qh, kh, v, g, beta, S0, dy, dST)
+    gam = np.cumsum(g)
+    want = sum(np.exp(gam[t]) * np.outer(dy[t], qh[t]) for t in range(T)) + np.exp(gam[-1]) * dST
+    np.testing.assert_allclose(got["dS0"], want, rtol=1e-12, atol=1e-12)
+    assert np.all(got["dv"] == 0)
