@@ -19,6 +19,7 @@
 #include "k_decode.cuh"
 #include "k_decode_multi.cuh"
 #include "k_proj.cuh"
+#include "k_bwd.cuh"
 #include "k_stream.cuh"
 
 using namespace gdn;
@@ -583,6 +584,31 @@ int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// Workspace of the recurrence backward, carved from the caller's buffer in this order.
+struct BwWs {
+  size_t tab, seqc0, ck, scr, dqh, dkh, total;
+  int max_chunks;
+};
+BwWs bw_ws(const gdn_dims_t* d) {
+  BwWs L{};
+  const size_t T = (size_t)d->total_tokens, hv = (size_t)d->h_v, N = (size_t)d->n_seqs;
+  L.max_chunks = (int)((T + CH - 1) / CH + N);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.tab = take((size_t)L.max_chunks * sizeof(ChunkEntry));
+  L.seqc0 = take((N + 1) * sizeof(int));
+  L.ck = take((size_t)L.max_chunks * hv * BW_CK_FLOATS * 4);
+  L.scr = take(N * hv * BW_SCR_FLOATS * 4);
+  L.dqh = take(T * hv * D * 4);
+  L.dkh = take(T * hv * D * 4);
+  L.total = off;
+  return L;
+}
+
 // C = A B^T on tcgen05 into the output segments of `po` (M rows of A, N rows of B, K columns).
 static int proj_launch(const void* A, long long M, const void* B, int N, int K, const ProjOut& po,
                        gdn_stream_t stream) {
@@ -653,6 +679,52 @@ int gdn_out_proj(const gdn_dims_t* d, int32_t hidden, const void* y, const void*
   po.seg[0].f32 = 0;
   po.seg[0].out = out;
   return proj_launch(y, d->total_tokens, w_out, hidden, K, po, stream);
+}
+
+size_t gdn_recurrence_backward_workspace_size(const gdn_dims_t* d) {
+  if (check_dims(d, false) != GDN_OK) return 0;
+  return bw_ws(d).total;
+}
+
+int gdn_recurrence_backward(const gdn_dims_t* d, const float* qh, const float* kh, const float* v, const float* g,
+                            const float* beta, const float* init_state, const int32_t* cu_seqlens, const float* dy,
+                            const float* dS_final, float* dq, float* dk, float* dv, float* dg, float* dbeta,
+                            float* dS_init, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+  int rc = check_dims(d, false);
+  if (rc != GDN_OK) return rc;
+  if (!dS_init) return GDN_ERR_NULL;
+  if (d->total_tokens > 0 && (!qh || !kh || !v || !g || !beta || !dy || !dq || !dk || !dv || !dg || !dbeta))
+    return GDN_ERR_NULL;
+  if (!cu_seqlens && d->n_seqs != 1) return GDN_ERR_NULL;
+  const void* ptrs[] = {qh, kh, v, g, beta, init_state, cu_seqlens, dy, dS_final, dq, dk, dv, dg, dbeta, dS_init,
+                        workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+  const BwWs L = bw_ws(d);
+  if (!workspace || workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+  rc = configure_device();
+  if (rc != GDN_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  ChunkEntry* tab = reinterpret_cast<ChunkEntry*>(ws + L.tab);
+  int* seqc0 = reinterpret_cast<int*>(ws + L.seqc0);
+  const Dims kd = kdims(d);
+  if (cu_seqlens) {
+    ProfScope p("tilemap", s);
+    k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0);
+  }
+  {
+    ProfScope p("recurrence_bwd", s);
+    k_bwd<<<dim3(d->n_seqs, d->h_v), BW_THREADS, 0, s>>>(kd, cu_seqlens, cu_seqlens ? seqc0 : nullptr, qh, kh, v, g,
+                                                         beta, init_state, dy, dS_final, dv, dg, dbeta, dS_init,
+                                                         F(L.ck), F(L.scr), F(L.dqh), F(L.dkh));
+  }
+  if (d->total_tokens > 0) {
+    ProfScope p("recurrence_bwd_sum", s);
+    k_bwd_sum<<<dim3(d->total_tokens, d->h_qk), D, 0, s>>>(kd, F(L.dqh), F(L.dkh), dq, dk);
+  }
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 int gdn_prefill_conv_state(const gdn_dims_t* d, const void* q, const void* k, const void* v,

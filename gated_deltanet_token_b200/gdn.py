@@ -77,6 +77,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_in_proj.argtypes = [dp, ctypes.c_int32] + [vp] * 8 + [vp]
         L.gdn_out_proj.restype = ctypes.c_int
         L.gdn_out_proj.argtypes = [dp, ctypes.c_int32] + [vp] * 3 + [vp]
+        L.gdn_recurrence_backward_workspace_size.restype = ctypes.c_size_t
+        L.gdn_recurrence_backward_workspace_size.argtypes = [dp]
+        L.gdn_recurrence_backward.restype = ctypes.c_int
+        L.gdn_recurrence_backward.argtypes = [dp] + [vp] * 15 + [vp, ctypes.c_size_t, vp]
         L.gdn_prefill_conv_state.restype = ctypes.c_int
         L.gdn_prefill_conv_state.argtypes = [dp] + [vp] * 5 + [vp]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -380,3 +384,33 @@ def gdn_out_proj(y, w_out, h_qk, h_v, *, d_v=128, out=None, stream=None):
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_out_proj")
     return out
+
+
+def gdn_recurrence_backward(qh, kh, v, g, beta, init_state, cu_seqlens, dy, dS_final, *, workspace=None,
+                            stream=None):
+    """Gradients of the recurrence core: qh, kh [T, h_qk, d_k], v [T, h_v, d_v], g, beta [T, h_v],
+    init_state [N, h_v, d_v, d_k] or None, cu_seqlens [N + 1] int32 or None (one sequence), dy
+    [T, h_v, d_v] (dL/dy before the output norm), dS_final [N, h_v, d_v, d_k] or None.  All fp32.
+    Returns (dq, dk, dv, dg, dbeta, dS_init)."""
+    T, h_qk, d_k = qh.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    for t in (qh, kh, v, g, beta, dy):
+        if t.dtype != torch.float32:
+            raise TypeError("the backward takes fp32 tensors")
+    dims = make_dims(N, T, h_qk, h_v, GDN_DTYPE_F32, GDN_DTYPE_F32, d_k, d_v)
+    dev = qh.device
+    dq, dk = torch.empty_like(qh), torch.empty_like(kh)
+    dv = torch.empty_like(v)
+    dg, dbeta = torch.empty_like(g), torch.empty_like(beta)
+    dS_init = torch.empty((N, h_v, d_v, d_k), dtype=torch.float32, device=dev)
+    need = lib().gdn_recurrence_backward_workspace_size(ctypes.byref(dims))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    rc = lib().gdn_recurrence_backward(ctypes.byref(dims), _ptr(qh), _ptr(kh), _ptr(v), _ptr(g), _ptr(beta),
+                                       _ptr(init_state), _ptr(cu_seqlens), _ptr(dy), _ptr(dS_final), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dS_init), _ptr(workspace),
+                                       ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrence_backward")
+    return dq, dk, dv, dg, dbeta, dS_init

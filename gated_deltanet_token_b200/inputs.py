@@ -131,3 +131,31 @@ def make_proj_inputs(T: int, hidden: int = 2048, h_qk: int = 16, h_v: int = 32, 
             "w_in": _normal(rng, (n_in, hidden), "bf16", float(hidden) ** -0.5),
             "w_out": _normal(rng, (hidden, h_v * d), "bf16", float(h_v * d) ** -0.5),
             "y": _normal(rng, (T, h_v, d), "bf16")}
+
+
+def make_bwd_inputs(lengths, h_qk: int = 2, h_v: int = 4, d: int = 128, seed: int = 0) -> dict:
+    """Synthetic inputs of the recurrence core's backward pass (fp32): unit query and key
+    vectors qh, kh [T, h_qk, d]; v ~ N(0, 1) [T, h_v, d]; the decay g = -exp(A_log) softplus(a +
+    dt_bias) with the configs' distributions and beta = sigmoid(b), both [T, h_v]; initial states
+    ~ N(0, 0.02^2) [N, h_v, d, d]; upstream gradients dy ~ N(0, 1) [T, h_v, d] and dS_T ~ N(0,
+    0.02^2).  `lengths` is a list of sequence lengths (packed, cu_seqlens returned)."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lengths, dtype=np.int64)
+    cu = np.zeros(len(lens) + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    T, N = int(cu[-1]), len(lens)
+    qh = rng.standard_normal((T, h_qk, d)).astype(np.float32)
+    kh = rng.standard_normal((T, h_qk, d)).astype(np.float32)
+    qh /= np.maximum(np.linalg.norm(qh, axis=2, keepdims=True), 1e-6)
+    kh /= np.maximum(np.linalg.norm(kh, axis=2, keepdims=True), 1e-6)
+    v = rng.standard_normal((T, h_v, d)).astype(np.float32)
+    A_log = np.log(rng.uniform(1.0, 16.0, size=h_v))
+    dt_bias = rng.standard_normal(h_v) * 0.1
+    a = rng.standard_normal((T, h_v))
+    x = a + dt_bias
+    g = (-np.exp(A_log) * (np.maximum(x, 0) + np.log1p(np.exp(-np.abs(x))))).astype(np.float32)
+    beta = (1.0 / (1.0 + np.exp(-rng.standard_normal((T, h_v))))).astype(np.float32)
+    return {"qh": qh, "kh": kh, "v": v, "g": g, "beta": beta, "cu_seqlens": cu,
+            "init_state": (rng.standard_normal((N, h_v, d, d)) * 0.02).astype(np.float32),
+            "dy": rng.standard_normal((T, h_v, d)).astype(np.float32),
+            "dS_T": (rng.standard_normal((N, h_v, d, d)) * 0.02).astype(np.float32)}

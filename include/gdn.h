@@ -215,6 +215,32 @@ int gdn_in_proj(const gdn_dims_t* d, int32_t hidden, const void* x, const void* 
 int gdn_out_proj(const gdn_dims_t* d, int32_t hidden, const void* y, const void* w_out, void* out,
                  gdn_stream_t stream);
 
+/*
+ * Backward pass of the recurrence core (training).  The forward is the field guide's §02 rule
+ * (steps 1-6) on already convolved and normalised streams, per (sequence, value head h) with QK
+ * head j = h / (h_v / h_qk) and alpha_t = e^{g_t}:
+ *   S'_t = alpha_t S_{t-1};  e_t = v_t - S'_t k_t;  S_t = S'_t + beta_t e_t k_t^T;  y_t = S_t q_t
+ * (the query enters as given: d->q_scale is not applied).  Given dL/dy_t and dL/dS_T, this
+ * call returns dL/dq, dL/dk (summed over the value heads sharing a QK head), dL/dv, dL/dg,
+ * dL/dbeta and dL/dS_0, all fp32:
+ *   qh, kh, dq, dk        [T][h_qk][d_k]
+ *   v, dy, dv             [T][h_v][d_v]        (dy: the gradient of y before the output norm)
+ *   g, beta, dg, dbeta    [T][h_v]             (g: the log-decay, so that alpha = e^g)
+ *   init_state, dS_final, dS_init   [N][h_v][d_v][d_k]   (init_state, dS_final may be NULL: 0)
+ *   cu_seqlens            [N + 1] device int32, or NULL for one sequence
+ * d->in_dtype and d->out_dtype are not read (fp32 throughout).  The workspace holds a state
+ * checkpoint per chunk and value head, 4 MiB per (sequence, value head) of chunk scratch, and
+ * per-value-head dq, dk: gdn_recurrence_backward_workspace_size(d) bytes.  Asynchronous on
+ * `stream`.  Returns GDN_OK, GDN_ERR_NULL, GDN_ERR_SHAPE, GDN_ERR_ALIGN, GDN_ERR_WORKSPACE or
+ * GDN_ERR_CUDA.
+ */
+size_t gdn_recurrence_backward_workspace_size(const gdn_dims_t* d);
+int gdn_recurrence_backward(const gdn_dims_t* d, const float* qh, const float* kh, const float* v,
+                            const float* g, const float* beta, const float* init_state,
+                            const int32_t* cu_seqlens, const float* dy, const float* dS_final, float* dq,
+                            float* dk, float* dv, float* dg, float* dbeta, float* dS_init, void* workspace,
+                            size_t workspace_bytes, gdn_stream_t stream);
+
 /* Static, NUL-terminated name of a return code ("GDN_OK", "GDN_ERR_SHAPE", ...). */
 const char* gdn_status_string(int code);
 
