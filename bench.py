@@ -182,6 +182,7 @@ KERNEL_SOURCES = {
     "chunk_scan_tc_norm": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "decode_multi": ("k_decode_multi.cuh", "gdn_common.cuh"),
     "proj_gemm": ("k_proj.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
+    "recurrence_bwd": ("k_bwd.cuh", "gdn_common.cuh"),
     "decode": ("k_decode.cuh", "gdn_common.cuh"),
     "chunk_phaseB_simt": ("k_chunk_simt.cuh", "gdn_common.cuh"),
 }
@@ -556,6 +557,38 @@ def gpu_arm(args):
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         proj = f"failed: {exc}"
 
+    # --- the backward of the recurrence core at T = 4096 (fp32), synthetic inputs ---------------
+    bwd = None
+    try:
+        from gated_deltanet_token_b200.inputs import make_bwd_inputs
+
+        bi = make_bwd_inputs([T], 16, 32, seed=rank)
+        bt = {k: to_dev(bi[k], dev) for k in ("qh", "kh", "v", "g", "beta", "init_state", "dy", "dS_T")}
+        del bi
+        bdims = gdn.make_dims(1, T, 16, 32, gdn.GDN_DTYPE_F32, gdn.GDN_DTYPE_F32)
+        bws = torch.empty(gdn.lib().gdn_recurrence_backward_workspace_size(bdims), dtype=torch.uint8, device=dev)
+
+        def bcall():
+            gdn.gdn_recurrence_backward(bt["qh"], bt["kh"], bt["v"], bt["g"], bt["beta"], bt["init_state"], None,
+                                        bt["dy"], bt["dS_T"], workspace=bws)
+
+        for _ in range(2):
+            bcall()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(5):
+            bcall()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        bms = max_over_ranks(e0.elapsed_time(e1), dev) / 5
+        bwd = {"ms_per_call": bms, "tokens_per_s": T / (bms / 1e3), "workspace_MB": bws.numel() / 1e6,
+               "shape": "T=4096, 16 QK / 32 value heads, fp32, one sequence"}
+        del bt, bws
+    except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
+        bwd = f"failed: {exc}"
+
     # --- end to end through the public call with host buffers ----------------------------------
     # Every step copies its own inputs in from pinned host memory and its y and final state back
     # out.  Three streams (host->device copies, the prefill, device->host copies) and two buffer
@@ -635,6 +668,7 @@ def gpu_arm(args):
         "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "pipeline": "3 streams, 2 slots", "matches_device": e2e_match},
         "gpu_launches": launches, "clocks": clk, "decode": decode, "projections": proj,
+        "backward": bwd,
     }
     print(json.dumps(out), flush=True)
     return 0
