@@ -286,6 +286,7 @@ int configure_device() {
       cudaFuncSetAttribute(k_chunkscan_tc<PB_Y_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)PB_TC_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_proj_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PJ_SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(k_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BW_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_decode_multi<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)DECM_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(k_decode_multi<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -586,7 +587,7 @@ int gdn_decode_multi(const gdn_dims_t* d, int32_t n_tokens, const void* q, const
 
 // Workspace of the recurrence backward, carved from the caller's buffer in this order.
 struct BwWs {
-  size_t tab, seqc0, ck, scr, dqh, dkh, total;
+  size_t tab, seqc0, ck, part, total;
   int max_chunks;
 };
 BwWs bw_ws(const gdn_dims_t* d) {
@@ -602,9 +603,7 @@ BwWs bw_ws(const gdn_dims_t* d) {
   L.tab = take((size_t)L.max_chunks * sizeof(ChunkEntry));
   L.seqc0 = take((N + 1) * sizeof(int));
   L.ck = take((size_t)L.max_chunks * hv * BW_CK_FLOATS * 4);
-  L.scr = take(N * hv * BW_SCR_FLOATS * 4);
-  L.dqh = take(T * hv * D * 4);
-  L.dkh = take(T * hv * D * 4);
+  L.part = take((size_t)BW_SL * T * hv * BW_RED * 4);
   L.total = off;
   return L;
 }
@@ -716,13 +715,13 @@ int gdn_recurrence_backward(const gdn_dims_t* d, const float* qh, const float* k
   }
   {
     ProfScope p("recurrence_bwd", s);
-    k_bwd<<<dim3(d->n_seqs, d->h_v), BW_THREADS, 0, s>>>(kd, cu_seqlens, cu_seqlens ? seqc0 : nullptr, qh, kh, v, g,
-                                                         beta, init_state, dy, dS_final, dv, dg, dbeta, dS_init,
-                                                         F(L.ck), F(L.scr), F(L.dqh), F(L.dkh));
+    k_bwd<<<dim3(d->n_seqs, d->h_v, BW_SL), BW_THREADS, BW_SMEM, s>>>(
+        kd, cu_seqlens, cu_seqlens ? seqc0 : nullptr, qh, kh, v, g, beta, init_state, dy, dS_final, dv, dS_init,
+        F(L.ck), F(L.part));
   }
   if (d->total_tokens > 0) {
     ProfScope p("recurrence_bwd_sum", s);
-    k_bwd_sum<<<dim3(d->total_tokens, d->h_qk), D, 0, s>>>(kd, F(L.dqh), F(L.dkh), dq, dk);
+    k_bwd_sum<<<dim3(d->total_tokens, d->h_qk), D, 0, s>>>(kd, F(L.part), g, dq, dk, dbeta, dg);
   }
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -229,8 +229,9 @@ int gdn_out_proj(const gdn_dims_t* d, int32_t hidden, const void* y, const void*
  *   init_state, dS_final, dS_init   [N][h_v][d_v][d_k]   (init_state, dS_final may be NULL: 0)
  *   cu_seqlens            [N + 1] device int32, or NULL for one sequence
  * d->in_dtype and d->out_dtype are not read (fp32 throughout).  The workspace holds a state
- * checkpoint per chunk and value head, 4 MiB per (sequence, value head) of chunk scratch, and
- * per-value-head dq, dk: gdn_recurrence_backward_workspace_size(d) bytes.  Asynchronous on
+ * checkpoint per chunk and value head (64 KiB each) and, per token and value head, the partial
+ * sums of dq, dk, dbeta and dg of each of the 4 row slices (4 x 1032 bytes):
+ * gdn_recurrence_backward_workspace_size(d) bytes.  Asynchronous on
  * `stream`.  Returns GDN_OK, GDN_ERR_NULL, GDN_ERR_SHAPE, GDN_ERR_ALIGN, GDN_ERR_WORKSPACE or
  * GDN_ERR_CUDA.
  */
