@@ -58,7 +58,7 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     p.add_argument("--decode-steps", type=int, default=None)
-    p.add_argument("--profile", choices=["prefill", "decode", "decode_multi", "proj"], default=None,
+    p.add_argument("--profile", choices=["prefill", "decode", "decode_multi", "proj", "bwd"], default=None,
                    help="only run W + K calls of one workload (for ncu captures; prints no bench line)")
     p.add_argument("--configs", action="store_true",
                    help="time every workload (GPU and the oracle on a bounded sample) instead of the bench step")
@@ -800,6 +800,16 @@ def profile_case(args):
         for _ in range(n):
             gdn.gdn_in_proj(x, wi, 16, 32)
             gdn.gdn_out_proj(y, wo, 16, 32)
+    elif args.profile == "bwd":
+        from gated_deltanet_token_b200.inputs import make_bwd_inputs
+
+        bi = make_bwd_inputs([4096], 16, 32)
+        bt = {k: to_dev(bi[k], dev) for k in ("qh", "kh", "v", "g", "beta", "init_state", "dy", "dS_T")}
+        bdims = gdn.make_dims(1, 4096, 16, 32, gdn.GDN_DTYPE_F32, gdn.GDN_DTYPE_F32)
+        bws = torch.empty(gdn.lib().gdn_recurrence_backward_workspace_size(bdims), dtype=torch.uint8, device=dev)
+        for _ in range(n):
+            gdn.gdn_recurrence_backward(bt["qh"], bt["kh"], bt["v"], bt["g"], bt["beta"], bt["init_state"], None,
+                                        bt["dy"], bt["dS_T"], workspace=bws)
     elif args.profile == "prefill":
         inp = make_inputs(WORKLOAD)
         d = {k: to_dev(inp[k], dev) for k in ("q", "k", "v", "z", "a", "b", "A_log", "dt_bias", "conv_w", "norm_w")}

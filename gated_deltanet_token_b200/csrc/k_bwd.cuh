@@ -10,15 +10,21 @@
 // Rows of S (value components) evolve independently in both directions; only dq, dk, dbeta and
 // dg sum over rows.  So one CTA of 256 threads serves one (sequence, value head, slice of 32
 // rows): warp w owns slice rows 4w .. 4w + 3, lane l columns 4l .. 4l + 3, 16 elements of S
-// (forward) and of D (reverse) per thread.  Row dot products (S' k, D k) are warp reductions;
-// the column sums of dq, dk and the scalars dbeta, dg are reduced over the 8 warps through
-// shared memory (double-buffered by token parity, one barrier per token) and written per slice;
-// k_bwd_sum adds the slices and the value heads that share a QK head, in a fixed order.
-//   1. Forward over the sequence, storing the state at every 64-token chunk start (global).
-//   2. For each chunk from the last: its inputs go to shared memory; a forward pass over the
-//      chunk keeps the state at every 8th token in shared memory; then, per 8-token sub-chunk
-//      from the last, the 8 states before its tokens are recomputed into registers and the
-//      sub-chunk's tokens are walked in reverse.  No state sequence goes through global memory.
+// (forward) and of D (reverse) per thread.  Row dot products are warp reductions: one group per
+// forward token (S_{t-1} k_t) and one per reverse token (D' k_t and <D', S_{t-1}> together, with
+// D' = D + dy q^T, since <dS', S_{t-1}> = <D', S_{t-1}> - sum_r de_r (S_{t-1} k_t)_r).  The
+// column sums of dq, dk and the scalars dbeta, dg are reduced over the 8 warps through shared
+// memory and written per slice, one token later (three buffers, one barrier per token), so the
+// sum is off the token chain; k_bwd_sum adds the slices and the value heads that share a QK
+// head, in a fixed order.
+//   1. Forward over the sequence, storing the state at every 64-token chunk start (global);
+//      the next chunk's inputs are copied to shared memory (cp.async) during the current one.
+//   2. For each chunk from the last: its k, v, g, beta go to shared memory; a forward pass over
+//      the chunk keeps the state at every 8th token in shared memory; then, per 8-token
+//      sub-chunk from the last, the 8 states before its tokens are recomputed into registers
+//      (with S_{t-1} k_t to shared memory) and the sub-chunk's tokens are walked in reverse,
+//      while the next sub-chunk's q and dy rows are copied in.  No state sequence goes
+//      through global memory.
 #pragma once
 #include "gdn_common.cuh"
 
@@ -34,40 +40,59 @@ constexpr int BW_SUB = 8;                              // tokens per sub-chunk
 constexpr int BW_NSUB = CH / BW_SUB;                   // sub-chunks per chunk
 constexpr int BW_RED = 2 * D + 2;                      // dq | dk | dbeta | dalpha partials
 constexpr int BW_RED_LD = 2 * D + 4;                   // their row pitch (16-byte aligned rows)
+constexpr int BW_NRED = 3;                             // partial buffers: a token's are summed one token later
 constexpr size_t BW_CK_FLOATS = (size_t)D * D;         // one checkpoint of a value head's state
 
-// Shared memory, in floats: the chunk's k, q (64 x 128), v and dy of the slice (64 x 32),
-// alpha and beta (64); the sub-chunk checkpoints ([8][4 quads][256 threads] float4, so that a
-// warp's accesses are consecutive); the per-warp partials [2][8][BW_RED_LD].
-constexpr int BWS_K = 0, BWS_Q = BWS_K + CH * D, BWS_V = BWS_Q + CH * D, BWS_DY = BWS_V + CH * BW_NR;
-constexpr int BWS_A = BWS_DY + CH * BW_NR, BWS_B = BWS_A + CH, BWS_SUBCK = BWS_B + CH;
-constexpr int BWS_RED = BWS_SUBCK + BW_NSUB * BW_EL * BW_THREADS;
-constexpr size_t BW_SMEM = (size_t)(BWS_RED + 2 * BW_WARPS * BW_RED_LD) * 4;
+// A chunk's input block (floats): k [64][128], v of the slice [64][32], g [64], beta [64].
+constexpr int BWI_K = 0, BWI_V = CH * D, BWI_G = BWI_V + CH * BW_NR, BWI_B = BWI_G + CH, BWI_FLOATS = BWI_B + CH;
+// Shared memory (floats): the input block; the sub-chunk checkpoints ([8][4 quads][256 threads]
+// float4, a warp's accesses consecutive), which hold the second input block during the forward
+// sweep; q and dy rows of a sub-chunk, double-buffered ([2][8][128], [2][8][32]); S_{t-1} k_t of
+// the sub-chunk ([8 tokens][8 warps][4 rows]); the per-warp partials [3][8][BW_RED_LD].
+constexpr int BWS_IN = 0, BWS_SUBCK = BWS_IN + BWI_FLOATS;
+constexpr int BWS_Q = BWS_SUBCK + BW_NSUB * BW_EL * BW_THREADS, BWS_DY = BWS_Q + 2 * BW_SUB * D;
+constexpr int BWS_SK = BWS_DY + 2 * BW_SUB * BW_NR, BWS_RED = BWS_SK + BW_SUB * BW_WARPS * BW_ROWS;
+constexpr size_t BW_SMEM = (size_t)(BWS_RED + BW_NRED * BW_WARPS * BW_RED_LD) * 4;
 static_assert(BW_SMEM <= 227 * 1024, "k_bwd shared memory");
+static_assert(BWI_FLOATS <= BW_NSUB * BW_EL * BW_THREADS, "the second input block fits the sub-checkpoints");
+static_assert(BWS_SUBCK % 4 == 0 && BWS_Q % 4 == 0 && BWS_DY % 4 == 0 && BWS_SK % 4 == 0 && BWS_RED % 4 == 0,
+              "16-byte aligned regions");
 
-// One forward token on the thread's elements (rows r of BW_ROWS, columns c of 4): S <- S'' with
-// e_r = v_r - (alpha S k)_r.  k4: the thread's 4 key components; vrow: the warp's BW_ROWS values.
-__device__ __forceinline__ void bw_forward_token(float (&S)[BW_EL], float a, float bt, const float4 k4,
-                                                 const float* vrow) {
+__device__ __forceinline__ void bw_cp16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bw_cp4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bw_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bw_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One forward token on the thread's elements (rows r of BW_ROWS, columns c of 4):
+// sk_r = (S k)_r, e_r = beta (v_r - alpha sk_r), S <- alpha S + e k^T.  k4: the thread's 4 key
+// components; vrow: the warp's BW_ROWS values.  Every pass runs this same arithmetic.
+__device__ __forceinline__ void bw_forward_token(float (&S)[BW_EL], float (&sk)[BW_ROWS], float a, float bt,
+                                                 const float4 k4, const float* vrow, bool update) {
   const float kc[4] = {k4.x, k4.y, k4.z, k4.w};
-  float u[BW_ROWS];
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r) {
     float s = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      S[4 * r + c] *= a;
-      s = fmaf(S[4 * r + c], kc[c], s);
-    }
-    u[r] = s;
+    for (int c = 0; c < 4; ++c) s = fmaf(S[4 * r + c], kc[c], s);
+    sk[r] = s;
   }
 #pragma unroll
-  for (int r = 0; r < BW_ROWS; ++r) u[r] = warp_sum(u[r]);
+  for (int r = 0; r < BW_ROWS; ++r) sk[r] = warp_sum(sk[r]);
+  if (!update) return;
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r) {
-    const float e = bt * (vrow[r] - u[r]);
+    const float e = bt * (vrow[r] - a * sk[r]);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) S[4 * r + c] = fmaf(e, kc[c], S[4 * r + c]);
+    for (int c = 0; c < 4; ++c) S[4 * r + c] = fmaf(e, kc[c], a * S[4 * r + c]);
   }
 }
 
@@ -87,52 +112,55 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   const int i0 = sl * BW_NR;                       // the slice's first state row
   const int r0 = warp * BW_ROWS, c0 = lane * 4;    // slice rows r0 .. r0 + 3, columns c0 .. c0 + 3
   const size_t sbase = ((size_t)n * hv + h) * D * D;
+  const size_t T = (size_t)d.total_tokens;
   auto elem = [&](int r, int c) { return (size_t)(i0 + r0 + r) * D + c0 + c; };
-  float* sK = bsm + BWS_K;
-  float* sQ = bsm + BWS_Q;
-  float* sV = bsm + BWS_V;
-  float* sDY = bsm + BWS_DY;
-  float* sA = bsm + BWS_A;
-  float* sB = bsm + BWS_B;
-  float4* sSub = reinterpret_cast<float4*>(bsm + BWS_SUBCK);
-  float* red = bsm + BWS_RED;
+  float* const in0 = bsm + BWS_IN;
+  float* const in1 = bsm + BWS_SUBCK;  // the forward sweep's second input block
+  float4* const sSub = reinterpret_cast<float4*>(bsm + BWS_SUBCK);
+  float* const sQ = bsm + BWS_Q;
+  float* const sDY = bsm + BWS_DY;
+  float* const sSK = bsm + BWS_SK;
+  float* const red = bsm + BWS_RED;
   // checkpoint of chunk ci: slot (gc0 + ci, h), slice sl, [4 quads][256 threads] float4
   auto ckp = [&](int ci) {
     return reinterpret_cast<float4*>(ck_ws + ((size_t)(gc0 + ci) * hv + h) * BW_CK_FLOATS +
                                      (size_t)sl * BW_EL * BW_THREADS) + tid;
   };
-  auto put = [&](float4* p, int stride, const float (&x)[BW_EL]) {
+  auto put = [&](float4* p, const float (&x)[BW_EL]) {
 #pragma unroll
-    for (int i = 0; i < BW_EL / 4; ++i) p[i * stride] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    for (int i = 0; i < BW_EL / 4; ++i)
+      p[i * BW_THREADS] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   };
-  auto get = [&](const float4* p, int stride, float (&x)[BW_EL]) {
+  auto get = [&](const float4* p, float (&x)[BW_EL]) {
 #pragma unroll
     for (int i = 0; i < BW_EL / 4; ++i) {
-      const float4 f = p[i * stride];
+      const float4 f = p[i * BW_THREADS];
       x[4 * i] = f.x; x[4 * i + 1] = f.y; x[4 * i + 2] = f.z; x[4 * i + 3] = f.w;
     }
   };
-  // the chunk's inputs to shared memory (k, v, alpha, beta; with q and dy for the reverse pass)
-  auto load_chunk = [&](int t0, int L, bool rev) {
-    for (int i = tid; i < L * (D / 4); i += BW_THREADS) {
-      const int tt = i / (D / 4), c4 = i % (D / 4);
-      const size_t o = ((size_t)(t0 + tt) * hq + j) * D;
-      reinterpret_cast<float4*>(sK)[i] = __ldg(reinterpret_cast<const float4*>(kh + o) + c4);
-      if (rev) reinterpret_cast<float4*>(sQ)[i] = __ldg(reinterpret_cast<const float4*>(qh + o) + c4);
-    }
-    for (int i = tid; i < L * (BW_NR / 4); i += BW_THREADS) {
-      const int tt = i / (BW_NR / 4), c4 = i % (BW_NR / 4);
-      const size_t o = ((size_t)(t0 + tt) * hv + h) * D + i0;
-      reinterpret_cast<float4*>(sV)[i] = __ldg(reinterpret_cast<const float4*>(v + o) + c4);
-      if (rev) reinterpret_cast<float4*>(sDY)[i] = __ldg(reinterpret_cast<const float4*>(dy + o) + c4);
-    }
+  // copies (cp.async, not committed) of the L tokens from t0 into an input block
+  auto load_inputs = [&](float* blk, int t0, int L) {
+    for (int i = tid; i < L * (D / 4); i += BW_THREADS)
+      bw_cp16(blk + BWI_K + 4 * i, kh + ((size_t)(t0 + i / (D / 4)) * hq + j) * D + 4 * (i % (D / 4)));
+    for (int i = tid; i < L * (BW_NR / 4); i += BW_THREADS)
+      bw_cp16(blk + BWI_V + 4 * i, v + ((size_t)(t0 + i / (BW_NR / 4)) * hv + h) * D + i0 + 4 * (i % (BW_NR / 4)));
     for (int i = tid; i < L; i += BW_THREADS) {
-      sA[i] = __expf(g[(size_t)(t0 + i) * hv + h]);
-      sB[i] = beta[(size_t)(t0 + i) * hv + h];
+      bw_cp4(blk + BWI_G + i, g + (size_t)(t0 + i) * hv + h);
+      bw_cp4(blk + BWI_B + i, beta + (size_t)(t0 + i) * hv + h);
     }
   };
-  auto fwd = [&](float (&S)[BW_EL], int tt) {
-    bw_forward_token(S, sA[tt], sB[tt], *reinterpret_cast<const float4*>(sK + tt * D + c0), sV + tt * BW_NR + r0);
+  // copies of the q and dy rows of nt tokens from t0 into buffer b
+  auto load_qdy = [&](int b, int t0, int nt) {
+    for (int i = tid; i < nt * (D / 4); i += BW_THREADS)
+      bw_cp16(sQ + b * BW_SUB * D + 4 * i, qh + ((size_t)(t0 + i / (D / 4)) * hq + j) * D + 4 * (i % (D / 4)));
+    for (int i = tid; i < nt * (BW_NR / 4); i += BW_THREADS)
+      bw_cp16(sDY + b * BW_SUB * BW_NR + 4 * i,
+              dy + ((size_t)(t0 + i / (BW_NR / 4)) * hv + h) * D + i0 + 4 * (i % (BW_NR / 4)));
+  };
+  auto fwd = [&](float (&S)[BW_EL], const float* blk, int tt) {
+    float sk[BW_ROWS];
+    bw_forward_token(S, sk, __expf(blk[BWI_G + tt]), blk[BWI_B + tt],
+                     *reinterpret_cast<const float4*>(blk + BWI_K + tt * D + c0), blk + BWI_V + tt * BW_NR + r0, true);
   };
 
   // ---- 1. forward, a checkpoint at every chunk start ---------------------------------------
@@ -141,13 +169,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   for (int r = 0; r < BW_ROWS; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) S[4 * r + c] = init_state ? init_state[sbase + elem(r, c)] : 0.0f;
+  if (nchunks > 0) load_inputs(in0, ts, min(CH, te - ts));
+  bw_commit();
   for (int ci = 0; ci < nchunks; ++ci) {
     const int t0 = ts + ci * CH, L = min(CH, te - t0);
-    put(ckp(ci), BW_THREADS, S);
-    __syncthreads();  // the previous chunk's inputs are no longer read
-    load_chunk(t0, L, false);
+    float* blk = (ci & 1) ? in1 : in0;
+    put(ckp(ci), S);
+    if (ci + 1 < nchunks) load_inputs((ci & 1) ? in0 : in1, t0 + CH, min(CH, te - t0 - CH));
+    bw_commit();
+    bw_wait<1>();  // this chunk's copies landed (the next chunk's may be in flight)
     __syncthreads();
-    for (int tt = 0; tt < L; ++tt) fwd(S, tt);
+    for (int tt = 0; tt < L; ++tt) fwd(S, blk, tt);
+    __syncthreads();  // the next iteration copies into this block
   }
 
   // ---- 2. reverse, chunk by chunk from the last ---------------------------------------------
@@ -156,57 +189,95 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   for (int r = 0; r < BW_ROWS; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) Dm[4 * r + c] = dS_final ? dS_final[sbase + elem(r, c)] : 0.0f;
-  int par = 0;
-  const size_t T = (size_t)d.total_tokens;
+  // the slice's partials of token tp in buffer rb: summed over the warps, in warp order
+  auto reduce = [&](int rb, int tp) {
+    for (int x = tid; x < BW_RED; x += BW_THREADS) {
+      float s2 = 0.0f;
+#pragma unroll
+      for (int ww = 0; ww < BW_WARPS; ++ww) s2 += red[(rb * BW_WARPS + ww) * BW_RED_LD + x];
+      part[(((size_t)sl * T + tp) * hv + h) * BW_RED + x] = s2;
+    }
+  };
+  int kred = 0;      // reverse tokens done: the partial buffer of the next is kred % 3
+  int pend = -1;     // the token whose partials wait in buffer (kred + 2) % 3
+  int nsub = 0;      // sub-chunks done: the q / dy buffer of the next is nsub & 1
+  if (nchunks > 0) {
+    const int t0 = ts + (nchunks - 1) * CH, L = te - t0, tb = (L - 1) / BW_SUB * BW_SUB;
+    load_qdy(0, t0 + tb, L - tb);
+  }
+  bw_commit();
   for (int ci = nchunks - 1; ci >= 0; --ci) {
     const int t0 = ts + ci * CH, L = min(CH, te - t0);
-    __syncthreads();  // the later chunk's inputs and partials are no longer read
-    load_chunk(t0, L, true);
-    get(ckp(ci), BW_THREADS, S);
+    __syncthreads();  // the later chunk's inputs and sub-checkpoints are no longer read
+    load_inputs(in0, t0, L);
+    bw_commit();
+    get(ckp(ci), S);
+    bw_wait<0>();
     __syncthreads();
     // the state before every 8th token, to this thread's own sub-checkpoint slots
     for (int tt = 0; tt < L; ++tt) {
-      if (tt % BW_SUB == 0) put(sSub + (tt / BW_SUB) * BW_EL / 4 * BW_THREADS + tid, BW_THREADS, S);
-      fwd(S, tt);
+      if (tt % BW_SUB == 0) put(sSub + (tt / BW_SUB) * (BW_EL / 4) * BW_THREADS + tid, S);
+      fwd(S, in0, tt);
     }
     for (int sc = (L + BW_SUB - 1) / BW_SUB - 1; sc >= 0; --sc) {
       const int tb = sc * BW_SUB, nt = min(BW_SUB, L - tb);  // block-uniform
-      float St[BW_SUB][BW_EL];  // St[i]: the state before token tb + i
-      get(sSub + sc * BW_EL / 4 * BW_THREADS + tid, BW_THREADS, St[0]);
+      const int b = nsub & 1;
+      // the next sub-chunk's q and dy rows into the other buffer (read by the previous one,
+      // whose last token's barrier every thread has passed)
+      const bool more = sc > 0 || ci > 0;
+      if (sc > 0) load_qdy(b ^ 1, t0 + tb - BW_SUB, BW_SUB);
+      else if (ci > 0) load_qdy(b ^ 1, t0 - BW_SUB, BW_SUB);
+      bw_commit();
+      // St[i]: the state before token tb + i; S_{t-1} k_t of every token to shared memory
+      float St[BW_SUB][BW_EL];
+      get(sSub + sc * (BW_EL / 4) * BW_THREADS + tid, St[0]);
 #pragma unroll
-      for (int i = 1; i < BW_SUB; ++i) {
+      for (int i = 0; i < BW_SUB; ++i) {
         if (i < nt) {
+          const int tt = tb + i;
+          float sk[BW_ROWS];
+          if (i + 1 < BW_SUB) {
 #pragma unroll
-          for (int x = 0; x < BW_EL; ++x) St[i][x] = St[i - 1][x];
-          fwd(St[i], tb + i - 1);
+            for (int x = 0; x < BW_EL; ++x) St[i + 1][x] = St[i][x];
+            bw_forward_token(St[i + 1], sk, __expf(in0[BWI_G + tt]), in0[BWI_B + tt],
+                             *reinterpret_cast<const float4*>(in0 + BWI_K + tt * D + c0),
+                             in0 + BWI_V + tt * BW_NR + r0, i + 1 < nt);
+          } else {
+            float Sx[BW_EL];
+#pragma unroll
+            for (int x = 0; x < BW_EL; ++x) Sx[x] = St[i][x];
+            bw_forward_token(Sx, sk, 0.0f, 0.0f, *reinterpret_cast<const float4*>(in0 + BWI_K + tt * D + c0),
+                             in0 + BWI_V + tt * BW_NR + r0, false);
+          }
+          if (lane == 0)
+            *reinterpret_cast<float4*>(sSK + (i * BW_WARPS + warp) * BW_ROWS) = make_float4(sk[0], sk[1], sk[2], sk[3]);
         }
       }
+      if (more) bw_wait<1>();  // this sub-chunk's q / dy copies landed
+      else bw_wait<0>();
+      __syncthreads();
+      const float* qb = sQ + b * BW_SUB * D;
+      const float* yb = sDY + b * BW_SUB * BW_NR;
 #pragma unroll
       for (int i = BW_SUB - 1; i >= 0; --i) {
         if (i >= nt) continue;
         const int tt = tb + i, t = t0 + tt;
         const float* Sprev = St[i];
-        const float a = sA[tt], bt = sB[tt];
-        const float4 k4 = *reinterpret_cast<const float4*>(sK + tt * D + c0);
-        const float4 q4 = *reinterpret_cast<const float4*>(sQ + tt * D + c0);
-        const float* vrow = sV + tt * BW_NR + r0;
-        const float* yrow = sDY + tt * BW_NR + r0;
+        const float a = __expf(in0[BWI_G + tt]), bt = in0[BWI_B + tt];
+        const float4 k4 = *reinterpret_cast<const float4*>(in0 + BWI_K + tt * D + c0);
+        const float4 q4 = *reinterpret_cast<const float4*>(qb + i * D + c0);
+        const float4 s4 = *reinterpret_cast<const float4*>(sSK + (i * BW_WARPS + warp) * BW_ROWS);
+        const float* vrow = in0 + BWI_V + tt * BW_NR + r0;
+        const float* yrow = yb + i * BW_NR + r0;
         const float kc[4] = {k4.x, k4.y, k4.z, k4.w}, qc[4] = {q4.x, q4.y, q4.z, q4.w};
-        // e_t = v_t - S'_t k_t with S'_t = alpha S_{t-1}
-        float e[BW_ROWS];
+        const float sk[BW_ROWS] = {s4.x, s4.y, s4.z, s4.w};
+        // e_t = v_t - alpha (S_{t-1} k_t);  dq partial = S_t^T dy (S_t = alpha S_{t-1} + beta e k^T)
+        // D' = D + dy q^T;  w = D' k;  P = <D', S_{t-1}>  (one reduction group)
+        float e[BW_ROWS], dqp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, w[BW_ROWS + 1];
+        w[BW_ROWS] = 0.0f;
 #pragma unroll
         for (int r = 0; r < BW_ROWS; ++r) {
-          float s2 = 0.0f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) s2 = fmaf(Sprev[4 * r + c], kc[c], s2);
-          e[r] = s2;
-        }
-#pragma unroll
-        for (int r = 0; r < BW_ROWS; ++r) e[r] = vrow[r] - a * warp_sum(e[r]);
-        // dq partial: S_t^T dy (S_t = alpha S_{t-1} + beta e k^T);  D += dy q^T;  w = D k
-        float dqp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, w[BW_ROWS];
-#pragma unroll
-        for (int r = 0; r < BW_ROWS; ++r) {
+          e[r] = vrow[r] - a * sk[r];
           const float gy = yrow[r];
           float s2 = 0.0f;
 #pragma unroll
@@ -214,29 +285,28 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             dqp[c] = fmaf(gy, fmaf(a, Sprev[4 * r + c], bt * e[r] * kc[c]), dqp[c]);
             Dm[4 * r + c] = fmaf(gy, qc[c], Dm[4 * r + c]);
             s2 = fmaf(Dm[4 * r + c], kc[c], s2);
+            w[BW_ROWS] = fmaf(Dm[4 * r + c], Sprev[4 * r + c], w[BW_ROWS]);
           }
           w[r] = s2;
         }
 #pragma unroll
-        for (int r = 0; r < BW_ROWS; ++r) w[r] = warp_sum(w[r]);
-        // de = beta w (= dv);  dbeta = e . w;  dk partial = beta D^T e - S'^T de;
-        // dS' = D - de k^T;  dalpha partial = <dS', S_{t-1}>;  D <- alpha dS'
-        float dkp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, dbp = 0.0f, dap = 0.0f;
+        for (int r = 0; r <= BW_ROWS; ++r) w[r] = warp_sum(w[r]);
+        // de = beta w (= dv);  dbeta = e . w;  dk partial = beta D'^T e - alpha S_{t-1}^T de;
+        // dS' = D' - de k^T;  dalpha = <dS', S_{t-1}> = P - de . (S_{t-1} k);  D <- alpha dS'
+        float dkp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, dbp = 0.0f, dap = w[BW_ROWS];
 #pragma unroll
         for (int r = 0; r < BW_ROWS; ++r) {
           const float de = bt * w[r];
           dbp = fmaf(e[r], w[r], dbp);
+          dap = fmaf(-de, sk[r], dap);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             dkp[c] = fmaf(bt * e[r], Dm[4 * r + c], fmaf(-de * a, Sprev[4 * r + c], dkp[c]));
-            const float dsp = fmaf(-de, kc[c], Dm[4 * r + c]);
-            dap = fmaf(dsp, Sprev[4 * r + c], dap);
-            Dm[4 * r + c] = a * dsp;
+            Dm[4 * r + c] = a * fmaf(-de, kc[c], Dm[4 * r + c]);
           }
           if (lane == r) dv[((size_t)t * hv + h) * D + i0 + r0 + r] = de;
         }
-        dap = warp_sum(dap);
-        float* rw = red + (par * BW_WARPS + warp) * BW_RED_LD;
+        float* rw = red + ((kred % BW_NRED) * BW_WARPS + warp) * BW_RED_LD;
         *reinterpret_cast<float4*>(rw + c0) = make_float4(dqp[0], dqp[1], dqp[2], dqp[3]);
         *reinterpret_cast<float4*>(rw + D + c0) = make_float4(dkp[0], dkp[1], dkp[2], dkp[3]);
         if (lane == 0) {
@@ -244,16 +314,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
           rw[2 * D + 1] = dap;
         }
         __syncthreads();
-        for (int x = tid; x < BW_RED; x += BW_THREADS) {  // the slice's sums over its warps, in warp order
-          float s2 = 0.0f;
-#pragma unroll
-          for (int ww = 0; ww < BW_WARPS; ++ww) s2 += red[(par * BW_WARPS + ww) * BW_RED_LD + x];
-          part[(((size_t)sl * T + t) * hv + h) * BW_RED + x] = s2;
-        }
-        par ^= 1;  // the next token writes the other buffer; this one is read before the next barrier
+        if (pend >= 0) reduce((kred + BW_NRED - 1) % BW_NRED, pend);
+        pend = t;
+        ++kred;
       }
+      ++nsub;
     }
   }
+  __syncthreads();
+  if (pend >= 0) reduce((kred + BW_NRED - 1) % BW_NRED, pend);
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r)
 #pragma unroll
