@@ -505,7 +505,13 @@ def gpu_arm(args):
         torch.cuda.synchronize()
         barrier()
         mms = max_over_ranks(e0.elapsed_time(e1), dev) / dsteps
-        multi = {"tokens_per_sequence": K4, "ms_per_call": mms, "tokens_per_s": 256 * K4 / (mms / 1e3)}
+        m_state = 256 * 32 * 128 * 128 * 4 * 2  # each state row read and written once per call
+        m_other = 256 * (K4 * (2 * 16 * 128 * 2 + 2 * 32 * 128 * 2 + 2 * 32 * 4 + 32 * 128 * 2) + 2 * 3 * 8192 * 2)
+        multi = {"tokens_per_sequence": K4, "ms_per_call": mms, "tokens_per_s": 256 * K4 / (mms / 1e3),
+                 "state_GBps": m_state / (mms / 1e3) / 1e9,
+                 "total_GBps": (m_state + m_other) / (mms / 1e3) / 1e9,
+                 "frac_state": m_state / (mms / 1e3) / 1e9 / hbm,
+                 "frac_total": (m_state + m_other) / (mms / 1e3) / 1e9 / hbm}
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         multi = f"failed: {exc}"
     clk = clocks.stop()

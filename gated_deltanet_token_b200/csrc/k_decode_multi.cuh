@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
     __syncwarp();  // every lane has read the buffer before group gi + 2 refills it
     if (gi + 2 < ngroups) load_group(gi + 2);
     else asm volatile("cp.async.commit_group;" ::: "memory");
+#pragma unroll 2  // two tokens at a time: the second token's k, q loads overlap the first's chain
     for (int t = 0; t < K; ++t) {
       float4 kr[DECM_CPL / 4], qr[DECM_CPL / 4];
 #pragma unroll
