@@ -617,7 +617,9 @@ static int proj_launch(const void* A, long long M, const void* B, int N, int K, 
   CUtensorMap ta, tb;
   if (make_kmajor_map(&ta, A, M, K, PJ_BM) != GDN_OK || make_kmajor_map(&tb, B, N, K, PJ_BN) != GDN_OK)
     return GDN_ERR_CUDA;
-  const dim3 grid((unsigned)((N + PJ_BN - 1) / PJ_BN), (unsigned)((M + PJ_BM - 1) / PJ_BM));
+  const long long ntiles = ((M + PJ_BM - 1) / PJ_BM) * (long long)((N + PJ_BN - 1) / PJ_BN);
+  if (ntiles > (1LL << 30)) return GDN_ERR_SHAPE;
+  const unsigned grid = (unsigned)std::min<long long>(ntiles, g_num_sms);  // persistent: one CTA per SM
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   ProfScope p("proj_gemm", s);
   k_proj_gemm<<<grid, 192, PJ_SMEM, s>>>((int)M, N, K, ta, tb, po);
