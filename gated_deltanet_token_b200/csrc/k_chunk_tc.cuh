@@ -794,8 +794,6 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
                    const float* init_state, float* __restrict__ y_raw,
                    float* final_state,
                    const uint16_t* __restrict__ z, const float* __restrict__ norm_w, void* __restrict__ y) {
-  tc::grid_dep_wait();  // phase A's tiles and gates are complete
-  tc::grid_dep_launch_dependents();
   constexpr int NV = TC_NV, NH = NV / 2;
   constexpr bool FUSED = YM != PB_Y_RAW;
   const int n = blockIdx.x, h = blockIdx.y, sl = blockIdx.z, i0 = sl * NV;
@@ -926,6 +924,12 @@ __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
   const uint32_t T_A = tbase, T_CD = tbase + 2 * NV, T_E = tbase + 4 * NV;
   const uint32_t t_a = T_A + lane_off + cb, t_cd = T_CD + lane_off + cb, t_e = T_E + lane_off + cb;
   auto par_cols = [](int c) { return (uint32_t)(c & 1) * 256u; };
+  // The setup above reads only the call's inputs (the initial state may be the previous call's
+  // final state: that call completed before this call's phase A started, and so before this
+  // grid was launched) and overlaps phase A's last CTAs; phase A's tiles and gates are read
+  // only from here on.
+  tc::grid_dep_wait();
+  tc::grid_dep_launch_dependents();
   int last_load = -1;  // (producer lane) the last chunk whose stage copies were issued
   if (producer && lane == 0 && nchunks > 0) {
     issue_load(0, 0);
