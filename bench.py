@@ -182,6 +182,7 @@ KERNEL_SOURCES = {
     "chunk_scan_tc_norm": ("k_chunk_tc.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "decode_multi": ("k_decode_multi.cuh", "gdn_common.cuh"),
     "proj_gemm": ("k_proj.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
+    "proj_gemm_out": ("k_proj.cuh", "tc_ptx.cuh", "gdn_common.cuh"),
     "recurrence_bwd": ("k_bwd.cuh", "gdn_common.cuh"),
     "decode": ("k_decode.cuh", "gdn_common.cuh"),
     "chunk_phaseB_simt": ("k_chunk_simt.cuh", "gdn_common.cuh"),
@@ -511,7 +512,8 @@ def gpu_arm(args):
                  "state_GBps": m_state / (mms / 1e3) / 1e9,
                  "total_GBps": (m_state + m_other) / (mms / 1e3) / 1e9,
                  "frac_state": m_state / (mms / 1e3) / 1e9 / hbm,
-                 "frac_total": (m_state + m_other) / (mms / 1e3) / 1e9 / hbm}
+                 "frac_total": (m_state + m_other) / (mms / 1e3) / 1e9 / hbm,
+                 "traffic": ncu_traffic("decode_multi")}
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         multi = f"failed: {exc}"
     clk = clocks.stop()
@@ -558,7 +560,8 @@ def gpu_arm(args):
                 "out_proj_us": ms_out * 1e3, "out_proj_tflops": fl_out / (ms_out / 1e3) / 1e12,
                 "peak_tflops": pk, "peak_source": f"{peak_src} bf16_tflops",
                 "in_proj_frac": fl_in / (ms_in / 1e3) / 1e12 / pk, "out_proj_frac": fl_out / (ms_out / 1e3) / 1e12 / pk,
-                "shape": "x [4096, 2048] -> 12352 features; y [4096, 4096] -> 2048"}
+                "shape": "x [4096, 2048] -> 12352 features; y [4096, 4096] -> 2048",
+                "traffic_in": ncu_traffic("proj_gemm"), "traffic_out": ncu_traffic("proj_gemm_out")}
         del xp, wi, wo, pouts, yo
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         proj = f"failed: {exc}"
@@ -590,7 +593,8 @@ def gpu_arm(args):
         barrier()
         bms = max_over_ranks(e0.elapsed_time(e1), dev) / 5
         bwd = {"ms_per_call": bms, "tokens_per_s": T / (bms / 1e3), "workspace_MB": bws.numel() / 1e6,
-               "shape": "T=4096, 16 QK / 32 value heads, fp32, one sequence"}
+               "shape": "T=4096, 16 QK / 32 value heads, fp32, one sequence",
+               "traffic": ncu_traffic("recurrence_bwd")}
         del bt, bws
     except RuntimeError as exc:  # an auxiliary figure: report, do not lose the bench line
         bwd = f"failed: {exc}"
