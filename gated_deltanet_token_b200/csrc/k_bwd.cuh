@@ -72,27 +72,31 @@ __device__ __forceinline__ void bw_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// One forward token on the thread's elements (rows r of BW_ROWS, columns c of 4):
-// sk_r = (S k)_r, e_r = beta (v_r - alpha sk_r), S <- alpha S + e k^T.  k4: the thread's 4 key
-// components; vrow: the warp's BW_ROWS values.  Every pass runs this same arithmetic.
-__device__ __forceinline__ void bw_forward_token(float (&S)[BW_EL], float (&sk)[BW_ROWS], float a, float bt,
+// A thread's state elements as paired floats: row r, columns (0, 1) at [2 r] and (2, 3) at
+// [2 r + 1], so that the row updates run as paired fp32 FMAs.
+constexpr int BW_EL2 = BW_EL / 2;
+__device__ __forceinline__ float2 bw_f2(float x) { return make_float2(x, x); }
+
+// One forward token on the thread's elements: sk_r = (S k)_r, e_r = beta (v_r - alpha sk_r),
+// S <- alpha S + e k^T.  k4: the thread's 4 key components; vrow: the warp's BW_ROWS values.
+// Every pass runs this same arithmetic.
+__device__ __forceinline__ void bw_forward_token(float2 (&S)[BW_EL2], float (&sk)[BW_ROWS], float a, float bt,
                                                  const float4 k4, const float* vrow, bool update) {
-  const float kc[4] = {k4.x, k4.y, k4.z, k4.w};
+  const float2 k01 = make_float2(k4.x, k4.y), k23 = make_float2(k4.z, k4.w);
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r) {
-    float s = 0.0f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) s = fmaf(S[4 * r + c], kc[c], s);
-    sk[r] = s;
+    const float2 p = __ffma2_rn(S[2 * r + 1], k23, __fmul2_rn(S[2 * r], k01));
+    sk[r] = p.x + p.y;
   }
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r) sk[r] = warp_sum(sk[r]);
   if (!update) return;
+  const float2 a2 = bw_f2(a);
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r) {
-    const float e = bt * (vrow[r] - a * sk[r]);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) S[4 * r + c] = fmaf(e, kc[c], a * S[4 * r + c]);
+    const float2 e2 = bw_f2(bt * (vrow[r] - a * sk[r]));
+    S[2 * r] = __ffma2_rn(e2, k01, __fmul2_rn(a2, S[2 * r]));
+    S[2 * r + 1] = __ffma2_rn(e2, k23, __fmul2_rn(a2, S[2 * r + 1]));
   }
 }
 
@@ -126,16 +130,27 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     return reinterpret_cast<float4*>(ck_ws + ((size_t)(gc0 + ci) * hv + h) * BW_CK_FLOATS +
                                      (size_t)sl * BW_EL * BW_THREADS) + tid;
   };
-  auto put = [&](float4* p, const float (&x)[BW_EL]) {
+  // row r of the thread's elements is float4 number r of its slots
+  auto put = [&](float4* p, const float2 (&x)[BW_EL2]) {
 #pragma unroll
-    for (int i = 0; i < BW_EL / 4; ++i)
-      p[i * BW_THREADS] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    for (int r = 0; r < BW_ROWS; ++r)
+      p[r * BW_THREADS] = make_float4(x[2 * r].x, x[2 * r].y, x[2 * r + 1].x, x[2 * r + 1].y);
   };
-  auto get = [&](const float4* p, float (&x)[BW_EL]) {
+  auto get = [&](const float4* p, float2 (&x)[BW_EL2]) {
 #pragma unroll
-    for (int i = 0; i < BW_EL / 4; ++i) {
-      const float4 f = p[i * BW_THREADS];
-      x[4 * i] = f.x; x[4 * i + 1] = f.y; x[4 * i + 2] = f.z; x[4 * i + 3] = f.w;
+    for (int r = 0; r < BW_ROWS; ++r) {
+      const float4 f = p[r * BW_THREADS];
+      x[2 * r] = make_float2(f.x, f.y);
+      x[2 * r + 1] = make_float2(f.z, f.w);
+    }
+  };
+  // the thread's elements of a [N][h_v][d_v][d_k] state (or zeros for a null pointer)
+  auto load_state = [&](const float* src, float2 (&x)[BW_EL2]) {
+#pragma unroll
+    for (int r = 0; r < BW_ROWS; ++r) {
+      const float4 f = src ? *reinterpret_cast<const float4*>(src + sbase + elem(r, 0)) : make_float4(0, 0, 0, 0);
+      x[2 * r] = make_float2(f.x, f.y);
+      x[2 * r + 1] = make_float2(f.z, f.w);
     }
   };
   // copies (cp.async, not committed) of the L tokens from t0 into an input block
@@ -157,18 +172,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       bw_cp16(sDY + b * BW_SUB * BW_NR + 4 * i,
               dy + ((size_t)(t0 + i / (BW_NR / 4)) * hv + h) * D + i0 + 4 * (i % (BW_NR / 4)));
   };
-  auto fwd = [&](float (&S)[BW_EL], const float* blk, int tt) {
+  auto fwd = [&](float2 (&S)[BW_EL2], const float* blk, int tt) {
     float sk[BW_ROWS];
     bw_forward_token(S, sk, __expf(blk[BWI_G + tt]), blk[BWI_B + tt],
                      *reinterpret_cast<const float4*>(blk + BWI_K + tt * D + c0), blk + BWI_V + tt * BW_NR + r0, true);
   };
 
   // ---- 1. forward, a checkpoint at every chunk start ---------------------------------------
-  float S[BW_EL];
-#pragma unroll
-  for (int r = 0; r < BW_ROWS; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) S[4 * r + c] = init_state ? init_state[sbase + elem(r, c)] : 0.0f;
+  float2 S[BW_EL2];
+  load_state(init_state, S);
   if (nchunks > 0) load_inputs(in0, ts, min(CH, te - ts));
   bw_commit();
   for (int ci = 0; ci < nchunks; ++ci) {
@@ -184,11 +196,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   }
 
   // ---- 2. reverse, chunk by chunk from the last ---------------------------------------------
-  float Dm[BW_EL];
-#pragma unroll
-  for (int r = 0; r < BW_ROWS; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) Dm[4 * r + c] = dS_final ? dS_final[sbase + elem(r, c)] : 0.0f;
+  float2 Dm[BW_EL2];
+  load_state(dS_final, Dm);
   // the slice's partials of token tp in buffer rb: summed over the warps, in warp order
   auto reduce = [&](int rb, int tp) {
     for (int x = tid; x < BW_RED; x += BW_THREADS) {
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       else if (ci > 0) load_qdy(b ^ 1, t0 - BW_SUB, BW_SUB);
       bw_commit();
       // St[i]: the state before token tb + i; S_{t-1} k_t of every token to shared memory
-      float St[BW_SUB][BW_EL];
+      float2 St[BW_SUB][BW_EL2];
       get(sSub + sc * (BW_EL / 4) * BW_THREADS + tid, St[0]);
 #pragma unroll
       for (int i = 0; i < BW_SUB; ++i) {
@@ -238,14 +247,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
           float sk[BW_ROWS];
           if (i + 1 < BW_SUB) {
 #pragma unroll
-            for (int x = 0; x < BW_EL; ++x) St[i + 1][x] = St[i][x];
+            for (int x = 0; x < BW_EL2; ++x) St[i + 1][x] = St[i][x];
             bw_forward_token(St[i + 1], sk, __expf(in0[BWI_G + tt]), in0[BWI_B + tt],
                              *reinterpret_cast<const float4*>(in0 + BWI_K + tt * D + c0),
                              in0 + BWI_V + tt * BW_NR + r0, i + 1 < nt);
           } else {
-            float Sx[BW_EL];
+            float2 Sx[BW_EL2];
 #pragma unroll
-            for (int x = 0; x < BW_EL; ++x) Sx[x] = St[i][x];
+            for (int x = 0; x < BW_EL2; ++x) Sx[x] = St[i][x];
             bw_forward_token(Sx, sk, 0.0f, 0.0f, *reinterpret_cast<const float4*>(in0 + BWI_K + tt * D + c0),
                              in0 + BWI_V + tt * BW_NR + r0, false);
           }
@@ -262,50 +271,53 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       for (int i = BW_SUB - 1; i >= 0; --i) {
         if (i >= nt) continue;
         const int tt = tb + i, t = t0 + tt;
-        const float* Sprev = St[i];
+        const float2* Sprev = St[i];
         const float a = __expf(in0[BWI_G + tt]), bt = in0[BWI_B + tt];
         const float4 k4 = *reinterpret_cast<const float4*>(in0 + BWI_K + tt * D + c0);
         const float4 q4 = *reinterpret_cast<const float4*>(qb + i * D + c0);
         const float4 s4 = *reinterpret_cast<const float4*>(sSK + (i * BW_WARPS + warp) * BW_ROWS);
         const float* vrow = in0 + BWI_V + tt * BW_NR + r0;
         const float* yrow = yb + i * BW_NR + r0;
-        const float kc[4] = {k4.x, k4.y, k4.z, k4.w}, qc[4] = {q4.x, q4.y, q4.z, q4.w};
+        const float2 k01 = make_float2(k4.x, k4.y), k23 = make_float2(k4.z, k4.w);
+        const float2 q01 = make_float2(q4.x, q4.y), q23 = make_float2(q4.z, q4.w), a2 = bw_f2(a);
         const float sk[BW_ROWS] = {s4.x, s4.y, s4.z, s4.w};
         // e_t = v_t - alpha (S_{t-1} k_t);  dq partial = S_t^T dy (S_t = alpha S_{t-1} + beta e k^T)
         // D' = D + dy q^T;  w = D' k;  P = <D', S_{t-1}>  (one reduction group)
-        float e[BW_ROWS], dqp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, w[BW_ROWS + 1];
-        w[BW_ROWS] = 0.0f;
+        float e[BW_ROWS], w[BW_ROWS + 1];
+        float2 dq01 = make_float2(0.0f, 0.0f), dq23 = dq01, pp = dq01;
 #pragma unroll
         for (int r = 0; r < BW_ROWS; ++r) {
           e[r] = vrow[r] - a * sk[r];
-          const float gy = yrow[r];
-          float s2 = 0.0f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            dqp[c] = fmaf(gy, fmaf(a, Sprev[4 * r + c], bt * e[r] * kc[c]), dqp[c]);
-            Dm[4 * r + c] = fmaf(gy, qc[c], Dm[4 * r + c]);
-            s2 = fmaf(Dm[4 * r + c], kc[c], s2);
-            w[BW_ROWS] = fmaf(Dm[4 * r + c], Sprev[4 * r + c], w[BW_ROWS]);
-          }
-          w[r] = s2;
+          const float2 gy2 = bw_f2(yrow[r]), be2 = bw_f2(bt * e[r]);
+          dq01 = __ffma2_rn(gy2, __ffma2_rn(a2, Sprev[2 * r], __fmul2_rn(be2, k01)), dq01);
+          dq23 = __ffma2_rn(gy2, __ffma2_rn(a2, Sprev[2 * r + 1], __fmul2_rn(be2, k23)), dq23);
+          Dm[2 * r] = __ffma2_rn(gy2, q01, Dm[2 * r]);
+          Dm[2 * r + 1] = __ffma2_rn(gy2, q23, Dm[2 * r + 1]);
+          const float2 wv = __ffma2_rn(Dm[2 * r + 1], k23, __fmul2_rn(Dm[2 * r], k01));
+          w[r] = wv.x + wv.y;
+          pp = __ffma2_rn(Dm[2 * r], Sprev[2 * r], pp);
+          pp = __ffma2_rn(Dm[2 * r + 1], Sprev[2 * r + 1], pp);
         }
+        w[BW_ROWS] = pp.x + pp.y;
 #pragma unroll
         for (int r = 0; r <= BW_ROWS; ++r) w[r] = warp_sum(w[r]);
         // de = beta w (= dv);  dbeta = e . w;  dk partial = beta D'^T e - alpha S_{t-1}^T de;
         // dS' = D' - de k^T;  dalpha = <dS', S_{t-1}> = P - de . (S_{t-1} k);  D <- alpha dS'
-        float dkp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, dbp = 0.0f, dap = w[BW_ROWS];
+        float2 dk01 = make_float2(0.0f, 0.0f), dk23 = dk01;
+        float dbp = 0.0f, dap = w[BW_ROWS];
 #pragma unroll
         for (int r = 0; r < BW_ROWS; ++r) {
           const float de = bt * w[r];
           dbp = fmaf(e[r], w[r], dbp);
           dap = fmaf(-de, sk[r], dap);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            dkp[c] = fmaf(bt * e[r], Dm[4 * r + c], fmaf(-de * a, Sprev[4 * r + c], dkp[c]));
-            Dm[4 * r + c] = a * fmaf(-de, kc[c], Dm[4 * r + c]);
-          }
+          const float2 be2 = bw_f2(bt * e[r]), mdea = bw_f2(-de * a), mde = bw_f2(-de);
+          dk01 = __ffma2_rn(be2, Dm[2 * r], __ffma2_rn(mdea, Sprev[2 * r], dk01));
+          dk23 = __ffma2_rn(be2, Dm[2 * r + 1], __ffma2_rn(mdea, Sprev[2 * r + 1], dk23));
+          Dm[2 * r] = __fmul2_rn(a2, __ffma2_rn(mde, k01, Dm[2 * r]));
+          Dm[2 * r + 1] = __fmul2_rn(a2, __ffma2_rn(mde, k23, Dm[2 * r + 1]));
           if (lane == r) dv[((size_t)t * hv + h) * D + i0 + r0 + r] = de;
         }
+        const float dqp[4] = {dq01.x, dq01.y, dq23.x, dq23.y}, dkp[4] = {dk01.x, dk01.y, dk23.x, dk23.y};
         float* rw = red + ((kred % BW_NRED) * BW_WARPS + warp) * BW_RED_LD;
         *reinterpret_cast<float4*>(rw + c0) = make_float4(dqp[0], dqp[1], dqp[2], dqp[3]);
         *reinterpret_cast<float4*>(rw + D + c0) = make_float4(dkp[0], dkp[1], dkp[2], dkp[3]);
@@ -325,8 +337,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   if (pend >= 0) reduce((kred + BW_NRED - 1) % BW_NRED, pend);
 #pragma unroll
   for (int r = 0; r < BW_ROWS; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) dS_init[sbase + elem(r, c)] = Dm[4 * r + c];
+    *reinterpret_cast<float4*>(dS_init + sbase + elem(r, 0)) =
+        make_float4(Dm[2 * r].x, Dm[2 * r].y, Dm[2 * r + 1].x, Dm[2 * r + 1].y);
 }
 
 // dq, dk of QK head j = the sum over its value heads and their row slices; dbeta, dg of value
