@@ -100,6 +100,33 @@ __device__ __forceinline__ void bw_forward_token(float2 (&S)[BW_EL2], float (&sk
   }
 }
 
+// The same token in the row layout of the two chunk-level forward passes: the thread holds one
+// row of the warp's four, in the 4-column groups cg + 8 m (m = 0..3, S[2 m], S[2 m + 1]), so
+// that a row product reduces over eight lanes (three shuffle levels).  krow: k_t (128 floats);
+// vr: v_t of the thread's row.
+__device__ __forceinline__ void bw_forward_row(float2 (&S)[BW_EL2], float a, float bt, const float* krow, float vr,
+                                               int cg) {
+  float2 k2[BW_EL2];
+#pragma unroll
+  for (int m = 0; m < BW_EL2 / 2; ++m) {
+    const float4 k4 = *reinterpret_cast<const float4*>(krow + 4 * (cg + 8 * m));
+    k2[2 * m] = make_float2(k4.x, k4.y);
+    k2[2 * m + 1] = make_float2(k4.z, k4.w);
+  }
+  float2 p0 = __fmul2_rn(S[0], k2[0]), p1 = __fmul2_rn(S[1], k2[1]);
+#pragma unroll
+  for (int x = 2; x < BW_EL2; x += 2) {
+    p0 = __ffma2_rn(S[x], k2[x], p0);
+    p1 = __ffma2_rn(S[x + 1], k2[x + 1], p1);
+  }
+  float sk = (p0.x + p0.y) + (p1.x + p1.y);
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) sk += __shfl_xor_sync(0xffffffffu, sk, o);
+  const float2 e2 = bw_f2(bt * (vr - a * sk)), a2 = bw_f2(a);
+#pragma unroll
+  for (int x = 0; x < BW_EL2; ++x) S[x] = __ffma2_rn(e2, k2[x], __fmul2_rn(a2, S[x]));
+}
+
 __global__ void __launch_bounds__(BW_THREADS, 1)
     k_bwd(Dims d, const int* __restrict__ cu, const int* __restrict__ seq_chunk0, const float* __restrict__ qh,
           const float* __restrict__ kh, const float* __restrict__ v, const float* __restrict__ g,
@@ -115,6 +142,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   const int gc0 = seq_chunk0 ? seq_chunk0[n] : 0;  // the sequence's first chunk slot
   const int i0 = sl * BW_NR;                       // the slice's first state row
   const int r0 = warp * BW_ROWS, c0 = lane * 4;    // slice rows r0 .. r0 + 3, columns c0 .. c0 + 3
+  const int rr = lane >> 3, cg = lane & 7;         // row layout: slice row r0 + rr, column groups cg + 8 m
   const size_t sbase = ((size_t)n * hv + h) * D * D;
   const size_t T = (size_t)d.total_tokens;
   auto elem = [&](int r, int c) { return (size_t)(i0 + r0 + r) * D + c0 + c; };
@@ -153,6 +181,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       x[2 * r + 1] = make_float2(f.z, f.w);
     }
   };
+  // row layout: the thread's elements of a [N][h_v][d_v][d_k] state (or zeros for a null pointer)
+  auto load_state_row = [&](const float* src, float2 (&x)[BW_EL2]) {
+#pragma unroll
+    for (int m = 0; m < BW_EL2 / 2; ++m) {
+      const float4 f = src ? *reinterpret_cast<const float4*>(src + sbase + (size_t)(i0 + r0 + rr) * D + 4 * (cg + 8 * m))
+                           : make_float4(0, 0, 0, 0);
+      x[2 * m] = make_float2(f.x, f.y);
+      x[2 * m + 1] = make_float2(f.z, f.w);
+    }
+  };
+  // sub-checkpoint sc in shared memory: [32 rows][32 four-column groups] float4, written in the
+  // row layout and read in the column layout, both as 128 contiguous bytes per eight lanes
+  auto sub_unit = [&](int sc, int row, int grp) { return sSub + ((sc * BW_NR + row) * (D / 4) + grp); };
   // copies (cp.async, not committed) of the L tokens from t0 into an input block
   auto load_inputs = [&](float* blk, int t0, int L) {
     for (int i = tid; i < L * (D / 4); i += BW_THREADS)
@@ -172,15 +213,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       bw_cp16(sDY + b * BW_SUB * BW_NR + 4 * i,
               dy + ((size_t)(t0 + i / (BW_NR / 4)) * hv + h) * D + i0 + 4 * (i % (BW_NR / 4)));
   };
-  auto fwd = [&](float2 (&S)[BW_EL2], const float* blk, int tt) {
-    float sk[BW_ROWS];
-    bw_forward_token(S, sk, __expf(blk[BWI_G + tt]), blk[BWI_B + tt],
-                     *reinterpret_cast<const float4*>(blk + BWI_K + tt * D + c0), blk + BWI_V + tt * BW_NR + r0, true);
+  auto fwd_row = [&](float2 (&S)[BW_EL2], const float* blk, int tt) {
+    bw_forward_row(S, __expf(blk[BWI_G + tt]), blk[BWI_B + tt], blk + BWI_K + tt * D, blk[BWI_V + tt * BW_NR + r0 + rr],
+                   cg);
   };
 
-  // ---- 1. forward, a checkpoint at every chunk start ---------------------------------------
+  // ---- 1. forward, a checkpoint at every chunk start (row layout) -------------------------
   float2 S[BW_EL2];
-  load_state(init_state, S);
+  load_state_row(init_state, S);
   if (nchunks > 0) load_inputs(in0, ts, min(CH, te - ts));
   bw_commit();
   for (int ci = 0; ci < nchunks; ++ci) {
@@ -191,7 +231,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     bw_commit();
     bw_wait<1>();  // this chunk's copies landed (the next chunk's may be in flight)
     __syncthreads();
-    for (int tt = 0; tt < L; ++tt) fwd(S, blk, tt);
+    for (int tt = 0; tt < L; ++tt) fwd_row(S, blk, tt);
     __syncthreads();  // the next iteration copies into this block
   }
 
@@ -223,11 +263,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     get(ckp(ci), S);
     bw_wait<0>();
     __syncthreads();
-    // the state before every 8th token, to this thread's own sub-checkpoint slots
+    // the state before every 8th token, to the sub-checkpoints (row layout)
     for (int tt = 0; tt < L; ++tt) {
-      if (tt % BW_SUB == 0) put(sSub + (tt / BW_SUB) * (BW_EL / 4) * BW_THREADS + tid, S);
-      fwd(S, in0, tt);
+      if (tt % BW_SUB == 0) {
+#pragma unroll
+        for (int m = 0; m < BW_EL2 / 2; ++m)
+          *sub_unit(tt / BW_SUB, r0 + rr, cg + 8 * m) = make_float4(S[2 * m].x, S[2 * m].y, S[2 * m + 1].x, S[2 * m + 1].y);
+      }
+      fwd_row(S, in0, tt);
     }
+    __syncthreads();  // the sub-checkpoints are read by other threads (column layout)
     for (int sc = (L + BW_SUB - 1) / BW_SUB - 1; sc >= 0; --sc) {
       const int tb = sc * BW_SUB, nt = min(BW_SUB, L - tb);  // block-uniform
       const int b = nsub & 1;
@@ -239,7 +284,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       bw_commit();
       // St[i]: the state before token tb + i; S_{t-1} k_t of every token to shared memory
       float2 St[BW_SUB][BW_EL2];
-      get(sSub + sc * (BW_EL / 4) * BW_THREADS + tid, St[0]);
+#pragma unroll
+      for (int r = 0; r < BW_ROWS; ++r) {
+        const float4 f = *sub_unit(sc, r0 + r, lane);
+        St[0][2 * r] = make_float2(f.x, f.y);
+        St[0][2 * r + 1] = make_float2(f.z, f.w);
+      }
 #pragma unroll
       for (int i = 0; i < BW_SUB; ++i) {
         if (i < nt) {
