@@ -60,3 +60,45 @@ def test_recurrence_backward_matches_oracle(oracle_mod, lengths, h_qk, h_v):
     torch.cuda.synchronize()
     for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (dg, "dg"), (dbeta, "dbeta"), (dS0, "dS0")):
         _compare(got, ref[name], name)
+
+
+def test_recurrence_backward_null_state_and_final_gradient(oracle_mod):
+    """init_state = NULL and dS_final = NULL read as zeros."""
+    inp = make_bwd_inputs([70, 3], 2, 4, seed=11)
+    inp["init_state"] = np.zeros_like(inp["init_state"])
+    inp["dS_T"] = np.zeros_like(inp["dS_T"])
+    ref = _oracle_grads(oracle_mod, inp, 2, 4)
+    t = {k: to_dev(inp[k]) for k in ("qh", "kh", "v", "g", "beta", "dy")}
+    cu = to_dev(inp["cu_seqlens"].astype(np.int32))
+    dq, dk, dv, dg, dbeta, dS0 = gdn.gdn_recurrence_backward(t["qh"], t["kh"], t["v"], t["g"], t["beta"], None, cu,
+                                                             t["dy"], None)
+    torch.cuda.synchronize()
+    for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (dg, "dg"), (dbeta, "dbeta"), (dS0, "dS0")):
+        _compare(got, ref[name], name)
+
+
+def test_recurrence_backward_full_size_sampled_heads(oracle_mod):
+    """The launch the benchmark times (one sequence, T = 4096, 16 QK / 32 value heads), compared
+    on QK head 15 and its two value heads 30, 31: every gradient of those heads, dq and dk of
+    the QK head (the sum over exactly those two value heads)."""
+    T, h_qk, h_v = 4096, 16, 32
+    inp = make_bwd_inputs([T], h_qk, h_v, seed=0)
+    t = {k: to_dev(inp[k]) for k in ("qh", "kh", "v", "g", "beta", "init_state", "dy", "dS_T")}
+    dq, dk, dv, dg, dbeta, dS0 = gdn.gdn_recurrence_backward(t["qh"], t["kh"], t["v"], t["g"], t["beta"],
+                                                             t["init_state"], None, t["dy"], t["dS_T"])
+    torch.cuda.synchronize()
+    j = 15
+    rdq = np.zeros((T, 128))
+    rdk = np.zeros((T, 128))
+    for h in (30, 31):
+        r = oracle_mod.recurrence_backward(inp["qh"][:, j], inp["kh"][:, j], inp["v"][:, h], inp["g"][:, h],
+                                           inp["beta"][:, h], inp["init_state"][0, h], inp["dy"][:, h],
+                                           inp["dS_T"][0, h])
+        rdq += r["dq"]
+        rdk += r["dk"]
+        _compare(dv[:, h], r["dv"], f"dv[{h}]")
+        _compare(dg[:, h], r["dg"], f"dg[{h}]")
+        _compare(dbeta[:, h], r["dbeta"], f"dbeta[{h}]")
+        _compare(dS0[0, h], r["dS0"], f"dS0[{h}]")
+    _compare(dq[:, j], rdq, "dq")
+    _compare(dk[:, j], rdk, "dk")
