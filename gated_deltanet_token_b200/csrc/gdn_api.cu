@@ -682,8 +682,17 @@ int gdn_out_proj(const gdn_dims_t* d, int32_t hidden, const void* y, const void*
   return proj_launch(y, d->total_tokens, w_out, hidden, K, po, stream);
 }
 
+// The backward runs in fp32 throughout: the dims' dtype codes are not read.
+static int check_dims_bwd(const gdn_dims_t* d) {
+  if (!d) return GDN_ERR_NULL;
+  gdn_dims_t df = *d;
+  df.in_dtype = GDN_DTYPE_F32;
+  df.out_dtype = GDN_DTYPE_F32;
+  return check_dims(&df, false);
+}
+
 size_t gdn_recurrence_backward_workspace_size(const gdn_dims_t* d) {
-  if (check_dims(d, false) != GDN_OK) return 0;
+  if (check_dims_bwd(d) != GDN_OK) return 0;
   return bw_ws(d).total;
 }
 
@@ -691,7 +700,7 @@ int gdn_recurrence_backward(const gdn_dims_t* d, const float* qh, const float* k
                             const float* beta, const float* init_state, const int32_t* cu_seqlens, const float* dy,
                             const float* dS_final, float* dq, float* dk, float* dv, float* dg, float* dbeta,
                             float* dS_init, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
-  int rc = check_dims(d, false);
+  int rc = check_dims_bwd(d);
   if (rc != GDN_OK) return rc;
   if (!dS_init) return GDN_ERR_NULL;
   if (d->total_tokens > 0 && (!qh || !kh || !v || !g || !beta || !dy || !dq || !dk || !dv || !dg || !dbeta))

@@ -9,12 +9,12 @@
 // Row layout: eight lanes share a state row, each holding four groups of four columns
 // (columns 32 c + 4 (lane % 8) .. + 3, c = 0..3).  A warp works on four rows at once, and the
 // two dot products of a token (S'k and S'q) reduce over eight lanes in three shuffle levels --
-// for four rows together.  A warp takes its rows in groups of eight (two four-row slabs):
-// each group is copied into shared memory by asynchronous 16-byte copies two groups ahead
-// (double-buffered; the first two start before the conv prologue), so the next 4 KB of state
-// is always in flight while the current group is updated in registers; the updated rows go
-// straight back to global memory.  The dot products
-// and the row update use paired fp32 FMAs.
+// for four rows together.  A warp takes its rows in groups of four (one four-row slab): each
+// group is copied into shared memory by asynchronous 16-byte copies two groups ahead (double-
+// buffered; the first two start before the conv prologue), so the next 2 KB of state is in
+// flight while the current group is updated in registers; the updated rows go straight back
+// to global memory.  The dot products and the row update use paired fp32 FMAs, and the token
+// loop runs two tokens at a time.
 #pragma once
 #include "gdn_common.cuh"
 
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) k_decode_multi(Dims d, int K, const void*
   const int ngroups = rows_per_warp / DECM_GROUP;
   const size_t wrow0 = ((size_t)n * hv + (size_t)j * G) * D + (size_t)warp * rows_per_warp;  // first row
   float* wbuf = sbuf + warp * 2 * DECM_GROUP * D;
-  // group gi of this warp's rows into buffer gi & 1: 256 chunks of 16 bytes, 8 per lane
+  // group gi of this warp's rows into buffer gi & 1: 128 chunks of 16 bytes, 4 per lane
   auto load_group = [&](int gi) {
     const float* src = state + (wrow0 + (size_t)gi * DECM_GROUP) * D;
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf + (gi & 1) * DECM_GROUP * D));

@@ -173,3 +173,72 @@ def test_path_options_round_trip(glib):
     finally:
         glib.gdn_set_options(prev)
     assert glib.gdn_get_options() == prev
+
+
+def test_projections_reject_bad_arguments(glib):
+    L = glib.lib()
+    bf = glib.make_dims(1, 16, 16, 32, glib.GDN_DTYPE_BF16, glib.GDN_DTYPE_BF16)
+
+    def inp(dims, hidden, ptrs=None):
+        p = [FAKE] * 8 if ptrs is None else ptrs
+        return L.gdn_in_proj(None if dims is None else ctypes.byref(dims), ctypes.c_int32(hidden),
+                             *[ctypes.c_void_p(x) if x else None for x in p], None)
+
+    def outp(dims, hidden, ptrs=None):
+        p = [FAKE] * 3 if ptrs is None else ptrs
+        return L.gdn_out_proj(None if dims is None else ctypes.byref(dims), ctypes.c_int32(hidden),
+                              *[ctypes.c_void_p(x) if x else None for x in p], None)
+
+    assert inp(None, 2048) == -1
+    assert inp(glib.make_dims(1, 16, 16, 32, glib.GDN_DTYPE_F32, glib.GDN_DTYPE_BF16), 2048) == -3
+    assert inp(bf, 2000) == -2  # hidden not a multiple of the 64-wide K block
+    assert inp(bf, 0) == -2
+    bad = [FAKE] * 8
+    bad[6] = None  # a
+    assert inp(bf, 2048, bad) == -1
+    bad = [FAKE] * 8
+    bad[0] = FAKE + 8  # x misaligned
+    assert inp(bf, 2048, bad) == -4
+    assert outp(None, 2048) == -1
+    assert outp(glib.make_dims(1, 16, 16, 32, glib.GDN_DTYPE_BF16, glib.GDN_DTYPE_F32), 2048) == -3
+    assert outp(bf, 2047) == -2
+    assert outp(bf, 2048, [FAKE, None, FAKE]) == -1
+    assert outp(bf, 2048, [FAKE, FAKE, FAKE + 4]) == -4
+
+
+def test_recurrence_backward_rejects_bad_arguments(glib):
+    L = glib.lib()
+    dims = glib.make_dims(1, 100, 2, 4, glib.GDN_DTYPE_F32, glib.GDN_DTYPE_F32)
+    need = L.gdn_recurrence_backward_workspace_size(ctypes.byref(dims))
+    assert need > 0
+    # the dims' dtype codes are not read by the fp32 backward
+    odd = glib.make_dims(1, 100, 2, 4, 7, 9)
+    assert L.gdn_recurrence_backward_workspace_size(ctypes.byref(odd)) == need
+
+    def call(d, ptrs=None, ws=FAKE, nbytes=None):
+        p = [FAKE] * 15 if ptrs is None else ptrs
+        return L.gdn_recurrence_backward(None if d is None else ctypes.byref(d),
+                                         *[ctypes.c_void_p(x) if x else None for x in p],
+                                         ctypes.c_void_p(ws) if ws else None,
+                                         ctypes.c_size_t(need if nbytes is None else nbytes), None)
+
+    assert call(None) == -1
+    assert call(glib.make_dims(1, 100, 3, 4, 1, 1)) == -2  # h_v not a multiple of h_qk
+    p = [FAKE] * 15
+    p[14] = None  # dS_init
+    assert call(dims, p) == -1
+    p = [FAKE] * 15
+    p[0] = None  # qh with tokens present
+    assert call(dims, p) == -1
+    p = [FAKE] * 15
+    p[6] = None  # no cu_seqlens for two sequences
+    assert call(glib.make_dims(2, 100, 2, 4, 1, 1), p) == -1
+    p = [FAKE] * 15
+    p[3] = FAKE + 4  # g misaligned
+    assert call(dims, p) == -4
+    assert call(dims, nbytes=need - 1) == -5
+    assert call(dims, ws=0) == -5
+
+
+def test_wait_limit_rejects_zero(glib):
+    assert glib.lib().gdn_set_wait_limit_ns(ctypes.c_uint64(0)) == -2
