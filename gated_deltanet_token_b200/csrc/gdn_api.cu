@@ -60,7 +60,7 @@ bool use_tc(const gdn_dims_t* d) {
 
 // Workspace of the prefill, carved from the caller's buffer in this order.
 struct WsLayout {
-  size_t tab, seqc0, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
+  size_t tab, seqc0, order, qn, kn, vc, g, beta, gam, W, Up, mqk, yraw, total;
   size_t kq, tp, gb, vs;  // tensor-core path
   int max_chunks;
   bool tc;
@@ -81,6 +81,7 @@ WsLayout ws_layout_tc(const gdn_dims_t* d) {
   };
   L.tab = take(MC * sizeof(ChunkEntry));
   L.seqc0 = take((N + 1) * sizeof(int));
+  L.order = take(N * sizeof(int));
   L.kq = take(MC * hq * KQ_BYTES);
   L.tp = take(MC * hv * TP_BYTES);
   L.gb = take(MC * hv * GB_FLOATS * 4);
@@ -150,9 +151,9 @@ struct ProfScope {
 // Launches a tensor-core prefill kernel with programmatic dependent launch: its CTAs may
 // become resident while the previous kernel on the stream drains, and wait in
 // griddepcontrol.wait (their first statement) until it has completed, unless the options ask for plain
-// stream order (option GDN_OPT_NO_PDL).  cluster_z > 1 adds a (1, 1, cluster_z) cluster shape.
+// stream order (option GDN_OPT_NO_PDL).  cluster_x > 1 adds a (cluster_x, 1, 1) cluster shape.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_z,
+cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_x,
                        Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -166,11 +167,11 @@ cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
-  if (cluster_z > 1) {
+  if (cluster_x > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.x = (unsigned)cluster_x;
     attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = (unsigned)cluster_z;
+    attr[na].val.clusterDim.z = 1;
     ++na;
   }
   cfg.attrs = attr;
@@ -310,14 +311,14 @@ int scan_clusters_per_wave() {
   const uint64_t bit = 1ull << (dev & 63);
   if (known.load() & bit) return cached[dev & 63];
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1, 1, D / TC_NV);
+  cfg.gridDim = dim3(D / TC_NV);
   cfg.blockDim = dim3(384);
   cfg.dynamicSmemBytes = PB_TC_SMEM;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = 1;
+  attr.val.clusterDim.x = D / TC_NV;
   attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = D / TC_NV;
+  attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int n = 0;
@@ -411,7 +412,8 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
   const bool need_map = !L.tc || cu_seqlens != nullptr;
   if (need_map) {
     ProfScope p("tilemap", s);
-    k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0);
+    k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0,
+                                 L.tc ? reinterpret_cast<int*>(ws + L.order) : nullptr);
   }
   if (L.tc) {
     const ChunkEntry* tabc = need_map ? tab : nullptr;
@@ -437,12 +439,17 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     const long waves_fused = per_wave > 0 ? (units + per_wave - 1) / per_wave : 0;
     const long waves_plain = (units * (D / TC_NV) + g_num_sms - 1) / g_num_sms;
     const bool fused = per_wave > 0 && waves_fused <= waves_plain && !opt(GDN_OPT_SEPARATE_NORM);
-    const dim3 grid(d->n_seqs, d->h_v, D / TC_NV);
+    // one CTA per (sequence, value head, slice), flattened slice-fastest and sequence-slowest
+    // in the order the tile map chose (longest sequence first)
+    const long long nblk = (long long)d->n_seqs * d->h_v * (D / TC_NV);
+    if (nblk > INT32_MAX) return GDN_ERR_SHAPE;
+    const dim3 grid((unsigned)nblk);
+    const int* order = need_map ? reinterpret_cast<const int*>(ws + L.order) : nullptr;
     if (fused) {
       ProfScope p("chunk_scan_tc_norm", s);
       const uint16_t* zb = static_cast<const uint16_t*>(z);
       cudaError_t e = launch_dep(kd.out_bf16 ? k_chunkscan_tc<PB_Y_BF16> : k_chunkscan_tc<PB_Y_F32>, grid, dim3(384),
-                                 PB_TC_SMEM, s, D / TC_NV, kd, (const int*)cu_seqlens, seqc0c, (const uint8_t*)kq,
+                                 PB_TC_SMEM, s, D / TC_NV, kd, (const int*)cu_seqlens, seqc0c, order, (const uint8_t*)kq,
                                  (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs), init_state,
                                  F(L.yraw), final_state, zb, norm_w, y);
       if (e != cudaSuccess) return GDN_ERR_CUDA;
@@ -451,7 +458,7 @@ int gdn_prefill(const gdn_dims_t* d, const void* q, const void* k, const void* v
     {
       ProfScope p("chunk_scan_tc", s);
       if (launch_dep(k_chunkscan_tc<PB_Y_RAW>, grid, dim3(288), PB_TC_SMEM, s, 1, kd, (const int*)cu_seqlens, seqc0c,
-                     (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
+                     order, (const uint8_t*)kq, (const uint8_t*)tp, (const float*)F(L.gb), (const float*)F(L.vs),
                      init_state, F(L.yraw), final_state, (const uint16_t*)nullptr, (const float*)nullptr,
                      (void*)nullptr) != cudaSuccess)
         return GDN_ERR_CUDA;
@@ -722,7 +729,7 @@ int gdn_recurrence_backward(const gdn_dims_t* d, const float* qh, const float* k
   const Dims kd = kdims(d);
   if (cu_seqlens) {
     ProfScope p("tilemap", s);
-    k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0);
+    k_tilemap<<<1, 1024, 0, s>>>(cu_seqlens, d->n_seqs, d->total_tokens, L.max_chunks, tab, seqc0, nullptr);
   }
   {
     ProfScope p("recurrence_bwd", s);

@@ -789,15 +789,18 @@ enum { PB_Y_RAW = 0, PB_Y_BF16 = 1, PB_Y_F32 = 2 };
 template <int YM>
 __global__ void __launch_bounds__(YM == PB_Y_RAW ? 288 : 384, 1)
     k_chunkscan_tc(Dims d, const int* __restrict__ cu, const int* __restrict__ seq_chunk0,
-                   const uint8_t* __restrict__ kq_ws, const uint8_t* __restrict__ tp_ws,
+                   const int* __restrict__ order, const uint8_t* __restrict__ kq_ws, const uint8_t* __restrict__ tp_ws,
                    const float* __restrict__ gb_ws, const float* __restrict__ vs_ws,
                    const float* init_state, float* __restrict__ y_raw,
                    float* final_state,
                    const uint16_t* __restrict__ z, const float* __restrict__ norm_w, void* __restrict__ y) {
   constexpr int NV = TC_NV, NH = NV / 2;
   constexpr bool FUSED = YM != PB_Y_RAW;
-  const int n = blockIdx.x, h = blockIdx.y, sl = blockIdx.z, i0 = sl * NV;
-  const int hq = d.h_qk, hv = d.h_v, G = hv / hq, j = h / G;
+  // blockIdx.x = (position * h_v + h) * 4 + slice: the four slices of a head are consecutive (one
+  // cluster), and the sequences come in the tile map's order, longest first
+  const int hq = d.h_qk, hv = d.h_v, G = hv / hq;
+  const int sl = blockIdx.x % (D / NV), h = (blockIdx.x / (D / NV)) % hv, qpos = blockIdx.x / (D / NV) / hv;
+  const int n = order ? order[qpos] : qpos, i0 = sl * NV, j = h / G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, cb = ((warp >> 2) & 1) * NH;
   const bool worker = warp < 8, producer = warp == 8;

@@ -10,9 +10,14 @@ namespace gdn {
 // chunk table (one entry per 64-token chunk, chunks aligned to sequence starts) and
 // seq_chunk0[n] = index of sequence n's first chunk (seq_chunk0[N] = total chunks).
 // Runs on the device, so the host never reads cu_seqlens.
+// Also, when `order` is given, the order in which phase B takes the sequences: by chunk count,
+// longest first (ties by index), so that the longest state chains start in the first wave of
+// CTAs; beyond TILEMAP_ORDER_MAX sequences, index order.
+constexpr int TILEMAP_ORDER_MAX = 1024;
 __global__ void __launch_bounds__(1024) k_tilemap(const int* __restrict__ cu, int N, int T_tot,
                                                   int max_chunks, ChunkEntry* __restrict__ tab,
-                                                  int* __restrict__ seq_chunk0) {
+                                                  int* __restrict__ seq_chunk0, int* __restrict__ order) {
+  __shared__ int s_nc[TILEMAP_ORDER_MAX];
   __shared__ int s_warp[32];
   __shared__ int s_carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -51,6 +56,23 @@ __global__ void __launch_bounds__(1024) k_tilemap(const int* __restrict__ cu, in
   }
   if (tid == 0) seq_chunk0[N] = s_carry;
   __syncthreads();
+  if (order) {
+    if (N <= TILEMAP_ORDER_MAX) {
+      for (int n = tid; n < N; n += blockDim.x) s_nc[n] = seq_chunk0[n + 1] - seq_chunk0[n];
+      __syncthreads();
+      for (int n = tid; n < N; n += blockDim.x) {
+        const int mine = s_nc[n];
+        int rank = 0;
+        for (int m = 0; m < N; ++m) {
+          const int other = s_nc[m];
+          rank += (other > mine) || (other == mine && m < n);
+        }
+        order[rank] = n;
+      }
+    } else {
+      for (int n = tid; n < N; n += blockDim.x) order[n] = n;
+    }
+  }
   const int total = s_carry;
   for (int c = tid; c < max_chunks; c += blockDim.x) {
     ChunkEntry e{0, 0, 0, 0};
