@@ -78,6 +78,19 @@ def test_varlen_with_empty_sequences_and_alias(oracle_mod):
             assert np.array_equal(S[n], inp["init_state"][n].astype(np.float64))
 
 
+@pytest.mark.parametrize("n_seqs", [1024, 1100])
+def test_many_short_sequences_dispatch_order(oracle_mod, n_seqs):
+    """Phase B takes the sequences longest first up to 1024 of them (the tile map ranks them)
+    and in index order beyond: both orders give every sequence its own result."""
+    rng = np.random.default_rng(n_seqs)
+    lens = [int(x) for x in rng.integers(0, 70, size=n_seqs)]
+    lens[3] = 200  # a long one late in the index order
+    inp = make_inputs("varlen8_prefill_bf16", lengths=lens, h_qk=1, h_v=2)
+    ref = _oracle(oracle_mod, inp)
+    y, S = run_prefill(inp, torch.float32)
+    check_bf16(y, ref["y"], S, ref["final_state"])
+
+
 def test_varlen_equals_separate_calls():
     lens = [37, 100, 64]
     inp = make_inputs("varlen8_prefill_bf16", lengths=lens, h_qk=4, h_v=8)
