@@ -9,8 +9,11 @@
 //
 // Rows of S (value components) evolve independently in both directions; only dq, dk, dbeta and
 // dg sum over rows.  So one CTA of 256 threads serves one (sequence, value head, slice of 32
-// rows): warp w owns slice rows 4w .. 4w + 3, lane l columns 4l .. 4l + 3, 16 elements of S
-// (forward) and of D (reverse) per thread.  Row dot products are warp reductions: one group per
+// rows), and warp w owns slice rows 4w .. 4w + 3, 16 elements of S or D per thread: in the
+// recompute and the reverse, lane l holds columns 4l .. 4l + 3 of all four rows (the column
+// sums of dq and dk stay in the thread); in the two chunk-level forward passes, lane l holds
+// row l / 8 in the column groups (l % 8) + 8 m (a row product reduces over eight lanes).  Row
+// dot products are warp reductions: one group per
 // forward token (S_{t-1} k_t) and one per reverse token (D' k_t and <D', S_{t-1}> together, with
 // D' = D + dy q^T, since <dS', S_{t-1}> = <D', S_{t-1}> - sum_r de_r (S_{t-1} k_t)_r).  The
 // column sums of dq, dk and the scalars dbeta, dg are reduced over the 8 warps through shared
