@@ -102,3 +102,24 @@ def test_recurrence_backward_full_size_sampled_heads(oracle_mod):
         _compare(dS0[0, h], r["dS0"], f"dS0[{h}]")
     _compare(dq[:, j], rdq, "dq")
     _compare(dk[:, j], rdk, "dk")
+
+
+def test_recurrence_backward_extreme_gates(oracle_mod):
+    """alpha = e^g underflowing to 0 (g = -1000), beta at 0 and at 1, by value head."""
+    inp = make_bwd_inputs([70, 130], 2, 4, seed=5)
+    g = inp["g"].copy()
+    beta = inp["beta"].copy()
+    g[:, 0] = -1000.0
+    beta[:, 1] = 0.0
+    beta[:, 2] = 1.0
+    g[::3, 3] = -1000.0
+    inp = dict(inp)
+    inp["g"], inp["beta"] = g.astype(np.float32), beta.astype(np.float32)
+    ref = _oracle_grads(oracle_mod, inp, 2, 4)
+    t = {k: to_dev(inp[k]) for k in ("qh", "kh", "v", "g", "beta", "init_state", "dy", "dS_T")}
+    cu = to_dev(inp["cu_seqlens"].astype(np.int32))
+    dq, dk, dv, dg, dbeta, dS0 = gdn.gdn_recurrence_backward(t["qh"], t["kh"], t["v"], t["g"], t["beta"],
+                                                             t["init_state"], cu, t["dy"], t["dS_T"])
+    torch.cuda.synchronize()
+    for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (dg, "dg"), (dbeta, "dbeta"), (dS0, "dS0")):
+        _compare(got, ref[name], name)

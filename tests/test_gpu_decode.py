@@ -259,3 +259,28 @@ def _check_multi(oracle_mod, inp, K, dtype):
     exp = bf16_from_f64(o["conv_state"]) if dtype == "bf16" else o["conv_state"].astype(np.float32)
     assert np.array_equal(got, exp)  # the raw history, bit-exact
 
+
+
+def _extreme_decode_gates(inp):
+    """Gates at the ends of their ranges, by value-head group: A_log = log 1e6 (e^g underflows
+    to 0), b = +30 (beta = 1), b = -30 (beta ~ 1e-13), and a = +20 on the last group."""
+    h_v = inp["A_log"].shape[0]
+    q4 = max(1, h_v // 4)
+    out = dict(inp)
+    A_log = inp["A_log"].copy()
+    A_log[:q4] = np.log(1e6)
+    a = inp["a"].copy()
+    b = inp["b"].copy()
+    b[..., q4:2 * q4] = 30.0
+    b[..., 2 * q4:3 * q4] = -30.0
+    a[..., 3 * q4:] = 20.0
+    out["A_log"], out["a"], out["b"] = A_log.astype(np.float32), a.astype(np.float32), b.astype(np.float32)
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_multi_extreme_gates(oracle_mod, dtype):
+    """The multi-token decode with the decay underflowing to zero, beta at 0 and 1 and a strong
+    single-token decay, against the oracle's successive steps (the one-token decode is the same
+    kernel at K = 1)."""
+    _check_multi(oracle_mod, _extreme_decode_gates(_multi_inputs(4, N=3, dtype=dtype, h_qk=2, h_v=8)), 4, dtype)
