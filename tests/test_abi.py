@@ -242,3 +242,15 @@ def test_recurrence_backward_rejects_bad_arguments(glib):
 
 def test_wait_limit_rejects_zero(glib):
     assert glib.lib().gdn_set_wait_limit_ns(ctypes.c_uint64(0)) == -2
+
+
+def test_noalloc_token_limits_match_the_header(glib):
+    """gdn.h states what fits the allocation-free prefill's 64 MiB scratch at the model shape
+    (one sequence, 16 QK / 32 value heads): 960 tokens with bf16 inputs, 740 with fp32."""
+    cap = 64 << 20
+
+    def fits(T, dt):
+        return glib.gdn_prefill_workspace_size(glib.make_dims(1, T, 16, 32, dt, glib.GDN_DTYPE_F32)) <= cap
+
+    assert fits(960, glib.GDN_DTYPE_BF16) and not fits(961, glib.GDN_DTYPE_BF16)
+    assert fits(740, glib.GDN_DTYPE_F32) and not fits(741, glib.GDN_DTYPE_F32)
